@@ -1,0 +1,234 @@
+/*
+ * strata_moe.h -- C ABI of libstrata_moe.so, the B200 (sm_100a) routed-expert
+ * FFN layer of a very sparse mixture-of-experts model.
+ *
+ * The layer (Strata walk-through, blog.5616760.com/0039, section 5 "MoE 的本质",
+ * flowchart "Router -> Top-10 -> softmax 加权合并"): a router scores every
+ * token against all experts, the k best experts are chosen, each chosen
+ * expert's SwiGLU FFN runs on the token, and the expert outputs are summed
+ * with the routing softmax weights.  The pages' geometry is hidden 2560, 512
+ * experts per layer, expert width 640, top-10 (lcz.me/topic/2153 section 3.2;
+ * ai-coding.wiselychen.com Strata review, "30 秒定位" table); every size here
+ * is a runtime argument.
+ *
+ * Call order for one layer (all on one CUDA stream):
+ *   moe_rmsnorm -> moe_router_topk -> moe_bucket -> moe_experts
+ *   [-> moe_shared_expert] -> moe_combine
+ * or the composite moe_layer_forward, which runs exactly that sequence.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer owned by the caller unless the
+ *     argument says otherwise.  The library never allocates, frees or
+ *     synchronises device memory (the one exception, strata_read_status, says
+ *     so).  Scratch memory comes from a caller-provided `workspace` whose size
+ *     the matching *_workspace_size() query returns; its contents need not be
+ *     initialised and are clobbered.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous: they enqueue kernels and return.
+ *   - Return value: a strata_status.  Arguments are validated on the host
+ *     before anything is enqueued; on STRATA_EINVAL / STRATA_EUNSUPPORTED
+ *     nothing has been enqueued and no output was touched.  STRATA_ECUDA
+ *     means a launch failed (cudaGetLastError), outputs are undefined.
+ *   - `dev_status` (device int32, may be NULL where stated) is a sticky error
+ *     word: kernels never trap; on a device-detected problem (a bounded wait
+ *     that ran out, an index out of range) they OR a STRATA_DEV_* bit into it
+ *     and skip the offending access.  Zero it once; read it with
+ *     strata_read_status.
+ *   - bf16 and fp16 values travel as uint16_t bit patterns.
+ *   - Shapes: T tokens, H hidden, E experts, I expert width, k experts per
+ *     token, P = T*k (token, slot) pairs; pair p = t*k + j.
+ */
+#ifndef STRATA_MOE_H
+#define STRATA_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---------------------------------------------------------------- status */
+typedef enum strata_status {
+  STRATA_OK = 0,
+  STRATA_EINVAL = 1,       /* bad shape, NULL pointer, misalignment, k > E, K % 32 != 0 */
+  STRATA_ECUDA = 2,        /* a CUDA launch or API call failed */
+  STRATA_EUNSUPPORTED = 3, /* valid but outside what the kernels implement */
+  STRATA_ETIMEOUT = 4,     /* device-reported: a bounded wait ran out */
+  STRATA_EBOUNDS = 5       /* device-reported: an index was out of range */
+} strata_status;
+
+/* Bits a kernel ORs into *dev_status. */
+#define STRATA_DEV_TIMEOUT 0x1
+#define STRATA_DEV_BOUNDS 0x2
+
+/* ---------------------------------------------------------------- formats
+ * Block-quantised expert weights.  Each weight matrix is stored as
+ * output-feature rows with the K (input) dimension contiguous; blocks are 32
+ * consecutive K elements of one row with one IEEE fp16 scale d per block.
+ *
+ *   STRATA_FMT_Q2_32   2-bit code c in 0..3; w = d * (c - 1.5).
+ *                      Codes plane uint8 [N][K/4]: element k is byte k/4,
+ *                      bits 2*(k%4) .. 2*(k%4)+1 (least significant first).
+ *                      2.5 bits per weight.
+ *   STRATA_FMT_Q4CB_32 4-bit code c in 0..15; w = d * KV[c] with the 16-entry
+ *                      non-linear codebook
+ *                      KV = {-127,-104,-83,-65,-49,-35,-22,-10,
+ *                               1,  13, 25, 38, 53, 69, 89,113}
+ *                      (the IQ4_NL codebook; the Strata walk-through names
+ *                      IQ4_NL in section 13).  Codes plane uint8 [N][K/2]:
+ *                      element k is byte k/2, low nibble for even k, high
+ *                      nibble for odd k.  4.5 bits per weight.
+ *   Scales plane (both formats): fp16 [N][K/32], little-endian.
+ *
+ * One expert blob, in this order, every plane starting on a 256-byte boundary:
+ *   gate codes [I][H..] | gate scales | up codes [I][H..] | up scales |
+ *   down codes [H][I..] | down scales
+ * strata_expert_bytes() gives its size: 1,536,000 B for Q2_32 at H=2560,
+ * I=640 (the pages' own 2.25-bit Q2_0 blob is 1,382,400 B, lcz.me/topic/2153
+ * section 3.4; its bit layout is not on the pages), 2,764,800 B for Q4CB_32
+ * at H=2560, I=640 and 14,155,776 B at H=4096, I=2048. */
+#define STRATA_FMT_Q2_32 1
+#define STRATA_FMT_Q4CB_32 2
+
+/* Element types of expert outputs y. */
+#define STRATA_DTYPE_F32 0
+#define STRATA_DTYPE_F16 1
+
+/* Largest T served by the weight-streaming decode path of moe_experts;
+ * larger T takes the tensor-core grouped-GEMM path. */
+#define STRATA_DECODE_MAX_T 16
+
+typedef struct strata_qweights {
+  int32_t fmt;            /* STRATA_FMT_* */
+  int32_t num_experts;    /* E (1 for a shared expert) */
+  int32_t hidden;         /* H, multiple of 128 */
+  int32_t inter;          /* I, multiple of 128 */
+  const void* base;       /* device; expert e starts at base + e*expert_stride; 256-byte aligned */
+  uint64_t expert_stride; /* bytes; multiple of 256 and >= strata_expert_bytes(fmt, H, I) */
+} strata_qweights;
+
+/* ---------------------------------------------------------------- helpers */
+int32_t strata_abi_version(void);
+const char* strata_status_string(int32_t status);
+/* Blob size of one expert; 0 for an unknown format or H, I not multiples of 32. */
+uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t inter);
+/* Reads *dev_status (device) into host memory: enqueues a copy on `stream` and
+ * SYNCHRONISES that stream.  Returns STRATA_OK, STRATA_ETIMEOUT,
+ * STRATA_EBOUNDS (the first set bit, timeout first) or STRATA_ECUDA. */
+int32_t strata_read_status(const int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------- calls */
+
+/* RMSNorm with unit gain, the layer's input normalisation:
+ *   hidden[t,h] = bf16_rne( x[t,h] / sqrt(mean_h x[t,h]^2 + eps) ).
+ * x fp32 [T,H] row-major; hidden bf16 [T,H] row-major.  T >= 0 (T == 0 is a
+ * no-op), H in 32..16384, multiple of 8.  x and hidden 16-byte aligned. */
+int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps,
+                    uint16_t* hidden, void* stream);
+
+/* Router: logits[t,e] = sum_h hidden[t,h]*w_router[h,e] (fp32 accumulation)
+ * + bias[e]; p = softmax over all E; the k largest logits are chosen (ties to
+ * the lower expert index) and listed in descending-logit order; the weights
+ * are renormalised over the chosen k: w_j = p_j / sum_chosen p.
+ * (Strata walk-through section 5 flowchart: the router scores each token,
+ * top-10 are selected, outputs merged with softmax weights; the Strata review,
+ * "success idea one" step 1: the GPU runs the router.)
+ *   hidden    bf16 [T,H];  w_router bf16 [H,E] row-major;  bias fp32 [E] or NULL
+ *   topk_ids  int32 [T,k] out;  topk_w fp32 [T,k] out
+ *   logits_opt fp32 [T,E] out, or NULL
+ * Limits: 1 <= k <= min(E, 32); E even, 2..1024; H multiple of 64. */
+uint64_t moe_router_topk_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
+int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router,
+                        const float* bias, int32_t T, int32_t H, int32_t E,
+                        int32_t k, int32_t* topk_ids, float* topk_w,
+                        float* logits_opt, void* workspace, uint64_t ws_bytes,
+                        int32_t* dev_status, void* stream);
+
+/* Bucketing of the P = T*k (token, slot) pairs by expert: a deterministic
+ * counting sort, stable in pair order (the pages do not name this step; it is
+ * what lets one prepared expert weight serve all of its tokens, Strata
+ * memory-tier article devotd.net, "读取提示与写出回答时").
+ *   counts  int32 [E]     pairs routed to each expert
+ *   offsets int32 [E+1]   exclusive prefix sum of counts, offsets[E] = P
+ *   perm    int32 [P]     perm[sorted position] = pair p
+ *   inv     int32 [P]     inv[p] = sorted position
+ *   active  int32 [E+1]   active[0] = U, the number of experts with
+ *                         counts > 0; active[1..U] their ids, ascending
+ * A topk id outside [0,E) sets STRATA_DEV_BOUNDS and that pair is dropped. */
+uint64_t moe_bucket_workspace_size(int32_t T, int32_t k, int32_t E);
+int32_t moe_bucket(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+                   int32_t* counts, int32_t* offsets, int32_t* perm,
+                   int32_t* inv, int32_t* active, void* workspace,
+                   uint64_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* Routed experts: for every sorted position s with pair p = perm[s], token
+ * t = p / k, expert e (offsets[e] <= s < offsets[e+1]):
+ *   g = W_gate[e] . hidden[t],  u = W_up[e] . hidden[t],
+ *   h = silu(g) * u,            y[s] = W_down[e] . h
+ * with fp32 accumulation (the SwiGLU expert FFN; the pages' experts are run by
+ * the GPU when resident, Strata review "success idea one" step 2).
+ *   y: [P,H] in SORTED order.  T <= STRATA_DECODE_MAX_T: fp32 (decode path,
+ *      weight-streaming dequant-GEMV).  T > STRATA_DECODE_MAX_T: fp16 (prefill
+ *      path, tcgen05 grouped GEMM over dequantised fp16 tiles).
+ *   offsets/perm/active: as written by moe_bucket for the same (T, k, E).
+ * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket. */
+uint64_t moe_experts_workspace_size(const strata_qweights* w, int32_t T, int32_t k);
+int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
+                    const int32_t* offsets, const int32_t* perm,
+                    const int32_t* active, int32_t T, int32_t k, void* y,
+                    void* workspace, uint64_t ws_bytes, int32_t* dev_status,
+                    void* stream);
+
+/* Shared expert: the same SwiGLU FFN with one always-on expert (w->num_experts
+ * == 1) applied to every token, y[t] = FFN(hidden[t]); y [T,H] in token order,
+ * fp32 for T <= STRATA_DECODE_MAX_T, fp16 otherwise.  The shared expert is
+ * resident and read for every token (Strata review, Table 1 of the paper it
+ * quotes; devotd.net memory-tier article, "各层内存承担的数据"). */
+uint64_t moe_shared_expert_workspace_size(const strata_qweights* w, int32_t T);
+int32_t moe_shared_expert(const uint16_t* hidden, const strata_qweights* w,
+                          int32_t T, void* y, void* workspace, uint64_t ws_bytes,
+                          int32_t* dev_status, void* stream);
+
+/* Weighted combine ("softmax 加权合并", Strata walk-through section 5), in a
+ * fixed order so the result is deterministic:
+ *   acc = sum_{j=0..k-1} topk_w[t,j] * y[inv[t*k+j]]   (fp32, j ascending)
+ *   acc += shared_y[t]                                 (if shared_y != NULL)
+ *   out[t] = bf16_rne(acc);  residual_out[t] = residual[t] + acc  (if given)
+ *   y        [P,H] sorted order, y_dtype STRATA_DTYPE_F32 or _F16
+ *   shared_y [T,H] or NULL, shared_dtype as y_dtype
+ *   residual fp32 [T,H] or NULL (required if residual_out != NULL)
+ *   out      bf16 [T,H];  residual_out fp32 [T,H] or NULL (may alias residual)
+ * H multiple of 8; all row pointers 16-byte aligned. */
+int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* inv,
+                    const float* topk_w, const void* shared_y,
+                    int32_t shared_dtype, const float* residual, int32_t T,
+                    int32_t k, int32_t H, uint16_t* out, float* residual_out,
+                    int32_t* dev_status, void* stream);
+
+/* The whole layer in one call: moe_rmsnorm(x) -> moe_router_topk ->
+ * moe_bucket -> moe_experts -> moe_shared_expert (if `shared` != NULL) ->
+ * moe_combine(residual = x).  Every intermediate lives in `workspace`.
+ *   x            fp32 [T,H]  layer input (the residual stream)
+ *   w_router     bf16 [H,E]; bias fp32 [E] or NULL
+ *   w            routed experts (num_experts = E); shared: NULL or one expert
+ *   out          bf16 [T,H]  the MoE output, before the residual add
+ *   residual_out fp32 [T,H] or NULL: x + MoE output (may alias x)
+ *   topk_ids_opt int32 [T,k] / topk_w_opt fp32 [T,k]: copies of the routing,
+ *                or NULL */
+uint64_t moe_layer_workspace_size(int32_t T, int32_t E, int32_t k,
+                                  const strata_qweights* w,
+                                  const strata_qweights* shared);
+int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router,
+                          const float* bias, int32_t E, int32_t k,
+                          const strata_qweights* w, const strata_qweights* shared,
+                          float eps, uint16_t* out, float* residual_out,
+                          int32_t* topk_ids_opt, float* topk_w_opt,
+                          void* workspace, uint64_t ws_bytes,
+                          int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STRATA_MOE_H */
