@@ -1,0 +1,129 @@
+// combine.cu -- RMSNorm and the fixed-order weighted combine.
+#include "decode.cuh"
+
+namespace strata {
+
+// hidden[t,h] = bf16_rne(x[t,h] / sqrt(mean_h x^2 + eps)), one CTA per token.
+__global__ void __launch_bounds__(256)
+rmsnorm_kernel(const float* __restrict__ x, int H, float eps, uint16_t* __restrict__ out) {
+  __shared__ float red[8];
+  const float* xr = x + (size_t)blockIdx.x * H;
+  float ss = 0.f;
+  for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + h);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tot += red[i];
+  const float inv = 1.0f / sqrtf(tot / (float)H + eps);
+  uint16_t* orow = out + (size_t)blockIdx.x * H;
+  for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + h);
+    const uint32_t lo = float_to_bf16_bits(v.x * inv) | (uint32_t(float_to_bf16_bits(v.y * inv)) << 16);
+    const uint32_t hi = float_to_bf16_bits(v.z * inv) | (uint32_t(float_to_bf16_bits(v.w * inv)) << 16);
+    *reinterpret_cast<uint2*>(orow + h) = make_uint2(lo, hi);
+  }
+}
+
+STRATA_DEVFN void load8(const void* base, int dtype, size_t idx, float (&v)[8]) {
+  if (dtype == STRATA_DTYPE_F32) {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    const float4 b =
+        *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(base) + idx);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const __half2 h = u32_as_h2(w[i]);
+      v[2 * i] = __low2float(h);
+      v[2 * i + 1] = __high2float(h);
+    }
+  }
+}
+
+// acc = sum_j w_j * y[inv[t*k+j]] (j ascending, separate multiply and add,
+// no contraction), + shared_y; out = bf16(acc); residual_out = residual + acc.
+__global__ void __launch_bounds__(256)
+combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restrict__ inv,
+               const float* __restrict__ w, const void* __restrict__ shared_y, int shared_dtype,
+               const float* __restrict__ residual, int k, int H, uint16_t* __restrict__ out,
+               float* __restrict__ residual_out, int32_t* status) {
+  const int t = blockIdx.x;
+  __shared__ int s_pos[32];
+  __shared__ float s_w[32];
+  if (threadIdx.x < k) {
+    const int p = t * k + threadIdx.x;
+    s_pos[threadIdx.x] = inv[p];
+    s_w[threadIdx.x] = w[p];
+  }
+  __syncthreads();
+  for (int h = threadIdx.x * 8; h < H; h += blockDim.x * 8) {
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int pos = s_pos[j];
+      if (pos < 0) {
+        if (h == threadIdx.x * 8) dev_flag(status, STRATA_DEV_BOUNDS);
+        continue;
+      }
+      float v[8];
+      load8(y, y_dtype, (size_t)pos * H + h, v);
+      const float wj = s_w[j];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, v[i]));
+    }
+    if (shared_y) {
+      float v[8];
+      load8(shared_y, shared_dtype, (size_t)t * H + h, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      o[i] = float_to_bf16_bits(acc[2 * i]) | (uint32_t(float_to_bf16_bits(acc[2 * i + 1])) << 16);
+    *reinterpret_cast<uint4*>(out + (size_t)t * H + h) = make_uint4(o[0], o[1], o[2], o[3]);
+    if (residual_out) {
+      const float* r = residual + (size_t)t * H + h;
+      const float4 r0 = *reinterpret_cast<const float4*>(r);
+      const float4 r1 = *reinterpret_cast<const float4*>(r + 4);
+      float4 o0 = make_float4(__fadd_rn(r0.x, acc[0]), __fadd_rn(r0.y, acc[1]),
+                              __fadd_rn(r0.z, acc[2]), __fadd_rn(r0.w, acc[3]));
+      float4 o1 = make_float4(__fadd_rn(r1.x, acc[4]), __fadd_rn(r1.y, acc[5]),
+                              __fadd_rn(r1.z, acc[6]), __fadd_rn(r1.w, acc[7]));
+      float* ro = residual_out + (size_t)t * H + h;
+      *reinterpret_cast<float4*>(ro) = o0;
+      *reinterpret_cast<float4*>(ro + 4) = o1;
+    }
+  }
+}
+
+cudaError_t launch_rmsnorm(const float* x, int T, int H, float eps, uint16_t* out,
+                           cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  rmsnorm_kernel<<<T, 256, 0, st>>>(x, H, eps, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y, int y_dtype, const int32_t* inv, const float* w,
+                           const void* shared_y, int shared_dtype, const float* residual,
+                           int T, int k, int H, uint16_t* out, float* residual_out,
+                           int32_t* status, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  int threads = (H / 8 + 31) / 32 * 32;
+  if (threads > 256) threads = 256;
+  if (threads < 32) threads = 32;
+  combine_kernel<<<T, threads, 0, st>>>(y, y_dtype, inv, w, shared_y, shared_dtype, residual, k,
+                                         H, out, residual_out, status);
+  return cudaGetLastError();
+}
+
+}  // namespace strata

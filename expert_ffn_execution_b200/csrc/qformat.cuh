@@ -1,0 +1,123 @@
+// qformat.cuh -- block-quantised expert weight formats (device side).
+//
+// Storage (include/strata_moe.h): per matrix, output-feature rows with K
+// contiguous; a codes plane (Q2_32: K/4 bytes per row, element k at byte k/4,
+// bits 2(k%4)..; Q4CB_32: K/2 bytes per row, low nibble = even k) and an fp16
+// scales plane [rows][K/32].  Blob = gate codes|scales, up codes|scales, down
+// codes|scales, each plane on a 256-byte boundary.
+//
+// Register-level decode for the mma.sync decode path.  A "group" is 16
+// consecutive K elements of one row.  Decoding a group yields eight fp16x2
+// registers R[0..7]; R[i] holds the elements (pi(2i), pi(2i+1)) of the group,
+// where pi is a fixed permutation chosen per format to minimise instructions:
+//   Q2_32  : pi(2i) = i, pi(2i+1) = i + 8  (pairs (0,8), (1,9), ...)
+//   Q4CB_32: identity                      (pairs (0,1), (2,3), ...)
+// The activation operand is stored with the same permutation, so the dot
+// product over a group is unchanged.
+#pragma once
+
+#include "common.cuh"
+
+namespace strata {
+
+struct Planes {
+  uint64_t codes[3];   // gate, up, down
+  uint64_t scales[3];
+};
+
+__host__ __device__ inline uint64_t round_up_256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+__host__ __device__ inline uint64_t codes_row_bytes(int fmt, int K) {
+  return fmt == STRATA_FMT_Q2_32 ? uint64_t(K) / 4 : uint64_t(K) / 2;
+}
+
+__host__ __device__ inline Planes plane_offsets(int fmt, int H, int I, uint64_t* total = nullptr) {
+  Planes p;
+  uint64_t off = 0;
+  for (int m = 0; m < 3; ++m) {
+    int rows = (m == 2) ? H : I;
+    int K = (m == 2) ? I : H;
+    p.codes[m] = off;
+    off = round_up_256(off + uint64_t(rows) * codes_row_bytes(fmt, K));
+    p.scales[m] = off;
+    off = round_up_256(off + uint64_t(rows) * uint64_t(K / 32) * 2);
+  }
+  if (total) *total = off;
+  return p;
+}
+
+// Position of group element e (0..15) in the permuted operand layout.
+template <int FMT>
+__host__ __device__ inline int group_slot(int e) {
+  if (FMT == STRATA_FMT_Q2_32) return e < 8 ? 2 * e : 2 * (e - 8) + 1;
+  return e;
+}
+
+// ---------------------------------------------------------------- Q2_32
+// Element j of the 32-bit word sits at bits 2j.  Putting a code at mantissa
+// bit p of an fp16 whose exponent gives that bit unit weight yields
+// M_p + c exactly (M_p = 2^(10-p)); subtracting M_p + 1.5 gives c - 1.5
+// exactly; one multiply by the block scale rounds once to the nearest fp16.
+STRATA_DEVFN void dq_q2_group(uint32_t w, __half2 d2, uint32_t (&R)[8]) {
+  const uint32_t m2 = 0x000C000Cu, m4 = 0x00300030u, m6 = 0x00C000C0u, m8 = 0x03000300u;
+  const uint32_t M2 = 0x5C005C00u, M4 = 0x54005400u, M6 = 0x4C004C00u, M8 = 0x44004400u;
+  const __half2 S2 = u32_as_h2(0x5C065C06u);  // 257.5
+  const __half2 S4 = u32_as_h2(0x54185418u);  // 65.5
+  const __half2 S6 = u32_as_h2(0x4C604C60u);  // 17.5
+  const __half2 S8 = u32_as_h2(0x45804580u);  // 5.5
+  const uint32_t wl = w << 2;   // element 0 -> bit 2, element 8 -> bit 18
+  const uint32_t wr = w >> 8;   // elements 5,6,7 -> bits 2,4,6; 13,14,15 -> 18,20,22
+  R[0] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wl & m2) | M2), S2), d2));
+  R[1] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m2) | M2), S2), d2));
+  R[2] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m4) | M4), S4), d2));
+  R[3] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m6) | M6), S6), d2));
+  R[4] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m8) | M8), S8), d2));
+  R[5] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wr & m2) | M2), S2), d2));
+  R[6] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wr & m4) | M4), S4), d2));
+  R[7] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wr & m6) | M6), S6), d2));
+}
+
+// ---------------------------------------------------------------- Q4CB_32
+// Codebook stored as bytes KV[c] + 128, four entries per register.
+struct Q4Table {
+  uint32_t t0, t1, t2, t3;
+};
+STRATA_DEVFN Q4Table q4_table() {
+  // KV + 128 = 1,24,45,63, 79,93,106,118, 129,141,153,166, 181,197,217,241
+  Q4Table t;
+  t.t0 = 0x3F2D1801u;
+  t.t1 = 0x766A5D4Fu;
+  t.t2 = 0xA6998D81u;
+  t.t3 = 0xF1D9C5B5u;
+  return t;
+}
+
+// Four codes (nibbles of the low 16 bits of q) -> four bytes KV[c] + 128.
+// A byte permute over the low and the high half of the table picks both
+// candidates; a third permute keeps the one bit 3 of each code selects.
+STRATA_DEVFN uint32_t q4_lookup4(uint32_t q, const Q4Table& T) {
+  const uint32_t s = q & 0x7777u;
+  const uint32_t lo = __byte_perm(T.t0, T.t1, s);
+  const uint32_t hi = __byte_perm(T.t2, T.t3, s);
+  const uint32_t sel = ((q >> 1) & 0x4444u) | 0x3210u;
+  return __byte_perm(lo, hi, sel);
+}
+
+// One 16-element group from two code words (elements 0..7 and 8..15) into
+// R[i] = (element 2i, element 2i+1).  Bytes u = KV + 128 become fp16
+// 1024 + u exactly (byte under the exponent byte 0x64); subtracting 1152
+// gives KV exactly; one multiply by the block scale rounds once.
+STRATA_DEVFN void dq_q4_group(uint32_t w0, uint32_t w1, __half2 d2, const Q4Table& T,
+                              uint32_t (&R)[8]) {
+  const __half2 C = u32_as_h2(0x64806480u);  // 1152
+  const uint32_t u[4] = {q4_lookup4(w0, T), q4_lookup4(w0 >> 16, T), q4_lookup4(w1, T),
+                         q4_lookup4(w1 >> 16, T)};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    R[2 * i] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(__byte_perm(u[i], 0x64646464u, 0x4140u)), C), d2));
+    R[2 * i + 1] =
+        h2_as_u32(__hmul2(__hsub2(u32_as_h2(__byte_perm(u[i], 0x64646464u, 0x4342u)), C), d2));
+  }
+}
+
+}  // namespace strata

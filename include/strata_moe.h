@@ -44,6 +44,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#if defined(__GNUC__)
+#define STRATA_API __attribute__((visibility("default")))
+#else
+#define STRATA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -109,14 +115,14 @@ typedef struct strata_qweights {
 } strata_qweights;
 
 /* ---------------------------------------------------------------- helpers */
-int32_t strata_abi_version(void);
-const char* strata_status_string(int32_t status);
+STRATA_API int32_t strata_abi_version(void);
+STRATA_API const char* strata_status_string(int32_t status);
 /* Blob size of one expert; 0 for an unknown format or H, I not multiples of 32. */
-uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t inter);
+STRATA_API uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t inter);
 /* Reads *dev_status (device) into host memory: enqueues a copy on `stream` and
  * SYNCHRONISES that stream.  Returns STRATA_OK, STRATA_ETIMEOUT,
  * STRATA_EBOUNDS (the first set bit, timeout first) or STRATA_ECUDA. */
-int32_t strata_read_status(const int32_t* dev_status, void* stream);
+STRATA_API int32_t strata_read_status(const int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------- calls */
 
@@ -124,7 +130,7 @@ int32_t strata_read_status(const int32_t* dev_status, void* stream);
  *   hidden[t,h] = bf16_rne( x[t,h] / sqrt(mean_h x[t,h]^2 + eps) ).
  * x fp32 [T,H] row-major; hidden bf16 [T,H] row-major.  T >= 0 (T == 0 is a
  * no-op), H in 32..16384, multiple of 8.  x and hidden 16-byte aligned. */
-int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps,
+STRATA_API int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps,
                     uint16_t* hidden, void* stream);
 
 /* Router: logits[t,e] = sum_h hidden[t,h]*w_router[h,e] (fp32 accumulation)
@@ -138,8 +144,8 @@ int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps,
  *   topk_ids  int32 [T,k] out;  topk_w fp32 [T,k] out
  *   logits_opt fp32 [T,E] out, or NULL
  * Limits: 1 <= k <= min(E, 32); E even, 2..1024; H multiple of 64. */
-uint64_t moe_router_topk_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
-int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router,
+STRATA_API uint64_t moe_router_topk_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
+STRATA_API int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router,
                         const float* bias, int32_t T, int32_t H, int32_t E,
                         int32_t k, int32_t* topk_ids, float* topk_w,
                         float* logits_opt, void* workspace, uint64_t ws_bytes,
@@ -156,8 +162,8 @@ int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router,
  *   active  int32 [E+1]   active[0] = U, the number of experts with
  *                         counts > 0; active[1..U] their ids, ascending
  * A topk id outside [0,E) sets STRATA_DEV_BOUNDS and that pair is dropped. */
-uint64_t moe_bucket_workspace_size(int32_t T, int32_t k, int32_t E);
-int32_t moe_bucket(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
+STRATA_API uint64_t moe_bucket_workspace_size(int32_t T, int32_t k, int32_t E);
+STRATA_API int32_t moe_bucket(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
                    int32_t* counts, int32_t* offsets, int32_t* perm,
                    int32_t* inv, int32_t* active, void* workspace,
                    uint64_t ws_bytes, int32_t* dev_status, void* stream);
@@ -173,8 +179,8 @@ int32_t moe_bucket(const int32_t* topk_ids, int32_t T, int32_t k, int32_t E,
  *      path, tcgen05 grouped GEMM over dequantised fp16 tiles).
  *   offsets/perm/active: as written by moe_bucket for the same (T, k, E).
  * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket. */
-uint64_t moe_experts_workspace_size(const strata_qweights* w, int32_t T, int32_t k);
-int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
+STRATA_API uint64_t moe_experts_workspace_size(const strata_qweights* w, int32_t T, int32_t k);
+STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
                     const int32_t* offsets, const int32_t* perm,
                     const int32_t* active, int32_t T, int32_t k, void* y,
                     void* workspace, uint64_t ws_bytes, int32_t* dev_status,
@@ -185,8 +191,8 @@ int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
  * fp32 for T <= STRATA_DECODE_MAX_T, fp16 otherwise.  The shared expert is
  * resident and read for every token (Strata review, Table 1 of the paper it
  * quotes; devotd.net memory-tier article, "各层内存承担的数据"). */
-uint64_t moe_shared_expert_workspace_size(const strata_qweights* w, int32_t T);
-int32_t moe_shared_expert(const uint16_t* hidden, const strata_qweights* w,
+STRATA_API uint64_t moe_shared_expert_workspace_size(const strata_qweights* w, int32_t T);
+STRATA_API int32_t moe_shared_expert(const uint16_t* hidden, const strata_qweights* w,
                           int32_t T, void* y, void* workspace, uint64_t ws_bytes,
                           int32_t* dev_status, void* stream);
 
@@ -200,7 +206,7 @@ int32_t moe_shared_expert(const uint16_t* hidden, const strata_qweights* w,
  *   residual fp32 [T,H] or NULL (required if residual_out != NULL)
  *   out      bf16 [T,H];  residual_out fp32 [T,H] or NULL (may alias residual)
  * H multiple of 8; all row pointers 16-byte aligned. */
-int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* inv,
+STRATA_API int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* inv,
                     const float* topk_w, const void* shared_y,
                     int32_t shared_dtype, const float* residual, int32_t T,
                     int32_t k, int32_t H, uint16_t* out, float* residual_out,
@@ -216,10 +222,10 @@ int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* inv,
  *   residual_out fp32 [T,H] or NULL: x + MoE output (may alias x)
  *   topk_ids_opt int32 [T,k] / topk_w_opt fp32 [T,k]: copies of the routing,
  *                or NULL */
-uint64_t moe_layer_workspace_size(int32_t T, int32_t E, int32_t k,
+STRATA_API uint64_t moe_layer_workspace_size(int32_t T, int32_t E, int32_t k,
                                   const strata_qweights* w,
                                   const strata_qweights* shared);
-int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router,
+STRATA_API int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router,
                           const float* bias, int32_t E, int32_t k,
                           const strata_qweights* w, const strata_qweights* shared,
                           float eps, uint16_t* out, float* residual_out,

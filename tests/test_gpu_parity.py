@@ -1,0 +1,235 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Inputs are the seeded synthetic workloads of moe_inputs, generated on the
+device; the oracle receives the same bytes (hidden rows, router weights, the
+blobs of the experts the routing touched).  Bars:
+  - RMSNorm: within one bf16 ulp of the oracle.
+  - Router: top-k ids exact except listed near-ties (oracle logits of two
+    adjacent ranks within 1e-5 relative); weights within 1e-5.
+  - Bucket: counts, offsets, perm, inv bit-exact vs the oracle on the GPU's ids.
+  - Combine: bit-exact vs the oracle given the GPU's expert outputs.
+  - Expert outputs and the layer output: per-token relative L2 <= 5e-3 vs the
+    oracle run with the GPU's ids (teacher forcing).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import expert_ffn_execution_b200 as sm  # noqa: E402
+import moe_inputs as mi  # noqa: E402
+import oracle  # noqa: E402
+from tests.harness import OUT_REL_L2, TOPK_W_ATOL, check_routing, rel_l2_rows  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def ws(nbytes):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=DEV)
+
+
+class Run:
+    """One layer through the individual C-ABI calls, all intermediates kept."""
+
+    def __init__(self, config, T, layer=0, E=None, x=None):
+        self.c = mi.CONFIGS[config]
+        self.inp = mi.make_layer(config, T, layer=layer, device=DEV, E=E)
+        if x is not None:
+            self.inp.x = x
+        self.T, self.H, self.I, self.k = T, self.c.H, self.c.I, self.c.k
+        self.E = self.inp.w_router.shape[1]
+        self.status = torch.zeros(1, dtype=torch.int32, device=DEV)
+        self.qw = sm.qweights(self.c.fmt, self.E, self.H, self.I, self.inp.experts,
+                              self.inp.experts.stride(0))
+        self.sqw = None
+        if self.inp.shared is not None:
+            self.sqw = sm.qweights(self.c.shared_fmt, 1, self.H, self.I, self.inp.shared,
+                                   self.inp.shared.stride(0))
+
+    def run(self):
+        T, H, E, k, I = self.T, self.H, self.E, self.k, self.I
+        st = self.status
+        self.hidden = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+        sm.moe_rmsnorm(self.inp.x, T, H, self.c.eps, self.hidden)
+        self.ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+        self.w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+        self.logits = torch.empty(T, E, dtype=torch.float32, device=DEV)
+        rw = ws(sm.moe_router_topk_workspace_size(T, H, E, k))
+        sm.moe_router_topk(self.hidden, self.inp.w_router, self.inp.bias, T, H, E, k, self.ids,
+                           self.w, self.logits, rw, rw.numel(), st)
+        P = T * k
+        self.counts = torch.empty(E, dtype=torch.int32, device=DEV)
+        self.offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+        self.perm = torch.empty(max(P, 1), dtype=torch.int32, device=DEV)
+        self.inv = torch.empty(max(P, 1), dtype=torch.int32, device=DEV)
+        self.active = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+        bw = ws(sm.moe_bucket_workspace_size(T, k, E))
+        sm.moe_bucket(self.ids, T, k, E, self.counts, self.offsets, self.perm, self.inv,
+                      self.active, bw, bw.numel(), st)
+        decode = T <= sm.DECODE_MAX_T
+        ydt = torch.float32 if decode else torch.float16
+        self.ydtype = sm.DTYPE_F32 if decode else sm.DTYPE_F16
+        self.y = torch.empty(max(P, 1), H, dtype=ydt, device=DEV)
+        ew = ws(sm.moe_experts_workspace_size(self.qw, T, k))
+        sm.moe_experts(self.hidden, self.qw, self.offsets, self.perm, self.active, T, k, self.y,
+                       ew, ew.numel(), st)
+        self.shy = None
+        if self.sqw is not None:
+            self.shy = torch.empty(T, H, dtype=ydt, device=DEV)
+            sw = ws(sm.moe_shared_expert_workspace_size(self.sqw, T))
+            sm.moe_shared_expert(self.hidden, self.sqw, T, self.shy, sw, sw.numel(), st)
+        self.out = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+        self.zero = torch.zeros(T, H, dtype=torch.float32, device=DEV)
+        self.acc = torch.empty(T, H, dtype=torch.float32, device=DEV)
+        sm.moe_combine(self.y, self.ydtype, self.inv, self.w, self.shy, self.ydtype, self.zero, T,
+                       k, H, self.out, self.acc, st)
+        torch.cuda.synchronize()
+        assert sm.strata_read_status(self.status) == 0
+        return self
+
+    def blobs_for(self, ids):
+        return {int(e): self.inp.experts[int(e)].cpu().numpy() for e in np.unique(ids)}
+
+
+def check_layer(r: Run, sample=None):
+    """Full check of one run; sample = token indices for the expert/output
+    checks (all tokens if None)."""
+    T, H, E, k = r.T, r.H, r.E, r.k
+    hid = u16(r.hidden)
+    # RMSNorm within one bf16 ulp
+    ref_h = oracle.rmsnorm(r.inp.x.cpu().numpy(), r.c.eps)
+    a = oracle.bf16_bits_to_f32(hid).astype(np.float64)
+    b = oracle.bf16_bits_to_f32(ref_h).astype(np.float64)
+    ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b), 1e-30))) - 7)
+    assert np.all(np.abs(a - b) <= ulp), "rmsnorm beyond one bf16 ulp"
+    # router on the GPU's hidden
+    wr = u16(r.inp.w_router)
+    bias = None if r.inp.bias is None else r.inp.bias.cpu().numpy()
+    toks = np.arange(T) if sample is None else np.asarray(sample)
+    ref_lg = oracle.router_logits(hid[toks], wr, bias)
+    gl = r.logits.cpu().numpy()[toks]
+    assert np.all(np.abs(gl - ref_lg) <= 1e-4 + 1e-4 * np.abs(ref_lg))
+    gids = r.ids.cpu().numpy()
+    ok, near, bad = check_routing(ref_lg, gids[toks], k)
+    assert ok, f"routing mismatch on tokens {bad[:10]}"
+    if near:
+        print(f"near-tie tokens: {list(toks[near])}")
+    _, ref_w = oracle.topk(gl, k)
+    ref_ids_gpu_logits, _ = oracle.topk(gl, k)
+    np.testing.assert_array_equal(ref_ids_gpu_logits, gids[toks])
+    assert np.abs(r.w.cpu().numpy()[toks] - ref_w).max() <= TOPK_W_ATOL
+    # bucket bit-exact on the GPU's ids
+    counts, offsets, perm, inv = oracle.bucket(gids, E)
+    np.testing.assert_array_equal(r.counts.cpu().numpy(), counts)
+    np.testing.assert_array_equal(r.offsets.cpu().numpy(), offsets)
+    np.testing.assert_array_equal(r.perm.cpu().numpy()[:T * k], perm)
+    np.testing.assert_array_equal(r.inv.cpu().numpy()[:T * k], inv)
+    act = r.active.cpu().numpy()
+    nz = np.nonzero(counts)[0]
+    assert act[0] == len(nz)
+    np.testing.assert_array_equal(act[1:1 + len(nz)], nz)
+    # combine bit-exact given the GPU's y
+    y = r.y.float().cpu().numpy()
+    yp = y[inv]
+    sh = None if r.shy is None else r.shy.float().cpu().numpy()
+    of, ob, _ = oracle.combine(yp, r.w.cpu().numpy(), sh)
+    np.testing.assert_array_equal(u16(r.out), ob)
+    np.testing.assert_array_equal(r.acc.cpu().numpy(), of)
+    # expert outputs and layer output vs the oracle on sampled tokens
+    blobs = r.blobs_for(gids[toks])
+    for t in toks:
+        for j in range(k):
+            e = int(gids[t, j])
+            ref_y = oracle.expert_ffn(r.c.fmt, blobs[e], H, r.I, hid[t])
+            got = y[inv[t * k + j]]
+            assert rel_l2_rows(got, ref_y) <= OUT_REL_L2, (t, j, e)
+    sb = None if r.inp.shared is None else r.inp.shared[0].cpu().numpy()
+    ref = oracle.moe_layer(hid[toks], wr, bias, E, k, r.c.fmt, r.I, blobs,
+                           shared_fmt=r.c.shared_fmt or 0, shared_blob=sb,
+                           forced_ids=gids[toks])
+    got = oracle.bf16_bits_to_f32(u16(r.out)[toks])
+    err = rel_l2_rows(got, ref["out_f32"])
+    assert err.max() <= OUT_REL_L2, f"max per-token rel L2 {err.max():.3e}"
+    return err
+
+
+@pytest.mark.parametrize("config,T", [(0, 1), (1, 4), (3, 1), (3, 4), (4, 1), (4, 4)])
+def test_decode_layer_parity(config, T):
+    r = Run(config, T).run()
+    err = check_layer(r)
+    print(f"C{config} T={T}: max rel L2 {err.max():.2e}")
+
+
+@pytest.mark.parametrize("T", [2, 7, 8, 9, 15, 16])
+def test_decode_ragged_token_counts(T):
+    """Token counts on both sides of the 8-column MMA tile, up to the decode
+    maximum (two column tiles)."""
+    check_layer(Run(1, T).run())
+
+
+def test_decode_small_expert_count_and_k1():
+    """E = 8 experts, every token on several: many tokens per expert."""
+    r = Run(0, 16, E=8)
+    r.k = 1
+    r.run()
+    check_layer(r)
+
+
+def test_decode_deterministic():
+    a = Run(1, 4).run()
+    b = Run(1, 4).run()
+    for x, y in ((a.ids, b.ids), (a.perm, b.perm), (a.y, b.y), (a.out, b.out)):
+        assert torch.equal(x, y)
+
+
+def test_layer_forward_matches_steps():
+    """moe_layer_forward gives bit-identical results to the individual calls,
+    and residual_out = x + acc."""
+    for config, T in ((1, 4), (3, 4)):
+        r = Run(config, T).run()
+        E, k, H = r.E, r.k, r.H
+        layer = sm.MoELayer(r.inp.w_router, r.inp.bias,
+                            sm.ExpertWeights(r.inp.experts, r.c.fmt, H, r.I), k,
+                            None if r.inp.shared is None else
+                            sm.ExpertWeights(r.inp.shared, r.c.shared_fmt, H, r.I), r.c.eps)
+        res = torch.empty(T, H, dtype=torch.float32, device=DEV)
+        ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+        out = layer.forward(r.inp.x, residual_out=res, topk_ids=ids, dev_status=r.status)
+        torch.cuda.synchronize()
+        assert torch.equal(out, r.out) and torch.equal(ids, r.ids)
+        assert torch.equal(res, r.inp.x + r.acc)
+
+
+def test_stacked_layers_teacher_forced():
+    """Config 1's 48-layer stack (first 6 layers here): each layer's input is
+    the previous GPU layer's residual output; every layer is checked."""
+    c = mi.CONFIGS[1]
+    x = mi.gen_x(4, c.H, mi.seed_for(1, 0, "xstep"), DEV)
+    for layer in range(6):
+        r = Run(1, 4, layer=layer, x=x).run()
+        check_layer(r)
+        x = (x + r.acc).contiguous()
+
+
+def test_dev_status_clean_and_invalid_ids_flagged():
+    """Out-of-range ids are skipped and flagged in dev_status, never trapped."""
+    T, k, E = 4, 2, 16
+    ids = torch.tensor([[0, 1], [2, 99], [3, 4], [5, -1]], dtype=torch.int32, device=DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.full((T * k,), -7, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    active = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    sm.moe_bucket(ids, T, k, E, counts, offsets, perm, inv, active, None, 0, st)
+    torch.cuda.synchronize()
+    assert sm.strata_read_status(st) == 5
+    assert int(offsets[-1]) == 6 and int(counts.sum()) == 6
+    assert inv[3].item() == -1 and inv[7].item() == -1
