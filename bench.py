@@ -166,8 +166,7 @@ class DecodeStack:
         self.out = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
         self.xa = torch.empty(T, H, dtype=torch.float32, device=dev)
         self.xb = torch.empty(T, H, dtype=torch.float32, device=dev)
-        n = max(sm.moe_router_topk_workspace_size(T, H, E, k),
-                sm.moe_bucket_workspace_size(T, k, E),
+        n = max(sm.moe_route_workspace_size(T, H, E, k),
                 sm.moe_experts_workspace_size(self.qw[0], T, k),
                 sm.moe_shared_expert_workspace_size(self.sqw[0], T) if self.sqw[0] else 0)
         self.ws = torch.empty(int(n) + 256, dtype=torch.uint8, device=dev)
@@ -183,11 +182,9 @@ class DecodeStack:
         for l in range(self.L):
             nxt = x_out if l == self.L - 1 else (self.xa if (l % 2 == 0) else self.xb)
             act = active_bufs[l]
-            sm.moe_rmsnorm(cur, T, H, self.c.eps, self.hidden)
-            sm.moe_router_topk(self.hidden, self.wr[l], self.bias[l], T, H, E, k, self.ids, self.w,
-                               None, ws, wn, st)
-            sm.moe_bucket(self.ids, T, k, E, self.counts, self.offsets, self.perm, self.inv, act,
-                          ws, wn, st)
+            sm.moe_route(cur, T, H, self.c.eps, self.wr[l], self.bias[l], E, k, self.hidden,
+                         self.ids, self.w, self.counts, self.offsets, self.perm, self.inv, act,
+                         ws, wn, st)
             if events is not None:
                 events[l][0].record()
             sm.moe_experts(self.hidden, self.qw[l], self.offsets, self.perm, act, T, k, self.y, ws,
@@ -203,10 +200,9 @@ class DecodeStack:
 
 def kernels_per_layer(T, k, shared):
     """Kernel launches the library enqueues per layer on the decode path:
-    rmsnorm 1, router 2 (partial GEMV + reduce/top-k), bucket 1 (P <= 1024),
+    moe_route 1 (one cluster kernel: RMSNorm, router, top-k, bucket),
     experts 2 (gate/up, down), shared expert 2, combine 1."""
-    n = 1 + 2 + (1 if T * k <= 1024 else 3) + 2 + 1
-    return n + (2 if shared else 0)
+    return 1 + 2 + 1 + (2 if shared else 0)
 
 
 def run_ours(args):

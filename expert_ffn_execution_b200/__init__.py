@@ -8,7 +8,8 @@ from ._binding import (DECODE_MAX_T, DEV_BOUNDS, DEV_TIMEOUT, DTYPE_F16, DTYPE_F
                        FMT_Q4CB_32, QWeights, StrataError, abi_version, exported_symbols, load,
                        moe_bucket, moe_bucket_workspace_size, moe_combine, moe_experts,
                        moe_experts_workspace_size, moe_layer_forward, moe_layer_workspace_size,
-                       moe_rmsnorm, moe_router_topk, moe_router_topk_workspace_size,
+                       moe_rmsnorm, moe_route, moe_route_workspace_size, moe_router_topk,
+                       moe_router_topk_workspace_size,
                        moe_shared_expert, moe_shared_expert_workspace_size, qweights,
                        status_string, strata_expert_bytes, strata_read_status)
 from .layer import ExpertWeights, MoELayer

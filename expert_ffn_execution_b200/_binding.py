@@ -50,6 +50,9 @@ _SIGS = {
     "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _U64, _P, _P]),
     "moe_bucket_workspace_size": (_U64, [_I, _I, _I]),
     "moe_bucket": (_I, [_P, _I, _I, _I, _P, _P, _P, _P, _P, _P, _U64, _P, _P]),
+    "moe_route_workspace_size": (_U64, [_I, _I, _I, _I]),
+    "moe_route": (_I, [_P, _I, _I, _F, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _U64,
+                       _P, _P]),
     "moe_experts_workspace_size": (_U64, [_QW, _I, _I]),
     "moe_experts": (_I, [_P, _QW, _P, _P, _P, _I, _I, _P, _P, _U64, _P, _P]),
     "moe_shared_expert_workspace_size": (_U64, [_QW, _I]),
@@ -160,6 +163,19 @@ def moe_bucket(topk_ids, T, k, E, counts, offsets, perm, inv, active, workspace,
                            _ptr(inv), _ptr(active), _ptr(workspace), ws_bytes, _ptr(dev_status),
                            _stream(stream))
     return _check("moe_bucket", rc) if check else rc
+
+
+def moe_route_workspace_size(T, H, E, k) -> int:
+    return int(load().moe_route_workspace_size(T, H, E, k))
+
+
+def moe_route(x, T, H, eps, w_router, bias, E, k, hidden, topk_ids, topk_w, counts, offsets,
+              perm, inv, active, workspace, ws_bytes, dev_status, stream=None, check=True):
+    rc = load().moe_route(_ptr(x), T, H, eps, _ptr(w_router), _ptr(bias), E, k, _ptr(hidden),
+                          _ptr(topk_ids), _ptr(topk_w), _ptr(counts), _ptr(offsets), _ptr(perm),
+                          _ptr(inv), _ptr(active), _ptr(workspace), ws_bytes, _ptr(dev_status),
+                          _stream(stream))
+    return _check("moe_route", rc) if check else rc
 
 
 def moe_experts_workspace_size(w: QWeights, T, k) -> int:

@@ -1,6 +1,6 @@
 // abi.cu -- extern "C" entry points of libstrata_moe.so: argument checks,
 // workspace carving and kernel launches.  See include/strata_moe.h.
-#include <mutex>
+#include <algorithm>
 
 #include "decode.cuh"
 
@@ -78,12 +78,8 @@ int32_t run_experts(const uint16_t* hidden, const strata_qweights* w, const int3
     a.hbuf = reinterpret_cast<uint16_t*>(ws);
     a.y = reinterpret_cast<float*>(y);
     a.status = status;
-    const int sms = num_sms_of_current_device();
-    const size_t xs = decode_smem_bytes(T, w->hidden);
-    int bps = (int)((200u * 1024u) / (xs ? xs : 1));
-    if (bps > 2) bps = 2;
-    if (bps < 1) bps = 1;
-    a.grid = sms * bps;
+    a.num_sms = num_sms_of_current_device();
+    if (decode_smem_bytes(T, w->hidden) > 200u * 1024u) return STRATA_EUNSUPPORTED;
     (void)ws_bytes;
     return from_cuda(launch_experts_decode(a, st));
   }
@@ -173,10 +169,75 @@ int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router, const 
   if (!aligned(w_router, 4) || !aligned(workspace, 16) || (logits_opt && !aligned(logits_opt, 4)))
     return STRATA_EINVAL;
   if (ws_bytes < moe_router_topk_workspace_size(T, H, E, k)) return STRATA_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T <= kDecodeMaxTokens && route_decode_supported(T, H, E, k)) {
+    RouteArgs a = {};
+    a.hidden = hidden;
+    a.wr = w_router;
+    a.bias = bias;
+    a.T = T;
+    a.H = H;
+    a.E = E;
+    a.k = k;
+    a.ids = topk_ids;
+    a.w = topk_w;
+    a.logits_opt = logits_opt;
+    a.status = dev_status;
+    const cudaError_t e = launch_route_decode(a, st);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+  }
   return from_cuda(launch_router_topk(hidden, w_router, bias, T, H, E, k, topk_ids, topk_w,
                                       logits_opt, workspace, dev_status,
-                                      num_sms_of_current_device(),
-                                      reinterpret_cast<cudaStream_t>(stream)));
+                                      num_sms_of_current_device(), st));
+}
+
+uint64_t moe_route_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k) {
+  if (T < 0 || H <= 0 || E <= 0 || k < 1) return 0;
+  return std::max(moe_router_topk_workspace_size(T, H, E, k), moe_bucket_workspace_size(T, k, E));
+}
+
+int32_t moe_route(const float* x, int32_t T, int32_t H, float eps, const uint16_t* w_router,
+                  const float* bias, int32_t E, int32_t k, uint16_t* hidden, int32_t* topk_ids,
+                  float* topk_w, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                  int32_t* active, void* workspace, uint64_t ws_bytes, int32_t* dev_status,
+                  void* stream) {
+  if (T < 0 || H < 64 || H % 64 || H > 16384 || E < 2 || E > 1024 || E % 2 || k < 1 || k > E ||
+      k > 32 || !(eps >= 0.f))
+    return STRATA_EINVAL;
+  if (T == 0) return STRATA_OK;
+  if (!x || !w_router || !hidden || !topk_ids || !topk_w || !counts || !offsets || !perm ||
+      !inv || !active || !aligned(x, 16) || !aligned(hidden, 16) || !aligned(w_router, 16))
+    return STRATA_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T <= kDecodeMaxTokens && route_decode_supported(T, H, E, k)) {
+    RouteArgs a = {};
+    a.x = x;
+    a.hidden_out = hidden;
+    a.eps = eps;
+    a.wr = w_router;
+    a.bias = bias;
+    a.T = T;
+    a.H = H;
+    a.E = E;
+    a.k = k;
+    a.ids = topk_ids;
+    a.w = topk_w;
+    a.counts = counts;
+    a.offsets = offsets;
+    a.perm = perm;
+    a.inv = inv;
+    a.active = active;
+    a.status = dev_status;
+    const cudaError_t e = launch_route_decode(a, st);
+    if (e != cudaErrorNotSupported) return from_cuda(e);
+  }
+  int32_t r;
+  if ((r = moe_rmsnorm(x, T, H, eps, hidden, stream)) != STRATA_OK) return r;
+  if ((r = moe_router_topk(hidden, w_router, bias, T, H, E, k, topk_ids, topk_w, nullptr,
+                           workspace, ws_bytes, dev_status, stream)) != STRATA_OK)
+    return r;
+  return moe_bucket(topk_ids, T, k, E, counts, offsets, perm, inv, active, workspace, ws_bytes,
+                    dev_status, stream);
 }
 
 uint64_t moe_bucket_workspace_size(int32_t T, int32_t k, int32_t E) {
@@ -322,12 +383,8 @@ int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router, c
   void* scratch = base + L.scratch;
   const uint64_t scratch_bytes = L.total - L.scratch;
   int32_t r;
-  if ((r = moe_rmsnorm(x, T, H, eps, hidden, stream)) != STRATA_OK) return r;
-  if ((r = moe_router_topk(hidden, w_router, bias, T, H, E, k, ids, tw, nullptr, scratch,
-                           scratch_bytes, dev_status, stream)) != STRATA_OK)
-    return r;
-  if ((r = moe_bucket(ids, T, k, E, counts, offsets, perm, inv, active, scratch, scratch_bytes,
-                      dev_status, stream)) != STRATA_OK)
+  if ((r = moe_route(x, T, H, eps, w_router, bias, E, k, hidden, ids, tw, counts, offsets, perm,
+                     inv, active, scratch, scratch_bytes, dev_status, stream)) != STRATA_OK)
     return r;
   if ((r = moe_experts(hidden, w, offsets, perm, active, T, k, y, scratch, scratch_bytes,
                        dev_status, stream)) != STRATA_OK)

@@ -3,23 +3,19 @@
 
 namespace strata {
 
-// hidden[t,h] = bf16_rne(x[t,h] / sqrt(mean_h x^2 + eps)), one CTA per token.
+// hidden[t,h] = bf16_rne(x[t,h] * (1 / sqrt(mean_h x^2 + eps))), one CTA per
+// token; the RMS comes from rms_inv_warp (the same bits as the fused routing
+// kernel).
 __global__ void __launch_bounds__(256)
 rmsnorm_kernel(const float* __restrict__ x, int H, float eps, uint16_t* __restrict__ out) {
-  __shared__ float red[8];
+  __shared__ float s_inv;
   const float* xr = x + (size_t)blockIdx.x * H;
-  float ss = 0.f;
-  for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
-    const float4 v = *reinterpret_cast<const float4*>(xr + h);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  if (threadIdx.x < 32) {
+    const float inv = rms_inv_warp(xr, H, eps);
+    if (threadIdx.x == 0) s_inv = inv;
   }
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
-  float tot = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) tot += red[i];
-  const float inv = 1.0f / sqrtf(tot / (float)H + eps);
+  const float inv = s_inv;
   uint16_t* orow = out + (size_t)blockIdx.x * H;
   for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
     const float4 v = *reinterpret_cast<const float4*>(xr + h);
@@ -50,7 +46,10 @@ STRATA_DEVFN void load8(const void* base, int dtype, size_t idx, float (&v)[8]) 
 
 // acc = sum_j w_j * y[inv[t*k+j]] (j ascending, separate multiply and add,
 // no contraction), + shared_y; out = bf16(acc); residual_out = residual + acc.
-__global__ void __launch_bounds__(256)
+// grid (T, ceil(H / (8 * 128))): each thread owns 8 consecutive features and
+// issues the loads of four expert rows before accumulating them in order.
+constexpr int kCombThreads = 128;
+__global__ void __launch_bounds__(kCombThreads)
 combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restrict__ inv,
                const float* __restrict__ w, const void* __restrict__ shared_y, int shared_dtype,
                const float* __restrict__ residual, int k, int H, uint16_t* __restrict__ out,
@@ -64,45 +63,57 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
     s_w[threadIdx.x] = w[p];
   }
   __syncthreads();
-  for (int h = threadIdx.x * 8; h < H; h += blockDim.x * 8) {
-    float acc[8];
+  const int h = (blockIdx.y * kCombThreads + threadIdx.x) * 8;
+  if (h >= H) return;
+  float acc[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int pos = s_pos[j];
-      if (pos < 0) {
-        if (h == threadIdx.x * 8) dev_flag(status, STRATA_DEV_BOUNDS);
-        continue;
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int j0 = 0; j0 < k; j0 += 4) {
+    float v[4][8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u;
+      const int pos = (j < k) ? s_pos[j] : -1;
+      if (pos >= 0) {
+        load8(y, y_dtype, (size_t)pos * H + h, v[u]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[u][i] = 0.f;
+        if (j < k && h == 0) dev_flag(status, STRATA_DEV_BOUNDS);
       }
-      float v[8];
-      load8(y, y_dtype, (size_t)pos * H + h, v);
-      const float wj = s_w[j];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, v[i]));
     }
-    if (shared_y) {
-      float v[8];
-      load8(shared_y, shared_dtype, (size_t)t * H + h, v);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
-    }
-    uint32_t o[4];
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u;
+      if (j < k && s_pos[j] >= 0) {
+        const float wj = s_w[j];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      o[i] = float_to_bf16_bits(acc[2 * i]) | (uint32_t(float_to_bf16_bits(acc[2 * i + 1])) << 16);
-    *reinterpret_cast<uint4*>(out + (size_t)t * H + h) = make_uint4(o[0], o[1], o[2], o[3]);
-    if (residual_out) {
-      const float* r = residual + (size_t)t * H + h;
-      const float4 r0 = *reinterpret_cast<const float4*>(r);
-      const float4 r1 = *reinterpret_cast<const float4*>(r + 4);
-      float4 o0 = make_float4(__fadd_rn(r0.x, acc[0]), __fadd_rn(r0.y, acc[1]),
-                              __fadd_rn(r0.z, acc[2]), __fadd_rn(r0.w, acc[3]));
-      float4 o1 = make_float4(__fadd_rn(r1.x, acc[4]), __fadd_rn(r1.y, acc[5]),
-                              __fadd_rn(r1.z, acc[6]), __fadd_rn(r1.w, acc[7]));
-      float* ro = residual_out + (size_t)t * H + h;
-      *reinterpret_cast<float4*>(ro) = o0;
-      *reinterpret_cast<float4*>(ro + 4) = o1;
+        for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], __fmul_rn(wj, v[u][i]));
+      }
     }
+  }
+  if (shared_y) {
+    float v[8];
+    load8(shared_y, shared_dtype, (size_t)t * H + h, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
+  }
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+    o[i] = float_to_bf16_bits(acc[2 * i]) | (uint32_t(float_to_bf16_bits(acc[2 * i + 1])) << 16);
+  *reinterpret_cast<uint4*>(out + (size_t)t * H + h) = make_uint4(o[0], o[1], o[2], o[3]);
+  if (residual_out) {
+    const float* r = residual + (size_t)t * H + h;
+    const float4 r0 = *reinterpret_cast<const float4*>(r);
+    const float4 r1 = *reinterpret_cast<const float4*>(r + 4);
+    const float4 o0 = make_float4(__fadd_rn(r0.x, acc[0]), __fadd_rn(r0.y, acc[1]),
+                                  __fadd_rn(r0.z, acc[2]), __fadd_rn(r0.w, acc[3]));
+    const float4 o1 = make_float4(__fadd_rn(r1.x, acc[4]), __fadd_rn(r1.y, acc[5]),
+                                  __fadd_rn(r1.z, acc[6]), __fadd_rn(r1.w, acc[7]));
+    float* ro = residual_out + (size_t)t * H + h;
+    *reinterpret_cast<float4*>(ro) = o0;
+    *reinterpret_cast<float4*>(ro + 4) = o1;
   }
 }
 
@@ -118,10 +129,8 @@ cudaError_t launch_combine(const void* y, int y_dtype, const int32_t* inv, const
                            int T, int k, int H, uint16_t* out, float* residual_out,
                            int32_t* status, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  int threads = (H / 8 + 31) / 32 * 32;
-  if (threads > 256) threads = 256;
-  if (threads < 32) threads = 32;
-  combine_kernel<<<T, threads, 0, st>>>(y, y_dtype, inv, w, shared_y, shared_dtype, residual, k,
+  dim3 grid(T, (H / 8 + kCombThreads - 1) / kCombThreads);
+  combine_kernel<<<grid, kCombThreads, 0, st>>>(y, y_dtype, inv, w, shared_y, shared_dtype, residual, k,
                                          H, out, residual_out, status);
   return cudaGetLastError();
 }

@@ -75,3 +75,95 @@ STRATA_DEVFN float warp_sum(float v) {
 }
 
 }  // namespace strata
+
+namespace strata {
+
+// ---------------------------------------------------------------- mbarrier / bulk copy
+// Every wait is bounded: after kWaitLimit polls it gives up, ORs
+// STRATA_DEV_TIMEOUT into the status word and returns false.
+constexpr uint32_t kWaitLimit = 1u << 26;
+
+STRATA_DEVFN uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+STRATA_DEVFN void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+               : "memory");
+}
+
+// Make mbarrier initialisation visible to the async proxy (bulk copies).
+STRATA_DEVFN void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+STRATA_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+STRATA_DEVFN bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of the barrier.
+STRATA_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
+  dev_flag(status, STRATA_DEV_TIMEOUT);
+  return false;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory; completion is counted on
+// `bar` in bytes.  dst, src and bytes must be multiples of 16.
+STRATA_DEVFN void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// ldmatrix x4, transposed (four 8x8 b16 tiles).
+STRATA_DEVFN void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
+// D[16x8] += A[16x16] * B[16x8], bf16 inputs, fp32 accumulate.
+STRATA_DEVFN void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// 1 / sqrt(mean(x^2) + eps) of one row, computed by one warp in a fixed order
+// (lane-strided float4 partial sums, then a butterfly), so every kernel that
+// normalises a row gets the same bits.
+STRATA_DEVFN float rms_inv_warp(const float* __restrict__ xr, int H, float eps) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+  for (int h = lane * 4; h < H; h += 128) {
+    const float4 v = *reinterpret_cast<const float4*>(xr + h);
+    ss = fmaf(v.x, v.x, ss);
+    ss = fmaf(v.y, v.y, ss);
+    ss = fmaf(v.z, v.z, ss);
+    ss = fmaf(v.w, v.w, ss);
+  }
+  ss = warp_sum(ss);
+  return 1.0f / sqrtf(ss / (float)H + eps);
+}
+
+}  // namespace strata

@@ -19,7 +19,7 @@ struct DecodeArgs {
   uint16_t* hbuf;  // scratch fp16 [rows, I]
   float* y;        // [rows, H]
   int32_t* status;
-  int grid;
+  int num_sms;
 };
 cudaError_t launch_experts_decode(const DecodeArgs& a, cudaStream_t st);
 size_t decode_smem_bytes(int T, int H);
@@ -41,6 +41,23 @@ struct PrefillArgs {
 };
 uint64_t prefill_workspace_bytes(int T, int H, int I, int E, int k, int shared_mode);
 cudaError_t launch_experts_prefill(const PrefillArgs& a, cudaStream_t st);
+
+struct RouteArgs {
+  const float* x;          // fp32 [T,H]: normalise it (hidden_out gets the bf16 result), or
+  const uint16_t* hidden;  // bf16 [T,H] input when x == nullptr
+  uint16_t* hidden_out;
+  float eps;
+  const uint16_t* wr;
+  const float* bias;
+  int T, H, E, k;
+  int32_t* ids;
+  float* w;
+  float* logits_opt;
+  int32_t *counts, *offsets, *perm, *inv, *active;  // bucket outputs (counts == nullptr: skip)
+  int32_t* status;
+};
+bool route_decode_supported(int T, int H, int E, int k);
+cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
 
 cudaError_t launch_rmsnorm(const float* x, int T, int H, float eps, uint16_t* out, cudaStream_t st);
 uint64_t router_workspace_bytes(int T, int H, int E, int k);

@@ -14,13 +14,17 @@
 
 namespace strata {
 
-constexpr int kRouterRows = 32;     // W_r rows per CTA (decode GEMV)
-constexpr int kRouterThreads = 512; // two experts per thread, E <= 1024
+constexpr int kRouterRows = 64;   // W_r rows per row slice (decode GEMV)
+constexpr int kRouterCols = 128;  // experts per column slice
+constexpr int kRouterGroups = 4;  // row groups per CTA (16 rows each)
 
-__global__ void __launch_bounds__(kRouterThreads)
+// grid (ceil(H/64), ceil(E/128)); thread (group, pair): 16 rows x 2 experts;
+// the 4 row groups are summed in a fixed order in shared memory.
+__global__ void __launch_bounds__(256)
 router_gemv_partial(const uint16_t* __restrict__ hidden, const uint16_t* __restrict__ wr, int T,
                     int H, int E, float* __restrict__ partial) {
   __shared__ float xs[kDecodeMaxTokens][kRouterRows];
+  __shared__ float red[kRouterGroups - 1][kDecodeMaxTokens][kRouterCols];
   const int s = blockIdx.x;
   const int h0 = s * kRouterRows;
   for (int i = threadIdx.x; i < T * kRouterRows; i += blockDim.x) {
@@ -28,30 +32,56 @@ router_gemv_partial(const uint16_t* __restrict__ hidden, const uint16_t* __restr
     xs[t][r] = (h0 + r < H) ? bf16_bits_to_float(hidden[(size_t)t * H + h0 + r]) : 0.f;
   }
   __syncthreads();
-  const int e2 = threadIdx.x;  // experts 2*e2, 2*e2+1
-  if (2 * e2 >= E) return;
+  const int grp = threadIdx.x / (kRouterCols / 2);
+  const int pr = threadIdx.x % (kRouterCols / 2);
+  const int e = blockIdx.y * kRouterCols + 2 * pr;
+  const bool live = e < E;
   float acc[kDecodeMaxTokens][2];
 #pragma unroll
   for (int t = 0; t < kDecodeMaxTokens; ++t) acc[t][0] = acc[t][1] = 0.f;
   const uint32_t* w32 = reinterpret_cast<const uint32_t*>(wr);
-  const int nr = min(kRouterRows, H - h0);
-#pragma unroll 8
-  for (int r = 0; r < nr; ++r) {
-    const uint32_t wv = ld_stream_u32(w32 + ((size_t)(h0 + r) * E) / 2 + e2);
-    const float w0 = __uint_as_float(wv << 16), w1 = __uint_as_float(wv & 0xffff0000u);
+  const int rbeg = grp * (kRouterRows / kRouterGroups);
+  if (live) {
+    uint32_t wv[kRouterRows / kRouterGroups];
 #pragma unroll
-    for (int t = 0; t < kDecodeMaxTokens; ++t) {
-      if (t < T) {
-        acc[t][0] = fmaf(xs[t][r], w0, acc[t][0]);
-        acc[t][1] = fmaf(xs[t][r], w1, acc[t][1]);
+    for (int r = 0; r < kRouterRows / kRouterGroups; ++r) {
+      const int h = h0 + rbeg + r;
+      wv[r] = (h < H) ? ld_stream_u32(w32 + ((size_t)h * E + e) / 2) : 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < kRouterRows / kRouterGroups; ++r) {
+      const float w0 = __uint_as_float(wv[r] << 16), w1 = __uint_as_float(wv[r] & 0xffff0000u);
+#pragma unroll
+      for (int t = 0; t < kDecodeMaxTokens; ++t) {
+        if (t < T) {
+          acc[t][0] = fmaf(xs[t][rbeg + r], w0, acc[t][0]);
+          acc[t][1] = fmaf(xs[t][rbeg + r], w1, acc[t][1]);
+        }
       }
     }
   }
+  if (grp > 0) {
 #pragma unroll
-  for (int t = 0; t < kDecodeMaxTokens; ++t) {
-    if (t < T) {
-      float2 v = make_float2(acc[t][0], acc[t][1]);
-      *reinterpret_cast<float2*>(partial + ((size_t)s * T + t) * E + 2 * e2) = v;
+    for (int t = 0; t < kDecodeMaxTokens; ++t) {
+      if (t < T) {
+        red[grp - 1][t][2 * pr] = acc[t][0];
+        red[grp - 1][t][2 * pr + 1] = acc[t][1];
+      }
+    }
+  }
+  __syncthreads();
+  if (grp == 0 && live) {
+#pragma unroll
+    for (int t = 0; t < kDecodeMaxTokens; ++t) {
+      if (t < T) {
+        float a0 = acc[t][0], a1 = acc[t][1];
+#pragma unroll
+        for (int g2 = 0; g2 < kRouterGroups - 1; ++g2) {
+          a0 += red[g2][t][2 * pr];
+          a1 += red[g2][t][2 * pr + 1];
+        }
+        *reinterpret_cast<float2*>(partial + ((size_t)s * T + t) * E + e) = make_float2(a0, a1);
+      }
     }
   }
 }
@@ -108,7 +138,7 @@ router_gemm(const uint16_t* __restrict__ hidden, const uint16_t* __restrict__ wr
 
 // One CTA per token: logits = bias + sum of slices (fixed order), then the
 // top-k by warp 0 with registers and shuffles.
-constexpr int kFinishThreads = 128;
+constexpr int kFinishThreads = 512;
 template <int NPL>  // logits per lane, E <= 32 * NPL
 __global__ void __launch_bounds__(kFinishThreads)
 router_finish(const float* __restrict__ partial, int nslices, int T, int E, int k,
@@ -117,8 +147,16 @@ router_finish(const float* __restrict__ partial, int nslices, int T, int E, int 
   __shared__ float lg[32 * NPL];
   const int t = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    float s = 0.f;
-    for (int sl = 0; sl < nslices; ++sl) s += partial[((size_t)sl * T + t) * E + e];
+    // eight independent partial sums (loads in flight), combined in a fixed order
+    float a[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = 0.f;
+    for (int sl = 0; sl < nslices; sl += 8) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (sl + u < nslices) a[u] += partial[((size_t)(sl + u) * T + t) * E + e];
+    }
+    float s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
     if (bias) s += bias[e];
     lg[e] = s;
     if (logits_opt) logits_opt[(size_t)t * E + e] = s;
@@ -190,7 +228,8 @@ cudaError_t launch_router_topk(const uint16_t* hidden, const uint16_t* wr, const
   int ns = 1;
   if (T <= kDecodeMaxTokens) {
     ns = (H + kRouterRows - 1) / kRouterRows;
-    router_gemv_partial<<<ns, kRouterThreads, 0, st>>>(hidden, wr, T, H, E, part);
+    dim3 grid(ns, (E + kRouterCols - 1) / kRouterCols);
+    router_gemv_partial<<<grid, 256, 0, st>>>(hidden, wr, T, H, E, part);
   } else {
     dim3 grid((T + kGBM - 1) / kGBM, (E + kGBN - 1) / kGBN);
     router_gemm<<<grid, 256, 0, st>>>(hidden, wr, T, H, E, part);

@@ -168,6 +168,22 @@ STRATA_API int32_t moe_bucket(const int32_t* topk_ids, int32_t T, int32_t k, int
                    int32_t* inv, int32_t* active, void* workspace,
                    uint64_t ws_bytes, int32_t* dev_status, void* stream);
 
+/* The routing step in one call: moe_rmsnorm(x) -> moe_router_topk ->
+ * moe_bucket, with the same outputs as those three calls (bit for bit).
+ * For T <= STRATA_DECODE_MAX_T (and E <= 512) it runs as ONE kernel: a
+ * 16-CTA thread-block cluster that streams W_r through shared memory,
+ * reduces the partial logits over distributed shared memory and sorts the
+ * pairs in the leader CTA.
+ *   x      fp32 [T,H];  hidden bf16 [T,H] out (the normalised tokens)
+ *   the other arguments as in moe_router_topk and moe_bucket. */
+STRATA_API uint64_t moe_route_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
+STRATA_API int32_t moe_route(const float* x, int32_t T, int32_t H, float eps,
+                             const uint16_t* w_router, const float* bias, int32_t E, int32_t k,
+                             uint16_t* hidden, int32_t* topk_ids, float* topk_w,
+                             int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                             int32_t* active, void* workspace, uint64_t ws_bytes,
+                             int32_t* dev_status, void* stream);
+
 /* Routed experts: for every sorted position s with pair p = perm[s], token
  * t = p / k, expert e (offsets[e] <= s < offsets[e+1]):
  *   g = W_gate[e] . hidden[t],  u = W_up[e] . hidden[t],

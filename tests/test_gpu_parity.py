@@ -233,3 +233,29 @@ def test_dev_status_clean_and_invalid_ids_flagged():
     assert sm.strata_read_status(st) == 5
     assert int(offsets[-1]) == 6 and int(counts.sum()) == 6
     assert inv[3].item() == -1 and inv[7].item() == -1
+
+
+@pytest.mark.parametrize("config,T", [(1, 1), (1, 4), (1, 16), (4, 4), (4, 16)])
+def test_route_matches_separate_calls(config, T):
+    """moe_route (the fused decode routing kernel for T <= 16) gives the same
+    bits as moe_rmsnorm -> moe_router_topk -> moe_bucket."""
+    r = Run(config, T).run()
+    E, k, H = r.E, r.k, r.H
+    hid = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    active = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    wsb = ws(sm.moe_route_workspace_size(T, H, E, k))
+    sm.moe_route(r.inp.x, T, H, r.c.eps, r.inp.w_router, r.inp.bias, E, k, hid, ids, w, counts,
+                 offsets, perm, inv, active, wsb, wsb.numel(), r.status)
+    torch.cuda.synchronize()
+    assert sm.strata_read_status(r.status) == 0
+    assert torch.equal(hid, r.hidden) and torch.equal(ids, r.ids) and torch.equal(w, r.w)
+    assert torch.equal(counts, r.counts) and torch.equal(offsets, r.offsets)
+    assert torch.equal(perm, r.perm[:T * k]) and torch.equal(inv, r.inv[:T * k])
+    nact = int(active[0])
+    assert torch.equal(active[:1 + nact], r.active[:1 + nact])
