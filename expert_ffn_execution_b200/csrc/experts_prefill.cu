@@ -1,17 +1,501 @@
 // experts_prefill.cu -- tensor-core grouped GEMM path of moe_experts (T > 16).
-#include "decode.cuh"
+//
+// With thousands of tokens the experts are compute-bound, so the weights are
+// dequantised to fp16 tiles in shared memory and multiplied on the 5th-gen
+// tensor cores (tcgen05.mma, fp16 x fp16 -> fp32 in tensor memory).  The
+// GEMMs are "swap-AB": the MMA's 128-row A operand is a tile of one expert's
+// weight rows and the N columns are that expert's tokens (<= 128 per tile,
+// padded to a multiple of 16), so skewed per-expert token counts waste at
+// most 15 columns per tile instead of up to 127 rows.
+//
+// Per call:
+//   1. plan:   per-expert token counts (from offsets) -> a list of n-tiles
+//              (expert, first sorted row, tokens), full tiles first, then the
+//              partial ones by decreasing size.
+//   2. gather: X[s] = fp16(hidden[token of sorted pair s]) (exact: bf16 has 8
+//              significant bits), so the B operand is a plain 2-D TMA tile.
+//   3. gate/up GEMM: units (n-tile, 128 rows of I); A = gate rows and the
+//              same up rows, two accumulators in TMEM; the epilogue applies
+//              SwiGLU and writes h fp16 [P, I] in sorted order.
+//   4. down GEMM: units (n-tile, 128 rows of H); B = h tiles by TMA; the
+//              epilogue writes y fp16 [P, H] in sorted order.
+//
+// GEMM kernel, one CTA per SM, persistent over units (static round robin over
+// the size-sorted list), warp-specialised:
+//   warps 0-3  epilogue: tcgen05.ld of their TMEM lane quarter, math, stores
+//   warps 4-7  producers: one weight row per thread; codes and scales are
+//              prefetched four K-chunks ahead in registers, decoded to fp16
+//              and stored into the 128-byte-swizzled K-major stage layout;
+//              producer thread 0 also issues the TMA load of the B tile
+//   warp 8     tensor memory allocation and the single MMA-issuing thread
+// Stages are guarded by mbarriers (full: producers + TMA bytes; empty:
+// tcgen05.commit), accumulators by tmem_full/tmem_empty.  Every wait is
+// bounded (clock budget) and reports STRATA_DEV_TIMEOUT instead of hanging.
+#include <algorithm>
+
+#include "routing.cuh"
+#include "tc05.cuh"
 
 namespace strata {
 
-uint64_t prefill_workspace_bytes(int T, int H, int I, int E, int k, int shared_mode) {
-  (void)H; (void)E;
+constexpr int kPM = 128;       // weight rows per tile (MMA M)
+constexpr int kPN = 128;       // tokens per n-tile (MMA N <= 128)
+constexpr int kPK = 64;        // K per stage: one 128-byte swizzle row of fp16
+constexpr int kPThreads = 9 * 32;
+constexpr int kTileBytes = kPM * kPK * 2;  // 16 KB per operand tile
+constexpr int kAccCols = 256;              // TMEM columns per accumulator set
+
+struct NTile {
+  int e, s0, n, pad;
+};
+
+template <int MODE>
+struct PCfg {  // MODE 0: gate/up, 1: down
+  static constexpr int NA = (MODE == 0) ? 2 : 1;
+  static constexpr int S = (MODE == 0) ? 4 : 6;
+  static constexpr int SB = (NA + 1) * kTileBytes;
+};
+
+template <int MODE>
+__host__ __device__ inline size_t prefill_smem_bytes() {
+  return 1024 + (size_t)PCfg<MODE>::S * PCfg<MODE>::SB + 256;
+}
+
+// ---------------------------------------------------------------- dequant (natural order)
+// Q2: one 32-bit word (16 codes) -> R[i] = (element 2i, element 2i+1) in fp16.
+// A byte is duplicated into both halves; each pair's two codes are masked
+// into mantissa positions p (low) and p' (high) of fp16 numbers whose
+// exponent gives that position unit weight, so M_p + c is exact; subtracting
+// M_p + 1.5 gives c - 1.5 exactly and one multiply by the scale rounds once.
+STRATA_DEVFN void dq_q2_natural(uint32_t w, __half2 d2, uint32_t (&R)[8]) {
+  const __half2 SA = u32_as_h2(0x54185C06u);  // (257.5, 65.5)
+  const __half2 SB = u32_as_h2(0x4C605418u);  // (65.5, 17.5)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t x = __byte_perm(w, 0, 0x4040 | (j << 8) | j);
+    const uint32_t a = ((x << 2) & 0x0030000Cu) | 0x54005C00u;
+    const uint32_t b = (x & 0x00C00030u) | 0x4C005400u;
+    R[2 * j] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(a), SA), d2));
+    R[2 * j + 1] = h2_as_u32(__hmul2(__hsub2(u32_as_h2(b), SB), d2));
+  }
+}
+
+template <int FMT>
+struct PChunk {  // one row's codes and scales for one K chunk of 64
+  uint4 c[FMT == STRATA_FMT_Q2_32 ? 1 : 2];
+  uint32_t s;
+};
+
+template <int FMT>
+STRATA_DEVFN void load_chunk(PChunk<FMT>& r, const uint8_t* codes_row, const uint8_t* scales_row,
+                             int kc) {
+  constexpr int CB = (FMT == STRATA_FMT_Q2_32) ? 16 : 32;
+#pragma unroll
+  for (int i = 0; i < CB / 16; ++i) r.c[i] = ld_stream_v4(codes_row + kc * CB + 16 * i);
+  r.s = ld_stream_u32(scales_row + kc * 4);
+}
+
+// Decode one row's chunk and store it, swizzled, into a [128 x 64] fp16 tile.
+template <int FMT>
+STRATA_DEVFN void store_chunk(const PChunk<FMT>& r, uint8_t* tile, int row, const Q4Table& T4) {
+  uint8_t* rbase = tile + row * 128;
+  const int sw = row & 7;
+  const __half2 d0 = u32_as_h2(__byte_perm(r.s, 0, 0x1010));
+  const __half2 d1 = u32_as_h2(__byte_perm(r.s, 0, 0x3232));
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {  // 16 elements per group, two 16-byte chunks
+    uint32_t R[8];
+    const __half2 d2 = (g < 2) ? d0 : d1;
+    if constexpr (FMT == STRATA_FMT_Q2_32) {
+      const uint32_t w = (g == 0) ? r.c[0].x : (g == 1) ? r.c[0].y : (g == 2) ? r.c[0].z : r.c[0].w;
+      dq_q2_natural(w, d2, R);
+    } else {
+      const uint4& v = r.c[g >> 1];
+      dq_q4_group((g & 1) ? v.z : v.x, (g & 1) ? v.w : v.y, d2, T4, R);
+    }
+    const int c0 = 2 * g, c1 = 2 * g + 1;
+    *reinterpret_cast<uint4*>(rbase + ((c0 ^ sw) << 4)) = make_uint4(R[0], R[1], R[2], R[3]);
+    *reinterpret_cast<uint4*>(rbase + ((c1 ^ sw) << 4)) = make_uint4(R[4], R[5], R[6], R[7]);
+  }
+}
+
+// ---------------------------------------------------------------- plan / gather
+// One CTA (blockDim >= E): n-tiles of <= kPN tokens per active expert, full
+// tiles first, then partial tiles by decreasing size.
+__global__ void __launch_bounds__(1024)
+prefill_plan_kernel(const int32_t* __restrict__ offsets, int E, int shared_T, NTile* tiles,
+                    int* ntiles) {
+  __shared__ int bins[kPN];
+  __shared__ int scr[40];
+  const int e = threadIdx.x;
+  for (int i = threadIdx.x; i < kPN; i += blockDim.x) bins[i] = 0;
+  __syncthreads();
+  int n = 0, beg = 0;
+  if (e < E) {
+    if (shared_T >= 0) {
+      n = shared_T;
+    } else {
+      beg = offsets[e];
+      n = offsets[e + 1] - beg;
+    }
+  }
+  const int nfull = n / kPN, part = n % kPN;
+  int total_full = 0;
+  const int fpos = block_excl_scan_any(nfull, scr, &total_full);
+  for (int i = 0; i < nfull; ++i) tiles[fpos + i] = NTile{e, beg + i * kPN, kPN, 0};
+  int slot = 0;
+  if (part > 0) slot = atomicAdd(&bins[part], 1);
+  __syncthreads();
+  // partial tiles ordered by decreasing size: base[size] = sum of bins above
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int sz = kPN - 1; sz >= 1; --sz) {
+      const int c = bins[sz];
+      bins[sz] = run;
+      run += c;
+    }
+    *ntiles = total_full + run;
+  }
+  __syncthreads();
+  if (part > 0) tiles[total_full + bins[part] + slot] = NTile{e, beg + nfull * kPN, part, 0};
+}
+
+// X[s] = fp16(hidden[token(s)]), token(s) = perm[s] / k (or s for the shared expert).
+__global__ void __launch_bounds__(256)
+prefill_gather_kernel(const uint16_t* __restrict__ hidden, const int32_t* __restrict__ perm,
+                      int k, int P, int T, int H, uint16_t* __restrict__ X, int32_t* status) {
+  const int groups = H / 8;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)P * groups;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int s = (int)(i / groups), g = (int)(i - (long long)s * groups);
+    int tok = perm ? perm[s] / k : s;
+    if (tok < 0 || tok >= T) {
+      dev_flag(status, STRATA_DEV_BOUNDS);
+      tok = 0;
+    }
+    const uint4 v = *reinterpret_cast<const uint4*>(hidden + (size_t)tok * H + g * 8);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      o[j] = h2_as_u32(__floats2half2_rn(__uint_as_float(w[j] << 16),
+                                         __uint_as_float(w[j] & 0xffff0000u)));
+    *reinterpret_cast<uint4*>(X + (size_t)s * H + g * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ---------------------------------------------------------------- grouped GEMM
+template <int MODE, int FMT>
+__global__ void __launch_bounds__(kPThreads, 1)
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __restrict__ wbase,
+                    uint64_t stride, int H, int I, const NTile* __restrict__ tiles,
+                    const int* __restrict__ ntiles_ptr, uint16_t* __restrict__ out,
+                    int32_t* status) {
+  using C = PCfg<MODE>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::S * C::SB);
+  uint64_t* empty = full + C::S;
+  uint64_t* tfull = empty + C::S;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int K = (MODE == 0) ? H : I;
+  const int Mtot = (MODE == 0) ? I : H;
+  const int MT = Mtot / kPM;
+  const int KC = K / kPK;
+  const int ntiles = *ntiles_ptr;
+  const int total = ntiles * MT;
+  const Planes P = plane_offsets(FMT, H, I);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::S; ++s) {
+      mbar_init(&full[s], 128);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 128);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 2 * kAccCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 4 * 32) prefetch_tensormap(&bmap);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp < 4) {
+    // ------------------------------------------------ epilogue
+    const int m = threadIdx.x;  // TMEM lane = weight row within the tile
+    int it = 0;
+    for (int u = blockIdx.x; u < total; u += gridDim.x, ++it) {
+      const NTile tl = tiles[u / MT];
+      const int mt = u % MT;
+      const int a = it & 1;
+      mbar_wait_guarded(&tfull[a], (it >> 1) & 1, status, abort_flag);
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(warp * 32) << 16) + a * kAccCols;
+      const int n16 = (tl.n + 15) & ~15;
+      for (int c0 = 0; c0 < n16; c0 += 16) {
+        uint32_t g[16];
+        tmem_ld16(tb + c0, g);
+        if constexpr (MODE == 0) {
+          uint32_t uu[16];
+          tmem_ld16(tb + 128 + c0, uu);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < tl.n) {
+              const float gv = __uint_as_float(g[j]), uv = __uint_as_float(uu[j]);
+              const float h = silu_f32(gv) * uv;
+              out[(size_t)(tl.s0 + n) * I + mt * kPM + m] = __half_as_ushort(__float2half_rn(h));
+            }
+          }
+        } else {
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = c0 + j;
+            if (n < tl.n)
+              out[(size_t)(tl.s0 + n) * H + mt * kPM + m] =
+                  __half_as_ushort(__float2half_rn(__uint_as_float(g[j])));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[a]);
+    }
+  } else if (warp < 8) {
+    // ------------------------------------------------ producers
+    const int r = threadIdx.x - 128;  // weight row within the tile
+    const Q4Table T4 = q4_table();
+    const uint64_t crow = codes_row_bytes(FMT, K), srow = (uint64_t)(K / 32) * 2;
+    constexpr int PD = 4;
+    constexpr int NA = C::NA;
+    PChunk<FMT> ring[PD + 1][NA];
+    // prefetch cursor over (unit, chunk)
+    int pu = blockIdx.x, pk = 0;
+    const uint8_t *pc[NA], *ps[NA];
+    auto set_ptrs = [&](int u) {
+      if (u < total) {
+        const NTile tl = tiles[u / MT];
+        const int row = (u % MT) * kPM + r;
+        const uint8_t* blob = wbase + (uint64_t)tl.e * stride;
+#pragma unroll
+        for (int a = 0; a < NA; ++a) {
+          const int mat = (MODE == 0) ? a : 2;
+          pc[a] = blob + P.codes[mat] + (uint64_t)row * crow;
+          ps[a] = blob + P.scales[mat] + (uint64_t)row * srow;
+        }
+      }
+    };
+    set_ptrs(pu);
+    auto prefetch = [&](PChunk<FMT> (&slot)[NA]) {
+      if (pu < total) {
+#pragma unroll
+        for (int a = 0; a < NA; ++a) load_chunk<FMT>(slot[a], pc[a], ps[a], pk);
+        if (++pk == KC) {
+          pk = 0;
+          pu += gridDim.x;
+          set_ptrs(pu);
+        }
+      }
+    };
+#pragma unroll
+    for (int s = 0; s < PD; ++s) prefetch(ring[s]);
+    int it_k = 0;
+    int u = blockIdx.x, kc = 0;
+    NTile cur_tile = (u < total) ? tiles[u / MT] : NTile{0, 0, 0, 0};
+    int s0 = cur_tile.s0;
+    while (u < total) {
+#pragma unroll
+      for (int q = 0; q <= PD; ++q) {
+        if (u < total) {
+          prefetch(ring[(q + PD) % (PD + 1)]);
+          const int s = it_k % C::S;
+          mbar_wait_guarded(&empty[s], ((it_k / C::S) & 1) ^ 1, status, abort_flag);
+          uint8_t* stage = smem + s * C::SB;
+          if (r == 0) {
+            // B tile: expected bytes first, then the copy; the arrival comes
+            // with the other producers' after this thread's A row is stored
+            mbar_expect_tx(&full[s], kTileBytes);
+            tma_load_2d(stage + C::NA * kTileBytes, &bmap, kc * kPK, s0, &full[s]);
+          }
+#pragma unroll
+          for (int a = 0; a < NA; ++a) store_chunk<FMT>(ring[q][a], stage + a * kTileBytes, r, T4);
+          fence_proxy_async_smem();
+          mbar_arrive(&full[s]);
+          ++it_k;
+          if (++kc == KC) {
+            kc = 0;
+            u += gridDim.x;
+            if (u < total) cur_tile = tiles[u / MT];
+          }
+          s0 = cur_tile.s0;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------ MMA issue (one thread)
+    if (elect_one()) {
+      int it_k = 0, it = 0;
+      for (int u = blockIdx.x; u < total; u += gridDim.x, ++it) {
+        const NTile tl = tiles[u / MT];
+        const int n16 = (tl.n + 15) & ~15;
+        const uint32_t idesc = idesc_f16_f32(n16);
+        const int a = it & 1;
+        mbar_wait_guarded(&tempty[a], ((it >> 1) & 1) ^ 1, status, abort_flag);
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + a * kAccCols;
+        for (int kc = 0; kc < KC; ++kc, ++it_k) {
+          const int s = it_k % C::S;
+          mbar_wait_guarded(&full[s], (it_k / C::S) & 1, status, abort_flag);
+          tc_fence_after();
+          const uint32_t st = smem_addr(smem + s * C::SB);
+          const uint32_t bb = st + C::NA * kTileBytes;
+#pragma unroll
+          for (int kk = 0; kk < kPK / 16; ++kk) {
+            const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+            const uint64_t bdesc = smem_desc_k128(bb + kk * 32);
+            mma_f16_ss(d0, smem_desc_k128(st + kk * 32), bdesc, idesc, acc);
+            if constexpr (MODE == 0)
+              mma_f16_ss(d0 + 128, smem_desc_k128(st + kTileBytes + kk * 32), bdesc, idesc, acc);
+          }
+          mma_commit(&empty[s]);
+        }
+        mma_commit(&tfull[a]);
+      }
+      mma_commit(done);
+      // all MMAs retired before the tensor memory is released (bounded)
+      mbar_wait_bounded(done, 0, status);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 2 * kAccCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+struct PrefillWs {
+  uint64_t x, h, tiles, count, total;
+};
+
+PrefillWs prefill_ws(int T, int H, int I, int E, int k, int shared_mode) {
   const uint64_t P = shared_mode ? (uint64_t)T : (uint64_t)T * k;
-  return ((P * I * 2) + 255) & ~uint64_t(255);
+  const uint64_t max_tiles = (uint64_t)(shared_mode ? 1 : E) + P / kPN + 1;
+  auto up = [](uint64_t x) { return (x + 255) & ~uint64_t(255); };
+  PrefillWs w;
+  uint64_t off = 0;
+  w.x = off;
+  off = up(off + P * H * 2);
+  w.h = off;
+  off = up(off + P * I * 2);
+  w.tiles = off;
+  off = up(off + max_tiles * sizeof(NTile));
+  w.count = off;
+  off = up(off + 16);
+  w.total = off;
+  return w;
+}
+
+// The driver's tensor-map encoder, looked up through the runtime so the
+// library does not link against libcuda (it still loads where no driver is
+// installed; the entry point is resolved on first use on a GPU machine).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool make_map(CUtensorMap* map, const void* base, int cols, long long rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)kPN};
+  const cuuint32_t estr[2] = {1, 1};
+  EncodeTiledFn enc = encode_tiled();
+  if (!enc) return false;
+  const CUresult r = enc(
+      map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int MODE, int FMT>
+cudaError_t launch_gemm(const CUtensorMap& map, const PrefillArgs& a, const NTile* tiles,
+                        const int* count, uint16_t* out, cudaStream_t st) {
+  auto kern = prefill_gemm_kernel<MODE, FMT>;
+  const size_t smem = prefill_smem_bytes<MODE>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<a.num_sms, kPThreads, smem, st>>>(map, a.wbase, a.stride, a.H, a.I, tiles, count, out,
+                                          a.status);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+uint64_t prefill_workspace_bytes(int T, int H, int I, int E, int k, int shared_mode) {
+  return prefill_ws(T, H, I, E, k, shared_mode).total;
 }
 
 cudaError_t launch_experts_prefill(const PrefillArgs& a, cudaStream_t st) {
-  (void)a; (void)st;
-  return cudaErrorNotSupported;
+  if (a.H % kPM || a.I % kPM || a.H % kPK || a.I % kPK) return cudaErrorNotSupported;
+  const PrefillWs L = prefill_ws(a.T, a.H, a.I, a.E, a.k, a.shared_mode);
+  if (a.ws_bytes < L.total) return cudaErrorInvalidValue;
+  uint8_t* base = reinterpret_cast<uint8_t*>(a.ws);
+  uint16_t* X = reinterpret_cast<uint16_t*>(base + L.x);
+  uint16_t* h = reinterpret_cast<uint16_t*>(base + L.h);
+  NTile* tiles = reinterpret_cast<NTile*>(base + L.tiles);
+  int* count = reinterpret_cast<int*>(base + L.count);
+  const long long P = a.shared_mode ? a.T : (long long)a.T * a.k;
+  const int E = a.shared_mode ? 1 : a.E;
+  if (E > 1024) return cudaErrorNotSupported;
+  prefill_plan_kernel<<<1, 1024, 0, st>>>(a.offsets, E, a.shared_mode ? a.T : -1, tiles, count);
+  const long long work = P * (a.H / 8);
+  const int gblocks = (int)std::min<long long>((work + 255) / 256, (long long)a.num_sms * 16);
+  prefill_gather_kernel<<<gblocks, 256, 0, st>>>(a.hidden, a.shared_mode ? nullptr : a.perm,
+                                                 a.k, (int)P, a.T, a.H, X, a.status);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap mx, mh;
+  if (!make_map(&mx, X, a.H, P) || !make_map(&mh, h, a.I, P)) return cudaErrorInvalidValue;
+  if (a.fmt == STRATA_FMT_Q2_32) {
+    if ((e = launch_gemm<0, STRATA_FMT_Q2_32>(mx, a, tiles, count, h, st)) != cudaSuccess) return e;
+    return launch_gemm<1, STRATA_FMT_Q2_32>(mh, a, tiles, count, a.y, st);
+  }
+  if ((e = launch_gemm<0, STRATA_FMT_Q4CB_32>(mx, a, tiles, count, h, st)) != cudaSuccess) return e;
+  return launch_gemm<1, STRATA_FMT_Q4CB_32>(mh, a, tiles, count, a.y, st);
 }
 
 }  // namespace strata

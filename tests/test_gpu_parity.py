@@ -99,8 +99,9 @@ class Run:
 
 
 def check_layer(r: Run, sample=None):
-    """Full check of one run; sample = token indices for the expert/output
-    checks (all tokens if None)."""
+    """Full check of one run; `sample` = token indices for the router,
+    expert and output checks (all tokens if None).  Bucket and RMSNorm are
+    always checked on every token."""
     T, H, E, k = r.T, r.H, r.E, r.k
     hid = u16(r.hidden)
     # RMSNorm within one bf16 ulp
@@ -121,11 +122,10 @@ def check_layer(r: Run, sample=None):
     assert ok, f"routing mismatch on tokens {bad[:10]}"
     if near:
         print(f"near-tie tokens: {list(toks[near])}")
-    _, ref_w = oracle.topk(gl, k)
-    ref_ids_gpu_logits, _ = oracle.topk(gl, k)
+    ref_ids_gpu_logits, ref_w = oracle.topk(gl, k)
     np.testing.assert_array_equal(ref_ids_gpu_logits, gids[toks])
     assert np.abs(r.w.cpu().numpy()[toks] - ref_w).max() <= TOPK_W_ATOL
-    # bucket bit-exact on the GPU's ids
+    # bucket bit-exact on the GPU's ids (all tokens)
     counts, offsets, perm, inv = oracle.bucket(gids, E)
     np.testing.assert_array_equal(r.counts.cpu().numpy(), counts)
     np.testing.assert_array_equal(r.offsets.cpu().numpy(), offsets)
@@ -135,22 +135,25 @@ def check_layer(r: Run, sample=None):
     nz = np.nonzero(counts)[0]
     assert act[0] == len(nz)
     np.testing.assert_array_equal(act[1:1 + len(nz)], nz)
-    # combine bit-exact given the GPU's y
-    y = r.y.float().cpu().numpy()
-    yp = y[inv]
-    sh = None if r.shy is None else r.shy.float().cpu().numpy()
-    of, ob, _ = oracle.combine(yp, r.w.cpu().numpy(), sh)
-    np.testing.assert_array_equal(u16(r.out), ob)
-    np.testing.assert_array_equal(r.acc.cpu().numpy(), of)
-    # expert outputs and layer output vs the oracle on sampled tokens
+    # combine bit-exact given the GPU's y (sampled tokens)
+    rows = inv.reshape(T, k)[toks]
+    yg = r.y[torch.as_tensor(rows.reshape(-1), device=DEV).long()].float().cpu().numpy()
+    sh = None if r.shy is None else r.shy[torch.as_tensor(toks, device=DEV).long()].float().cpu().numpy()
+    of, ob, _ = oracle.combine(yg, r.w.cpu().numpy()[toks], sh)
+    np.testing.assert_array_equal(u16(r.out)[toks], ob)
+    np.testing.assert_array_equal(r.acc.cpu().numpy()[toks], of)
+    # expert outputs and the layer output vs the oracle (teacher-forced ids)
     blobs = r.blobs_for(gids[toks])
-    for t in toks:
+    for i, t in enumerate(toks):
         for j in range(k):
             e = int(gids[t, j])
             ref_y = oracle.expert_ffn(r.c.fmt, blobs[e], H, r.I, hid[t])
-            got = y[inv[t * k + j]]
-            assert rel_l2_rows(got, ref_y) <= OUT_REL_L2, (t, j, e)
+            assert rel_l2_rows(yg[i * k + j], ref_y) <= OUT_REL_L2, (int(t), j, e)
     sb = None if r.inp.shared is None else r.inp.shared[0].cpu().numpy()
+    if sb is not None:
+        for i, t in enumerate(toks):
+            ref_s = oracle.expert_ffn(r.c.shared_fmt, sb, H, r.I, hid[t])
+            assert rel_l2_rows(sh[i], ref_s) <= OUT_REL_L2, ("shared", int(t))
     ref = oracle.moe_layer(hid[toks], wr, bias, E, k, r.c.fmt, r.I, blobs,
                            shared_fmt=r.c.shared_fmt or 0, shared_blob=sb,
                            forced_ids=gids[toks])
@@ -259,3 +262,43 @@ def test_route_matches_separate_calls(config, T):
     assert torch.equal(perm, r.perm[:T * k]) and torch.equal(inv, r.inv[:T * k])
     nact = int(active[0])
     assert torch.equal(active[:1 + nact], r.active[:1 + nact])
+
+
+# ---------------------------------------------------------------- prefill (T > 16)
+@pytest.mark.parametrize("T,E", [(17, 16), (100, 16), (300, 16), (300, 512)])
+def test_prefill_ragged(T, E):
+    """Tensor-core path at sizes that span several 128-token tiles per expert
+    (E = 16: ~T*10/16 tokens each) and ragged tails, checked on every token."""
+    r = Run(1, T, E=E).run()
+    err = check_layer(r)
+    print(f"prefill T={T} E={E}: max rel L2 {err.max():.2e}")
+
+
+def test_prefill_one_expert_takes_everything():
+    """All tokens routed to one expert (k = 1, E = 2, a bias of +50 on expert 1):
+    a single expert with T tokens = many full tiles plus a tail."""
+    T = 1000
+    r = Run(1, T, E=2)
+    r.k = 1
+    r.inp.bias = torch.tensor([0.0, 50.0], device=DEV)
+    r.run()
+    assert int(r.counts[1]) == T
+    check_layer(r, sample=np.arange(0, T, 37))
+
+
+@pytest.mark.parametrize("config", [2, 3, 4])
+def test_prefill_full_size(config):
+    """The T = 8192 prefill chunks (2-bit routed; + 4-bit shared expert; 4-bit
+    large experts) at full size, checked on 24 sampled tokens."""
+    r = Run(config, 8192).run()
+    rng = np.random.default_rng(config)
+    sample = np.sort(rng.choice(8192, 24, replace=False))
+    err = check_layer(r, sample=sample)
+    print(f"C{config} T=8192: max rel L2 {err.max():.2e} over {len(sample)} tokens")
+
+
+def test_prefill_deterministic():
+    a = Run(2, 2048).run()
+    b = Run(2, 2048).run()
+    for x, y in ((a.ids, b.ids), (a.perm, b.perm), (a.y, b.y), (a.out, b.out)):
+        assert torch.equal(x, y)
