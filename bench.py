@@ -56,6 +56,14 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def sustained_tflops():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        return 1400.0
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -215,9 +223,8 @@ def run_ours(args):
     cfg = mi.CONFIGS[args.config]
     T = args.tokens or cfg.Ts[0]
     L = args.layers or cfg.layers
-    if T > 16:
-        raise SystemExit("this bench line covers the decode path (T <= 16)")
     stack = DecodeStack(args.config, T, L, dev)
+    prefill = T > stack.sm.DECODE_MAX_T
     H, E, k = stack.H, stack.E, stack.k
     G = min(args.steps, args.graphs)
     # distinct seeded inputs per graph, per rank
@@ -277,6 +284,8 @@ def run_ours(args):
             durs.append(events[g][l][0].elapsed_time(events[g][l][1]) * 1e-3)
             U = int(actives[g][l][0].item())
             bytes_.append(U * stack.ebytes + T * H * 2 + T * k * H * 4)
+    # prefill: algorithmic flops of the expert GEMMs (routed + shared)
+    flops = 6.0 * H * stack.I * T * k + (6.0 * H * stack.I * T if cfg.shared_fmt else 0.0)
     # end-to-end: pinned host input -> device, step, result -> pinned host
     hx = [xs[g].cpu().pin_memory() for g in range(G)]
     hout = [torch.empty(T, H, dtype=torch.float32).pin_memory() for _ in range(G)]
@@ -304,9 +313,12 @@ def run_ours(args):
     value = tokens / (ms * 1e-3)
     e2e = tokens / (e2e_ms * 1e-3)
     hbm, bf16, src = peaks()
+    bf16_sus = sustained_tflops()
     avg_dur = sum(durs) / len(durs)
     avg_bytes = sum(bytes_) / len(bytes_)
     achieved = avg_bytes / avg_dur / 1e9
+    if prefill:
+        achieved_tf = flops / avg_dur / 1e12
     traffic = None
     try:
         with open(NCU_TRAFFIC_FILE) as f:
@@ -332,19 +344,31 @@ def run_ours(args):
                        "parallelism": f"replicas x{ws_}",
                        "accumulate": "f32", "weights": "2.5 bits/weight" if cfg.fmt == 1 else "4.5 bits/weight",
                        "l2": "no flush: per-step weight stream (~%.1f GB) >> 126 MB L2"
-                             % (sum(bytes_[:L]) / 1e9),
+                             % (sum(bytes_[:L]) / 1e9) if not prefill else
+                             "no flush: per-step working set (weights + activations) > 1 GB",
                        "graphs": G},
             "e2e": {"value": round(e2e, 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4},
             "gpu_launches": kernels_per_layer(T, k, cfg.shared_fmt is not None) * L * args.steps,
-            "roofline": {"kernel": "moe_experts decode stage (gate/up + down kernels)",
-                         "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
-                         "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                         "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, burst)"
-                         if src == "measured" else "fallback 6.65 TB/s",
-                         "avg_launch_us": round(avg_dur * 1e6, 3),
-                         "algorithmic_bytes_per_launch": int(avg_bytes),
-                         "traffic": traffic},
+            "roofline": ({"kernel": "moe_experts decode stage (gate/up + down kernels)",
+                          "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                          "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                          "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, burst)"
+                          if src == "measured" else "fallback 6.65 TB/s",
+                          "avg_launch_us": round(avg_dur * 1e6, 3),
+                          "algorithmic_bytes_per_launch": int(avg_bytes),
+                          "traffic": traffic} if not prefill else
+                         {"kernel": "moe_experts prefill stage (plan, gather, tcgen05 gate/up "
+                                    "and down grouped GEMMs)",
+                          "bound": "tensor", "achieved": round(achieved_tf, 1),
+                          "peak": bf16_sus, "unit": "TFLOP/s",
+                          "frac": round(achieved_tf / bf16_sus, 4),
+                          "frac_of_burst": round(achieved_tf / bf16, 4),
+                          "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained (fp16 "
+                                         "kind::f16 runs at the bf16 rate)",
+                          "avg_launch_us": round(avg_dur * 1e6, 3),
+                          "algorithmic_flops_per_launch": flops,
+                          "traffic": traffic}),
             "clocks": clk,
         }
         if cpu is not None:
@@ -360,45 +384,65 @@ def run_ours(args):
 
 # ---------------------------------------------------------------- CPU side
 def oracle_sample(config, T, layers, device_stack=None, target_s=15.0, x0=None):
-    """Time the oracle over the first layers of the workload, one layer at a
-    time, until about target_s seconds of CPU work; returns (seconds per
-    layer, layers run, threads)."""
+    """Time the oracle on the workload until about target_s seconds of CPU
+    work: decode (T <= 16) runs whole layers of the stack in order; prefill
+    runs 16-token slices of the first layer.  Returns (tokens/s of the whole
+    workload, description, threads)."""
     import numpy as np
 
     import oracle
     c = mi.CONFIGS[config]
     x = (x0.cpu() if x0 is not None else mi.gen_x(T, c.H, mi.seed_for(config, 0, "xstep"))).numpy()
     spent, n = 0.0, 0
-    for l in range(layers):
+
+    def layer_inputs(l):
         if device_stack is not None:
             wr = device_stack.wr[l].cpu().view(torch.int16).numpy().view(np.uint16)
             bias = None if device_stack.bias[l] is None else device_stack.bias[l].cpu().numpy()
             blobs = device_stack.experts[l].cpu().numpy()
             sh = None if device_stack.shared[l] is None else device_stack.shared[l][0].cpu().numpy()
         else:
-            inp = mi.make_layer(config, T, layer=l, device="cpu")
+            inp = mi.make_layer(config, 1, layer=l, device="cpu")
             wr = inp.w_router.view(torch.int16).numpy().view(np.uint16)
             bias = None if inp.bias is None else inp.bias.numpy()
             blobs = inp.experts.numpy()
             sh = None if inp.shared is None else inp.shared[0].numpy()
+        return wr, bias, blobs, sh
+
+    if T <= 16:
+        for l in range(layers):
+            wr, bias, blobs, sh = layer_inputs(l)
+            t0 = time.perf_counter()
+            hid = oracle.rmsnorm(x, c.eps)
+            r = oracle.moe_layer(hid, wr, bias, c.E, c.k, c.fmt, c.I, blobs,
+                                 shared_fmt=c.shared_fmt or 0, shared_blob=sh, residual=x)
+            spent += time.perf_counter() - t0
+            n += 1
+            x = r["residual_out"]
+            if spent >= target_s:
+                break
+        per_layer = spent / n
+        return (T / (per_layer * layers),
+                f"{n} of {layers} layers, T={T}, scaled to a {layers}-layer step "
+                f"({per_layer:.3f} s per layer)", min(oracle.num_threads(), T))
+    wr, bias, blobs, sh = layer_inputs(0)
+    tok = 0
+    while spent < target_s and tok < T:
+        sl = x[tok:tok + 16]
         t0 = time.perf_counter()
-        hid = oracle.rmsnorm(x, c.eps)
-        r = oracle.moe_layer(hid, wr, bias, c.E, c.k, c.fmt, c.I, blobs,
-                             shared_fmt=c.shared_fmt or 0, shared_blob=sh, residual=x)
+        hid = oracle.rmsnorm(sl, c.eps)
+        oracle.moe_layer(hid, wr, bias, c.E, c.k, c.fmt, c.I, blobs,
+                         shared_fmt=c.shared_fmt or 0, shared_blob=sh, residual=sl)
         spent += time.perf_counter() - t0
-        n += 1
-        x = r["residual_out"]
-        if spent >= target_s:
-            break
-    return spent / n, n, min(oracle.num_threads(), T)
+        tok += sl.shape[0]
+    return (tok / (spent * layers), f"{tok} of {T} tokens of layer 0 in 16-token slices, "
+            f"scaled to {layers} layer(s)", min(oracle.num_threads(), 16))
 
 
 def cpu_baseline(stack, x0, args):
-    per_layer, n, cores = oracle_sample(args.config, stack.T, stack.L, stack, args.cpu_seconds, x0)
-    tok_s = stack.T / (per_layer * stack.L)
+    tok_s, desc, cores = oracle_sample(args.config, stack.T, stack.L, stack, args.cpu_seconds, x0)
     return {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} of {stack.L} layers, T={stack.T}, timed on host cores and scaled "
-                      f"to a {stack.L}-layer step ({per_layer:.3f} s per layer)"}
+            "sample": desc}
 
 
 def run_reference(args):

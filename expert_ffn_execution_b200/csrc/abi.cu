@@ -162,7 +162,7 @@ int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router, const 
                         int32_t T, int32_t H, int32_t E, int32_t k, int32_t* topk_ids,
                         float* topk_w, float* logits_opt, void* workspace, uint64_t ws_bytes,
                         int32_t* dev_status, void* stream) {
-  if (T < 0 || H < 64 || H % 64 || E < 2 || E > 1024 || E % 2 || k < 1 || k > E || k > 32)
+  if (T < 0 || H < 64 || H % 64 || E < 8 || E > 1024 || E % 8 || k < 1 || k > E || k > 32)
     return STRATA_EINVAL;
   if (T == 0) return STRATA_OK;
   if (!hidden || !w_router || !topk_ids || !topk_w || !workspace) return STRATA_EINVAL;
@@ -201,7 +201,7 @@ int32_t moe_route(const float* x, int32_t T, int32_t H, float eps, const uint16_
                   float* topk_w, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                   int32_t* active, void* workspace, uint64_t ws_bytes, int32_t* dev_status,
                   void* stream) {
-  if (T < 0 || H < 64 || H % 64 || H > 16384 || E < 2 || E > 1024 || E % 2 || k < 1 || k > E ||
+  if (T < 0 || H < 64 || H % 64 || H > 16384 || E < 8 || E > 1024 || E % 8 || k < 1 || k > E ||
       k > 32 || !(eps >= 0.f))
     return STRATA_EINVAL;
   if (T == 0) return STRATA_OK;

@@ -108,36 +108,52 @@ bucket_hist(const int32_t* __restrict__ ids, int P, int E, int32_t* __restrict__
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(size_t)blockIdx.x * E + e] = sh[e];
 }
 
+// One warp per expert: exclusive prefix over the chunks' counts (in place),
+// so hist[g][e] becomes the number of the expert's pairs in chunks < g.
+__global__ void __launch_bounds__(256)
+bucket_colscan(int32_t* __restrict__ hist, int G, int E, int32_t* __restrict__ counts) {
+  const int e = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (e >= E) return;
+  const int per = (G + 31) / 32;
+  const int g0 = lane * per, g1 = min(G, g0 + per);
+  int mine = 0;
+  for (int g = g0; g < g1; ++g) mine += hist[(size_t)g * E + e];
+  int x = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  int run = x - mine;
+  for (int g = g0; g < g1; ++g) {
+    const int h = hist[(size_t)g * E + e];
+    hist[(size_t)g * E + e] = run;
+    run += h;
+  }
+  if (lane == 31) counts[e] = x;
+}
+
+// One CTA: offsets = exclusive scan of counts, and the active-expert list.
 __global__ void __launch_bounds__(kBucketThreads)
-bucket_scan(int32_t* __restrict__ hist, int G, int E, int32_t* __restrict__ counts,
-            int32_t* __restrict__ offsets, int32_t* __restrict__ active) {
+bucket_offsets(const int32_t* __restrict__ counts, int E, int32_t* __restrict__ offsets,
+               int32_t* __restrict__ active) {
   __shared__ int swarp[32];
   const int e = threadIdx.x;
-  int run = 0;
-  if (e < E) {
-    for (int g = 0; g < G; ++g) {
-      const int h = hist[(size_t)g * E + e];
-      hist[(size_t)g * E + e] = run;
-      run += h;
-    }
-  }
+  const int c = (e < E) ? counts[e] : 0;
   int total = 0;
-  const int off = block_excl_scan(e < E ? run : 0, swarp, &total);
-  if (e < E) {
-    counts[e] = run;
-    offsets[e] = off;
-    for (int g = 0; g < G; ++g) hist[(size_t)g * E + e] += off;
-  }
+  const int off = block_excl_scan(c, swarp, &total);
+  if (e < E) offsets[e] = off;
   if (e == 0) offsets[E] = total;
   int nact = 0;
-  const int apos = block_excl_scan((e < E && run > 0) ? 1 : 0, swarp, &nact);
-  if (e < E && run > 0) active[1 + apos] = e;
+  const int apos = block_excl_scan((e < E && c > 0) ? 1 : 0, swarp, &nact);
+  if (e < E && c > 0) active[1 + apos] = e;
   if (e == 0) active[0] = nact;
 }
 
 __global__ void __launch_bounds__(kChunk)
 bucket_scatter(const int32_t* __restrict__ ids, int P, int E, const int32_t* __restrict__ base,
-               int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+               const int32_t* __restrict__ offsets, int32_t* __restrict__ perm,
+               int32_t* __restrict__ inv) {
   __shared__ int sid[kChunk];
   const int p = blockIdx.x * kChunk + threadIdx.x;
   int e = -1;
@@ -150,7 +166,7 @@ bucket_scatter(const int32_t* __restrict__ ids, int P, int E, const int32_t* __r
   if (e >= 0) {
     int rank = 0;
     for (int i = 0; i < (int)threadIdx.x; ++i) rank += (sid[i] == e);
-    const int pos = base[(size_t)blockIdx.x * E + e] + rank;
+    const int pos = offsets[e] + base[(size_t)blockIdx.x * E + e] + rank;
     perm[pos] = p;
     inv[p] = pos;
   } else if (p < P) {
@@ -177,8 +193,9 @@ cudaError_t launch_bucket(const int32_t* ids, int T, int k, int E, int32_t* coun
   const int G = (P + kChunk - 1) / kChunk;
   int32_t* hist = reinterpret_cast<int32_t*>(ws);
   bucket_hist<<<G, kChunk, E * sizeof(int), st>>>(ids, P, E, hist, status);
-  bucket_scan<<<1, kBucketThreads, 0, st>>>(hist, G, E, counts, offsets, active);
-  bucket_scatter<<<G, kChunk, 0, st>>>(ids, P, E, hist, perm, inv);
+  bucket_colscan<<<(E + 7) / 8, 256, 0, st>>>(hist, G, E, counts);
+  bucket_offsets<<<1, kBucketThreads, 0, st>>>(counts, E, offsets, active);
+  bucket_scatter<<<G, kChunk, 0, st>>>(ids, P, E, hist, offsets, perm, inv);
   return cudaGetLastError();
 }
 

@@ -23,11 +23,12 @@
 // GEMM kernel, one CTA per SM, persistent over units (static round robin over
 // the size-sorted list), warp-specialised:
 //   warps 0-3  epilogue: tcgen05.ld of their TMEM lane quarter, math, stores
-//   warps 4-7  producers: one weight row per thread; codes and scales are
-//              prefetched four K-chunks ahead in registers, decoded to fp16
+//   warps 4-11 producers, two groups of four warps taking alternate K chunks
+//              (stages); one weight row per thread; codes and scales are
+//              prefetched four chunks ahead in registers, decoded to fp16
 //              and stored into the 128-byte-swizzled K-major stage layout;
-//              producer thread 0 also issues the TMA load of the B tile
-//   warp 8     tensor memory allocation and the single MMA-issuing thread
+//              thread 0 of a group also issues the TMA load of the B tile
+//   warp 12    tensor memory allocation and the single MMA-issuing thread
 // Stages are guarded by mbarriers (full: producers + TMA bytes; empty:
 // tcgen05.commit), accumulators by tmem_full/tmem_empty.  Every wait is
 // bounded (clock budget) and reports STRATA_DEV_TIMEOUT instead of hanging.
@@ -41,7 +42,7 @@ namespace strata {
 constexpr int kPM = 128;       // weight rows per tile (MMA M)
 constexpr int kPN = 128;       // tokens per n-tile (MMA N <= 128)
 constexpr int kPK = 64;        // K per stage: one 128-byte swizzle row of fp16
-constexpr int kPThreads = 9 * 32;
+constexpr int kPThreads = 13 * 32;  // 4 epilogue + 8 producer + 1 MMA warps
 constexpr int kTileBytes = kPM * kPK * 2;  // 16 KB per operand tile
 constexpr int kAccCols = 256;              // TMEM columns per accumulator set
 
@@ -225,7 +226,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(tmem_slot, 2 * kAccCols);
     tmem_relinquish();
   }
@@ -277,55 +278,57 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
       tc_fence_before();
       mbar_arrive(&tempty[a]);
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------ producers
-    const int r = threadIdx.x - 128;  // weight row within the tile
+    const int pg = (warp - 4) >> 2;   // group: takes chunks j = pg, pg + 2, ...
+    const int r = threadIdx.x & 127;  // weight row within the tile
     const Q4Table T4 = q4_table();
     const uint64_t crow = codes_row_bytes(FMT, K), srow = (uint64_t)(K / 32) * 2;
-    constexpr int PD = 4;
     constexpr int NA = C::NA;
+    constexpr int PD = (FMT == STRATA_FMT_Q4CB_32 && NA == 2) ? 3 : 4;  // register budget
+    const int nunits = (total > (int)blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    const int nchunks = nunits * KC;
+    // flat chunk sequence of this CTA: j -> unit blockIdx.x + (j / KC) * grid, chunk j % KC
     PChunk<FMT> ring[PD + 1][NA];
-    // prefetch cursor over (unit, chunk)
-    int pu = blockIdx.x, pk = 0;
+    int jp = pg, p_ui = -1;
     const uint8_t *pc[NA], *ps[NA];
-    auto set_ptrs = [&](int u) {
-      if (u < total) {
-        const NTile tl = tiles[u / MT];
-        const int row = (u % MT) * kPM + r;
-        const uint8_t* blob = wbase + (uint64_t)tl.e * stride;
-#pragma unroll
-        for (int a = 0; a < NA; ++a) {
-          const int mat = (MODE == 0) ? a : 2;
-          pc[a] = blob + P.codes[mat] + (uint64_t)row * crow;
-          ps[a] = blob + P.scales[mat] + (uint64_t)row * srow;
-        }
-      }
-    };
-    set_ptrs(pu);
     auto prefetch = [&](PChunk<FMT> (&slot)[NA]) {
-      if (pu < total) {
+      if (jp < nchunks) {
+        const int ui = jp / KC, kc = jp - ui * KC;
+        if (ui != p_ui) {
+          p_ui = ui;
+          const int u = blockIdx.x + ui * gridDim.x;
+          const NTile tl = tiles[u / MT];
+          const int row = (u % MT) * kPM + r;
+          const uint8_t* blob = wbase + (uint64_t)tl.e * stride;
 #pragma unroll
-        for (int a = 0; a < NA; ++a) load_chunk<FMT>(slot[a], pc[a], ps[a], pk);
-        if (++pk == KC) {
-          pk = 0;
-          pu += gridDim.x;
-          set_ptrs(pu);
+          for (int a = 0; a < NA; ++a) {
+            const int mat = (MODE == 0) ? a : 2;
+            pc[a] = blob + P.codes[mat] + (uint64_t)row * crow;
+            ps[a] = blob + P.scales[mat] + (uint64_t)row * srow;
+          }
         }
+#pragma unroll
+        for (int a = 0; a < NA; ++a) load_chunk<FMT>(slot[a], pc[a], ps[a], kc);
+        jp += 2;
       }
     };
 #pragma unroll
     for (int s = 0; s < PD; ++s) prefetch(ring[s]);
-    int it_k = 0;
-    int u = blockIdx.x, kc = 0;
-    NTile cur_tile = (u < total) ? tiles[u / MT] : NTile{0, 0, 0, 0};
-    int s0 = cur_tile.s0;
-    while (u < total) {
+    int c_ui = -1, s0 = 0;
+    for (int j0 = pg; j0 < nchunks; j0 += 2 * (PD + 1)) {
 #pragma unroll
       for (int q = 0; q <= PD; ++q) {
-        if (u < total) {
+        const int j = j0 + 2 * q;
+        if (j < nchunks) {
           prefetch(ring[(q + PD) % (PD + 1)]);
-          const int s = it_k % C::S;
-          mbar_wait_guarded(&empty[s], ((it_k / C::S) & 1) ^ 1, status, abort_flag);
+          const int ui = j / KC, kc = j - ui * KC;
+          if (ui != c_ui) {
+            c_ui = ui;
+            s0 = tiles[(blockIdx.x + ui * gridDim.x) / MT].s0;
+          }
+          const int s = j % C::S;
+          mbar_wait_guarded(&empty[s], ((j / C::S) & 1) ^ 1, status, abort_flag);
           uint8_t* stage = smem + s * C::SB;
           if (r == 0) {
             // B tile: expected bytes first, then the copy; the arrival comes
@@ -337,13 +340,6 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
           for (int a = 0; a < NA; ++a) store_chunk<FMT>(ring[q][a], stage + a * kTileBytes, r, T4);
           fence_proxy_async_smem();
           mbar_arrive(&full[s]);
-          ++it_k;
-          if (++kc == KC) {
-            kc = 0;
-            u += gridDim.x;
-            if (u < total) cur_tile = tiles[u / MT];
-          }
-          s0 = cur_tile.s0;
         }
       }
     }
@@ -385,7 +381,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * kAccCols);
   }

@@ -10,7 +10,7 @@
 // and a second kernel sums the slices in a fixed order (deterministic) and
 // runs the top-k.  T > 16: a tiled GEMM writes the logits, then the same
 // top-k kernel runs with a single slice.
-#include "decode.cuh"
+#include "routing.cuh"
 
 namespace strata {
 
@@ -86,53 +86,123 @@ router_gemv_partial(const uint16_t* __restrict__ hidden, const uint16_t* __restr
   }
 }
 
-// Tiled fp32 GEMM for large T: 64 tokens x 128 experts per CTA.
-constexpr int kGBM = 64, kGBN = 128, kGBK = 32;
+// Large T: logits = hidden . W_r (+ bias) on mma.sync (bf16 in, fp32
+// accumulate).  CTA tile 128 tokens x 128 experts, K steps of 32 staged with
+// cp.async (double buffered, padded rows so every ldmatrix is conflict-free);
+// 8 warps as 4 (tokens) x 2 (experts), each 32 x 64.
+constexpr int kGBM = 128, kGBN = 128, kGBK = 32;
+constexpr int kGAS = kGBK + 8;   // A row stride (bf16)
+constexpr int kGBS = kGBN + 8;   // B row stride (bf16)
+
+STRATA_DEVFN void cp_async16(void* dst, const void* src, bool pred) {
+  const uint32_t d = smem_addr(dst);
+  const int n = pred ? 16 : 0;  // zero-fill when out of range
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(n)
+               : "memory");
+}
+STRATA_DEVFN void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+STRATA_DEVFN void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+STRATA_DEVFN void ldsm_x4(uint32_t (&r)[4], const void* p) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_addr(p)));
+}
+
 __global__ void __launch_bounds__(256)
-router_gemm(const uint16_t* __restrict__ hidden, const uint16_t* __restrict__ wr, int T, int H,
-            int E, float* __restrict__ logits) {
-  __shared__ float As[kGBK][kGBM + 4];
-  __shared__ float Bs[kGBK][kGBN + 4];
+router_gemm_mma(const uint16_t* __restrict__ hidden, const uint16_t* __restrict__ wr,
+                const float* __restrict__ bias, int T, int H, int E, float* __restrict__ logits) {
+  __shared__ __align__(16) uint16_t As[2][kGBM * kGAS];
+  __shared__ __align__(16) uint16_t Bs[2][kGBK * kGBS];
   const int m0 = blockIdx.x * kGBM, n0 = blockIdx.y * kGBN;
-  const int tx = threadIdx.x % 16, ty = threadIdx.x / 16;  // 16 x 16 threads, 4 x 8 outputs each
-  float acc[4][8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
-  for (int k0 = 0; k0 < H; k0 += kGBK) {
-    for (int i = threadIdx.x; i < kGBM * kGBK; i += 256) {
-      const int m = i / kGBK, kk = i % kGBK;
-      As[kk][m] = (m0 + m < T) ? bf16_bits_to_float(hidden[(size_t)(m0 + m) * H + k0 + kk]) : 0.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wm = warp >> 1, wn = warp & 1;  // 4 x 2 warps
+  auto load = [&](int buf, int k0) {
+    // A: 128 rows x 32 bf16 = 512 16-byte pieces; B: 32 rows x 128 bf16 = 512 pieces
+    for (int i = threadIdx.x; i < kGBM * (kGBK / 8); i += 256) {
+      const int r = i / (kGBK / 8), c = i % (kGBK / 8);
+      const int m = m0 + r;
+      cp_async16(&As[buf][r * kGAS + c * 8], hidden + (size_t)min(m, T - 1) * H + k0 + c * 8, m < T);
     }
-    for (int i = threadIdx.x; i < kGBK * kGBN; i += 256) {
-      const int kk = i / kGBN, n = i % kGBN;
-      Bs[kk][n] = (n0 + n < E) ? bf16_bits_to_float(wr[(size_t)(k0 + kk) * E + n0 + n]) : 0.f;
+    for (int i = threadIdx.x; i < kGBK * (kGBN / 8); i += 256) {
+      const int r = i / (kGBN / 8), c = i % (kGBN / 8);
+      const int n = n0 + c * 8;
+      cp_async16(&Bs[buf][r * kGBS + c * 8], wr + (size_t)(k0 + r) * E + min(n, E - 8), n < E);
+    }
+    cp_async_commit();
+  };
+  float acc[2][8][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][j][c] = 0.f;
+  const int nk = H / kGBK;
+  load(0, 0);
+  for (int kt = 0; kt < nk; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nk) {
+      load(buf ^ 1, (kt + 1) * kGBK);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
-#pragma unroll 4
-    for (int kk = 0; kk < kGBK; ++kk) {
-      float a[4], b[8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) a[i] = As[kk][ty * 4 + i];
+    for (int ks = 0; ks < kGBK / 16; ++ks) {
+      uint32_t a[2][4];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) b[j] = Bs[kk][tx * 8 + j];
+      for (int i = 0; i < 2; ++i) {
+        const int r = wm * 32 + i * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int c = ks * 16 + (lane >> 4) * 8;
+        ldsm_x4(a[i], &As[buf][r * kGAS + c]);
+      }
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+      for (int j = 0; j < 4; ++j) {  // pairs of n8 tiles
+        uint32_t b[4];
+        const int r = ks * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        const int c = wn * 64 + j * 16 + (lane >> 4) * 8;
+        ldsm_x4_trans(b, &Bs[buf][r * kGBS + c]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        for (int i = 0; i < 2; ++i) {
+          mma_16816_bf16(acc[i][2 * j], a[i], b[0], b[1]);
+          mma_16816_bf16(acc[i][2 * j + 1], a[i], b[2], b[3]);
+        }
+      }
     }
     __syncthreads();
   }
+  const int g = lane >> 2, q = lane & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + ty * 4 + i;
-    if (m >= T) continue;
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int n = n0 + tx * 8 + j;
-      if (n < E) logits[(size_t)m * E + n] = acc[i][j];
-    }
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int m = m0 + wm * 32 + i * 16 + g + (c >> 1) * 8;
+        const int n = n0 + wn * 64 + j * 8 + 2 * q + (c & 1);
+        if (m < T && n < E) logits[(size_t)m * E + n] = acc[i][j][c] + (bias ? bias[n] : 0.f);
+      }
+}
+
+// Large T: one warp per token, top-k straight from the logits in memory.
+template <int NPL>
+__global__ void __launch_bounds__(256)
+router_topk_warps(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ ids,
+                  float* __restrict__ w, float* __restrict__ logits_opt) {
+  const int t = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (t >= T) return;
+  const float* lg = logits + (size_t)t * E;
+  if (logits_opt)
+    for (int e = lane; e < E; e += 32) logits_opt[(size_t)t * E + e] = lg[e];
+  int id;
+  float wt;
+  warp_topk<NPL>(lg, E, k, id, wt);
+  if (lane < k) {
+    ids[(size_t)t * k + lane] = id;
+    w[(size_t)t * k + lane] = wt;
   }
 }
 
@@ -163,49 +233,12 @@ router_finish(const float* __restrict__ partial, int nslices, int T, int E, int 
   }
   __syncthreads();
   if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
-  float v[NPL];
-  uint32_t taken = 0;
-#pragma unroll
-  for (int j = 0; j < NPL; ++j) {
-    const int e = lane + 32 * j;
-    v[j] = (e < E) ? lg[e] : -INFINITY;
-    if (e >= E) taken |= 1u << j;
-  }
-  float lmax = 0.f, sum = 0.f, my_l = 0.f;
-  int my_id = -1;
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
-#pragma unroll
-    for (int j = 0; j < NPL; ++j) {
-      const int e = lane + 32 * j;
-      if (!(taken & (1u << j)) && (v[j] > bv || (v[j] == bv && e < bi))) {
-        bv = v[j];
-        bi = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (r == 0) lmax = bv;
-    const float ex = expf(bv - lmax);
-    sum += ex;
-    if (lane == r) {
-      my_id = bi;
-      my_l = ex;
-    }
-  }
-  if (lane < k) {
-    ids[(size_t)t * k + lane] = (my_id < E) ? my_id : -1;
-    w[(size_t)t * k + lane] = my_l / sum;
+  int id;
+  float wt;
+  warp_topk<NPL>(lg, E, k, id, wt);
+  if (threadIdx.x < k) {
+    ids[(size_t)t * k + threadIdx.x] = id;
+    w[(size_t)t * k + threadIdx.x] = wt;
   }
 }
 
@@ -232,7 +265,17 @@ cudaError_t launch_router_topk(const uint16_t* hidden, const uint16_t* wr, const
     router_gemv_partial<<<grid, 256, 0, st>>>(hidden, wr, T, H, E, part);
   } else {
     dim3 grid((T + kGBM - 1) / kGBM, (E + kGBN - 1) / kGBN);
-    router_gemm<<<grid, 256, 0, st>>>(hidden, wr, T, H, E, part);
+    router_gemm_mma<<<grid, 256, 0, st>>>(hidden, wr, bias, T, H, E, part);
+    cudaError_t err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const int blocks = (T + 7) / 8;
+    if (E <= 256)
+      router_topk_warps<8><<<blocks, 256, 0, st>>>(part, T, E, k, ids, w, logits_opt);
+    else if (E <= 512)
+      router_topk_warps<16><<<blocks, 256, 0, st>>>(part, T, E, k, ids, w, logits_opt);
+    else
+      router_topk_warps<32><<<blocks, 256, 0, st>>>(part, T, E, k, ids, w, logits_opt);
+    return cudaGetLastError();
   }
   cudaError_t err = cudaGetLastError();
   if (err != cudaSuccess) return err;

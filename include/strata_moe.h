@@ -143,7 +143,7 @@ STRATA_API int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps,
  *   hidden    bf16 [T,H];  w_router bf16 [H,E] row-major;  bias fp32 [E] or NULL
  *   topk_ids  int32 [T,k] out;  topk_w fp32 [T,k] out
  *   logits_opt fp32 [T,E] out, or NULL
- * Limits: 1 <= k <= min(E, 32); E even, 2..1024; H multiple of 64. */
+ * Limits: 1 <= k <= min(E, 32); E a multiple of 8, 8..1024; H multiple of 64. */
 STRATA_API uint64_t moe_router_topk_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
 STRATA_API int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router,
                         const float* bias, int32_t T, int32_t H, int32_t E,

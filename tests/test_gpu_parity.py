@@ -275,12 +275,12 @@ def test_prefill_ragged(T, E):
 
 
 def test_prefill_one_expert_takes_everything():
-    """All tokens routed to one expert (k = 1, E = 2, a bias of +50 on expert 1):
+    """All tokens routed to one expert (k = 1, E = 8, a bias of +50 on expert 1):
     a single expert with T tokens = many full tiles plus a tail."""
     T = 1000
-    r = Run(1, T, E=2)
+    r = Run(1, T, E=8)
     r.k = 1
-    r.inp.bias = torch.tensor([0.0, 50.0], device=DEV)
+    r.inp.bias = torch.tensor([0.0, 50.0, 0, 0, 0, 0, 0, 0], device=DEV)
     r.run()
     assert int(r.counts[1]) == T
     check_layer(r, sample=np.arange(0, T, 37))
