@@ -55,6 +55,7 @@ _SIGS = {
                        _P, _P]),
     "moe_experts_workspace_size": (_U64, [_QW, _I, _I]),
     "moe_experts": (_I, [_P, _QW, _P, _P, _P, _I, _I, _P, _P, _U64, _P, _P]),
+    "moe_experts_static_scratch": (_I, [_P, _QW, _P, _P, _P, _I, _I, _P, _P, _P]),
     "moe_shared_expert_workspace_size": (_U64, [_QW, _I]),
     "moe_shared_expert": (_I, [_P, _QW, _I, _P, _P, _U64, _P, _P]),
     "moe_combine": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P]),
@@ -187,6 +188,14 @@ def moe_experts(hidden, w: QWeights, offsets, perm, active, T, k, y, workspace, 
     rc = load().moe_experts(_ptr(hidden), _qw(w), _ptr(offsets), _ptr(perm), _ptr(active), T, k,
                             _ptr(y), _ptr(workspace), ws_bytes, _ptr(dev_status), _stream(stream))
     return _check("moe_experts", rc) if check else rc
+
+
+def moe_experts_static_scratch(hidden, w: QWeights, offsets, perm, active, T, k, y, dev_status,
+                               stream=None, check=True):
+    rc = load().moe_experts_static_scratch(_ptr(hidden), _qw(w), _ptr(offsets), _ptr(perm),
+                                           _ptr(active), T, k, _ptr(y), _ptr(dev_status),
+                                           _stream(stream))
+    return _check("moe_experts_static_scratch", rc) if check else rc
 
 
 def moe_shared_expert_workspace_size(w: QWeights, T) -> int:

@@ -1,6 +1,7 @@
 // abi.cu -- extern "C" entry points of libstrata_moe.so: argument checks,
 // workspace carving and kernel launches.  See include/strata_moe.h.
 #include <algorithm>
+#include <mutex>
 
 #include "decode.cuh"
 
@@ -409,3 +410,61 @@ int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router, c
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- static-scratch experts
+// moe_experts_static_scratch: the decode path of moe_experts with its scratch
+// in a fixed array inside the library instead of a caller's workspace.  It
+// serves callers that cannot hand the library device memory: a plain-C host
+// with no device allocator of its own, or a serving process that has claimed
+// all free HBM up front (weights plus a cache pool), where a cudaMalloc in the
+// middle of a step would fail and a cudaFree would synchronise the device.
+// The call allocates nothing: no cudaMalloc, cudaFree or allocating library
+// routine.  Its only scratch is the fp16 SwiGLU activation h [T*k, I].
+//
+// Every call on a device shares the one array, which keeps the last call's
+// contents.  Nothing in it must start at zero: the down kernel reads only the
+// h rows that the gate/up kernel of the same call wrote.  Calls whose kernels
+// overlap on the GPU (other streams, other host threads) race on the array.
+namespace {
+constexpr uint64_t kStaticScratchBytes = 2ull << 20;  // T*k*I <= 1,048,576 fp16
+}  // namespace
+
+static __device__ __align__(256) uint8_t g_experts_static_scratch[kStaticScratchBytes];
+
+namespace {
+std::mutex g_static_scratch_mu;
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device, looked up once per
+// device (with that device current) and cached; nullptr if the lookup fails.
+void* static_scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress((void**)&ptr, g_experts_static_scratch);
+    if (e != cudaSuccess || !ptr) return nullptr;
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  return g_static_scratch_ptr[dev];
+}
+}  // namespace
+
+extern "C" int32_t moe_experts_static_scratch(const uint16_t* hidden, const strata_qweights* w,
+                                              const int32_t* offsets, const int32_t* perm,
+                                              const int32_t* active, int32_t T, int32_t k,
+                                              float* y, int32_t* dev_status, void* stream) {
+  if (!valid_weights(w) || T < 0 || k < 1 || k > w->num_experts || k > 32) return STRATA_EINVAL;
+  if (w->num_experts > 1024) return STRATA_EINVAL;
+  // sizes beyond the array (or beyond the decode path) are rejected up front
+  if (T > kDecodeMaxTokens || (uint64_t)T * k * w->inter * 2 > kStaticScratchBytes)
+    return STRATA_EUNSUPPORTED;
+  if (T == 0) return STRATA_OK;
+  if (!hidden || !offsets || !perm || !active || !y) return STRATA_EINVAL;
+  if (!aligned(hidden, 16) || !aligned(y, 16)) return STRATA_EINVAL;
+  void* scratch = static_scratch_on_current_device();
+  if (!scratch) return STRATA_ECUDA;
+  return run_experts(hidden, w, offsets, perm, active, T, k, y, scratch, kStaticScratchBytes,
+                     dev_status, reinterpret_cast<cudaStream_t>(stream), 0);
+}

@@ -202,6 +202,31 @@ STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
                     void* workspace, uint64_t ws_bytes, int32_t* dev_status,
                     void* stream);
 
+/* moe_experts on the decode path (T <= STRATA_DECODE_MAX_T) without a
+ * workspace argument.  The paper has no counterpart of this call.  It is for
+ * callers that cannot give the library device memory: a plain-C host with no
+ * device allocator of its own, or a process that has already claimed all free
+ * HBM (weights plus a cache pool), where a cudaMalloc during a step would fail
+ * and a cudaFree would synchronise the device.  The call allocates nothing (no
+ * cudaMalloc, cudaFree or allocating library routine); its scratch, the fp16
+ * activations h [T*k, I], lives in one file-scope 2 MiB array of the library.
+ *   Limit: T <= STRATA_DECODE_MAX_T and T*k*I <= 1,048,576 (2 MiB of fp16);
+ *   beyond it the call returns STRATA_EUNSUPPORTED and launches nothing.
+ *   Set-up: the first call on each device, with that device current, looks
+ *   up the array's device address (cudaGetSymbolAddress) and caches it; make
+ *   that first call before any stream capture.  A failed lookup returns
+ *   STRATA_ECUDA.
+ *   Sharing: all calls on a device use the same array, which keeps the last
+ *   call's contents; no part of it has to start at zero (each call reads only
+ *   the h rows it wrote).  Calls that overlap on the GPU (other streams, other
+ *   host threads) race on the array: serialise them.
+ * Other arguments, the output y (fp32 [T*k, H], sorted order) and the other
+ * errors are those of moe_experts. */
+STRATA_API int32_t moe_experts_static_scratch(const uint16_t* hidden, const strata_qweights* w,
+                                   const int32_t* offsets, const int32_t* perm,
+                                   const int32_t* active, int32_t T, int32_t k, float* y,
+                                   int32_t* dev_status, void* stream);
+
 /* Shared expert: the same SwiGLU FFN with one always-on expert (w->num_experts
  * == 1) applied to every token, y[t] = FFN(hidden[t]); y [T,H] in token order,
  * fp32 for T <= STRATA_DECODE_MAX_T, fp16 otherwise.  The shared expert is
