@@ -71,6 +71,27 @@ def dist_env():
     return ws, rank, local
 
 
+def replica_input_seed(config, rank, g):
+    """Seed of input batch g on a rank: every replica runs its own tokens."""
+    return mi.seed_for(config, 1000 * rank + g, "xstep")
+
+
+def max_over_ranks(values, device):
+    """Element-wise max of `values` over all ranks (the slowest rank sets the
+    job's time); the values themselves with one rank."""
+    dist = torch.distributed
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(tokens_per_step_per_rank, steps, world, ms):
+    """Whole-job throughput: the tokens all ranks processed / the job time."""
+    return tokens_per_step_per_rank * steps * world / (ms * 1e-3)
+
+
 class Clocks:
     """Samples nvidia-smi clocks and throttle reasons during the timed region."""
 
@@ -228,7 +249,7 @@ def run_ours(args):
     H, E, k = stack.H, stack.E, stack.k
     G = min(args.steps, args.graphs)
     # distinct seeded inputs per graph, per rank
-    xs = [mi.gen_x(T, H, mi.seed_for(args.config, 1000 * rank + g, "xstep"), dev, cfg.x_bf16)
+    xs = [mi.gen_x(T, H, replica_input_seed(args.config, rank, g), dev, cfg.x_bf16)
           for g in range(G)]
     x_out = [torch.empty(T, H, dtype=torch.float32, device=dev) for _ in range(G)]
     actives = [[torch.empty(E + 1, dtype=torch.int32, device=dev) for _ in range(L)]
@@ -305,13 +326,9 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1)
     if int(stack.status.item()) != 0:
         raise SystemExit(f"device status {int(stack.status.item())}")
-    if ws_ > 1:
-        t = torch.tensor([ms, e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms, e2e_ms = float(t[0]), float(t[1])
-    tokens = T * args.steps * ws_
-    value = tokens / (ms * 1e-3)
-    e2e = tokens / (e2e_ms * 1e-3)
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], dev)
+    value = job_tokens_per_s(T, args.steps, ws_, ms)
+    e2e = job_tokens_per_s(T, args.steps, ws_, e2e_ms)
     hbm, bf16, src = peaks()
     bf16_sus = sustained_tflops()
     avg_dur = sum(durs) / len(durs)
