@@ -228,10 +228,15 @@ class DecodeStack:
 
 
 def kernels_per_layer(T, k, shared):
-    """Kernel launches the library enqueues per layer on the decode path:
-    moe_route 1 (one cluster kernel: RMSNorm, router, top-k, bucket),
-    experts 2 (gate/up, down), shared expert 2, combine 1."""
-    return 1 + 2 + 1 + (2 if shared else 0)
+    """Kernel launches the library enqueues per layer.  Decode (T <= 16):
+    moe_route 2 (logits with RMSNorm; top-k and bucket), experts 2 (gate/up,
+    down), shared expert 2, combine 1.  Prefill: moe_route 7 (RMSNorm,
+    router GEMM, top-k, bucket histogram, column scan, offsets, scatter),
+    experts 4 (plan, gather, gate/up GEMM, down GEMM), shared expert 4,
+    combine 1."""
+    if T <= 16:
+        return 2 + 2 + 1 + (2 if shared else 0)
+    return 7 + 4 + 1 + (4 if shared else 0)
 
 
 def run_ours(args):

@@ -80,8 +80,10 @@ int32_t run_experts(const uint16_t* hidden, const strata_qweights* w, const int3
     a.y = reinterpret_cast<float*>(y);
     a.status = status;
     a.num_sms = num_sms_of_current_device();
-    if (decode_smem_bytes(T, w->hidden) > 200u * 1024u) return STRATA_EUNSUPPORTED;
     (void)ws_bytes;
+    if (decode_tc_supported(T, w->hidden, w->inter, shared ? 1 : E, w->fmt, a.num_sms))
+      return from_cuda(launch_experts_decode_tc(a, st));
+    if (decode_smem_bytes(T, w->hidden) > 200u * 1024u) return STRATA_EUNSUPPORTED;
     return from_cuda(launch_experts_decode(a, st));
   }
   PrefillArgs a;
@@ -184,6 +186,7 @@ int32_t moe_router_topk(const uint16_t* hidden, const uint16_t* w_router, const 
     a.w = topk_w;
     a.logits_opt = logits_opt;
     a.status = dev_status;
+    a.part = reinterpret_cast<float*>(workspace);
     const cudaError_t e = launch_route_decode(a, st);
     if (e != cudaErrorNotSupported) return from_cuda(e);
   }
@@ -210,8 +213,10 @@ int32_t moe_route(const float* x, int32_t T, int32_t H, float eps, const uint16_
       !inv || !active || !aligned(x, 16) || !aligned(hidden, 16) || !aligned(w_router, 16))
     return STRATA_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (T <= kDecodeMaxTokens && route_decode_supported(T, H, E, k)) {
+  if (T <= kDecodeMaxTokens && route_decode_supported(T, H, E, k) && workspace &&
+      ws_bytes >= route_decode_workspace_bytes(T, H, E)) {
     RouteArgs a = {};
+    a.part = reinterpret_cast<float*>(workspace);
     a.x = x;
     a.hidden_out = hidden;
     a.eps = eps;

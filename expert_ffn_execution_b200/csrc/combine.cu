@@ -1,5 +1,6 @@
 // combine.cu -- RMSNorm and the fixed-order weighted combine.
 #include "decode.cuh"
+#include "tc05.cuh"
 
 namespace strata {
 
@@ -57,6 +58,9 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
   const int t = blockIdx.x;
   __shared__ int s_pos[32];
   __shared__ float s_w[32];
+  // launched as a programmatic dependent: every input comes from earlier grids
+  pdl_wait_prior();
+  pdl_trigger();
   if (threadIdx.x < k) {
     const int p = t * k + threadIdx.x;
     s_pos[threadIdx.x] = inv[p];
@@ -129,10 +133,17 @@ cudaError_t launch_combine(const void* y, int y_dtype, const int32_t* inv, const
                            int T, int k, int H, uint16_t* out, float* residual_out,
                            int32_t* status, cudaStream_t st) {
   if (T == 0) return cudaSuccess;
-  dim3 grid(T, (H / 8 + kCombThreads - 1) / kCombThreads);
-  combine_kernel<<<grid, kCombThreads, 0, st>>>(y, y_dtype, inv, w, shared_y, shared_dtype, residual, k,
-                                         H, out, residual_out, status);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(T, (H / 8 + kCombThreads - 1) / kCombThreads);
+  cfg.blockDim = dim3(kCombThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, y, y_dtype, inv, w, shared_y, shared_dtype,
+                            residual, k, H, out, residual_out, status);
 }
 
 }  // namespace strata

@@ -23,6 +23,8 @@ struct DecodeArgs {
 };
 cudaError_t launch_experts_decode(const DecodeArgs& a, cudaStream_t st);
 size_t decode_smem_bytes(int T, int H);
+bool decode_tc_supported(int T, int H, int I, int E, int fmt, int grid);
+cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
 struct PrefillArgs {
   const uint16_t* hidden;
@@ -55,8 +57,10 @@ struct RouteArgs {
   float* logits_opt;
   int32_t *counts, *offsets, *perm, *inv, *active;  // bucket outputs (counts == nullptr: skip)
   int32_t* status;
+  float* part;  // workspace: partial logits, route_decode_workspace_bytes()
 };
 bool route_decode_supported(int T, int H, int E, int k);
+uint64_t route_decode_workspace_bytes(int T, int H, int E);
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
 
 cudaError_t launch_rmsnorm(const float* x, int T, int H, float eps, uint16_t* out, cudaStream_t st);

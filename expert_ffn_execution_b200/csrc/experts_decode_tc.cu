@@ -1,0 +1,756 @@
+// experts_decode_tc.cu -- weight-streaming decode path of moe_experts
+// (T <= STRATA_DECODE_MAX_T) on the 5th-generation tensor cores.
+//
+// With at most 16 tokens per call the expert FFN is bound by streaming the
+// quantised weights out of HBM and decoding them, not by multiply-adds.  So
+// every weight row is decoded by exactly one thread, straight into that row's
+// lane of tensor memory (tcgen05.st), and the MMA reads its A operand
+// (128 weight rows x 16 K, fp16) from tensor memory; B is the token block
+// (N = 16 columns, fp16, in shared memory).  Decoded weights never pass
+// through shared memory, whose bandwidth would otherwise cap the path.  Codes
+// and scales arrive by TMA into a ring of shared-memory stages.
+//
+// Two kernels per call, chained by programmatic dependent launch:
+//   gate/up  tiles of 64 rows of I: lanes 0-63 decode the gate rows, lanes
+//            64-127 the same up rows.  B = every token of the call, so a tile
+//            computes all T columns and the epilogue keeps the tokens routed
+//            to the tile's expert: h = SwiGLU(gate, up) -> fp16 [P, I] in
+//            sorted pair order, K permuted within 16-groups the way the down
+//            kernel's decode orders K.
+//   down     tiles of 128 rows of H of one expert.  B = that expert's h rows
+//            (TMA from h); y fp32 [P, H] in sorted order.
+//
+// One persistent CTA per SM with a static tile list.  Warps:
+//   0-3   epilogue: tcgen05.ld of their TMEM lane quarter
+//   4..   decoders: kTcGroups groups of four warps taking K chunks in turn;
+//         a thread owns one tile row (= TMEM lane), reads its codes from
+//         the swizzled stage (conflict-free), decodes to fp16 and stores them
+//         into the A stage in tensor memory
+//   then  the TMA producer warp (codes, scales; down: the tile's scales and
+//         h blocks) and the warp that allocates tensor memory and issues
+//         the MMAs (one thread)
+// Barriers: full/empty (smem stages), tfull/tempty (TMEM A stages),
+// afull/aempty (two accumulators), sfull/sempty and bfull/bempty (down:
+// per-tile scales, per-expert h block).  Every wait is bounded.
+#include <algorithm>
+
+#include "decode.cuh"
+#include "tc05.cuh"
+#include "tmap.h"
+
+namespace strata {
+
+constexpr int kTcGroups = 2;                      // decoder groups (4 warps each)
+constexpr int kTcProdWarp = 4 + 4 * kTcGroups;     // TMA producer warp
+constexpr int kTcMmaWarp = kTcProdWarp + 1;        // TMEM allocation + MMA warp
+constexpr int kTcWarps = kTcMmaWarp + 1;
+constexpr int kTcThreads = kTcWarps * 32;
+constexpr int kTcKC = 256;        // K per chunk (one smem stage / one TMEM A stage)
+constexpr int kTcTS = 3;          // TMEM A stages
+constexpr int kTcACol0 = 64;      // A stage t at columns 64 + 128 t (accumulators at 0, 32)
+constexpr int kTcTmemCols = 512;
+constexpr int kTcMaxStages = 16;
+constexpr int kTcSmemBudget = 227 * 1024;
+// Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
+// only after the MMAs of its previous one retired, so with at least as many
+// stages as groups no waiter runs two phases ahead of a stage's barrier.
+static_assert(kTcTS >= kTcGroups, "TMEM A stages must cover the decoder groups");
+
+struct TcParams {
+  const uint16_t* hidden;
+  int T, H, I, E, k;
+  const uint8_t* wbase;
+  uint64_t stride;
+  const int32_t* offsets;
+  const int32_t* perm;
+  const int32_t* active;
+  int shared_mode;
+  uint16_t* hbuf;  // gate/up output, down input: fp16 [P, I]
+  float* y;        // down output: fp32 [P, H]
+  int32_t* status;
+  int S;           // shared-memory stages (a multiple of kTcGroups)
+  int NB;          // B rows: 8 (T <= 8; rows 8-15 of the MMA repeat them) or 16
+  int maxT;        // capacity of the tile table: tiles per CTA at most
+};
+
+template <int FMT>
+__host__ __device__ constexpr int tc_cbr() {  // code bytes per row per chunk
+  return FMT == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
+}
+
+struct TcLayout {
+  uint32_t codes_bytes, stage_bytes, b, b_bytes, sbuf, s_bytes, xch, tbl, bars, total;
+};
+
+__host__ __device__ inline uint32_t up1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+
+// Shared memory, from a 1024-byte aligned base: S stages | B (gate/up: one
+// token block; down: two h blocks) | down: two per-tile scale blocks |
+// gate/up: the SwiGLU exchange buffer | the tile table (maxT entries of 80
+// bytes) | barriers.
+__host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, int I, int S,
+                                              int maxT) {
+  TcLayout L;
+  const uint32_t cbr = fmt == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
+  L.codes_bytes = 128u * cbr;
+  L.stage_bytes = L.codes_bytes + (mode == 0 ? 128u * 16u : 0u);
+  uint32_t off = (uint32_t)S * L.stage_bytes;
+  L.b = off;
+  L.b_bytes = (uint32_t)NB * (uint32_t)(mode == 0 ? H : I) * 2u;
+  off += (mode == 0 ? 1u : 2u) * L.b_bytes;
+  L.sbuf = off;
+  L.s_bytes = mode == 1 ? up1k(8u * (uint32_t)I) : 0u;
+  off += 2u * L.s_bytes;
+  L.xch = off;
+  off += mode == 0 ? up1k(2u * 64u * 17u * 4u) : 0u;
+  L.tbl = off;
+  off += up1k(80u * (uint32_t)maxT);
+  L.bars = off;
+  off += 1024u;
+  L.total = off;
+  return L;
+}
+
+// ---------------------------------------------------------------- decode
+// One Q2 word (16 codes, element j at bits 2j) -> R[i] = fp16x2 (element i,
+// element i + 8) * d.  A code placed at mantissa bit p of an fp16 whose
+// exponent gives that bit unit weight is M_p + c exactly (M_p = 2^(10-p));
+// subtracting M_p + 1.5 leaves c - 1.5 exactly; the multiply by the block
+// scale rounds once.
+STRATA_DEVFN void dq_q2_word(uint32_t w, uint32_t d2, uint32_t* R) {
+  const uint32_t wl = w << 2, wr = w >> 8;
+  const uint32_t src[8] = {wl, w, w, w, w, wr, wr, wr};
+  const uint32_t msk[8] = {0x000C000Cu, 0x000C000Cu, 0x00300030u, 0x00C000C0u,
+                           0x03000300u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
+  const uint32_t mag[8] = {0x5C005C00u, 0x5C005C00u, 0x54005400u, 0x4C004C00u,
+                           0x44004400u, 0x5C005C00u, 0x54005400u, 0x4C004C00u};
+  const uint32_t sub[8] = {0x5C065C06u, 0x5C065C06u, 0x54185418u, 0x4C604C60u,
+                           0x45804580u, 0x5C065C06u, 0x54185418u, 0x4C604C60u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t v, t;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(src[i]), "r"(msk[i]), "r"(mag[i]));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(v), "r"(sub[i]));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(R[i]) : "r"(t), "r"(d2));
+  }
+}
+
+STRATA_DEVFN uint32_t dup_lo(uint32_t x) { return __byte_perm(x, 0, 0x1010); }
+STRATA_DEVFN uint32_t dup_hi(uint32_t x) { return __byte_perm(x, 0, 0x3232); }
+
+STRATA_DEVFN uint4 lds128(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(smem_addr(p)));
+  return v;
+}
+STRATA_DEVFN uint2 lds64(const void* p) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(smem_addr(p)));
+  return v;
+}
+
+// Gate/up B operand: token rows n < T of hidden (bf16 -> fp16, exact in the
+// normal range), rows T..NB-1 zero, K permuted within each 16-group like the
+// decoded codes, in the 128-byte-swizzled K-major layout (atoms of 64 K x NB
+// rows, 128 bytes per row, 16-byte piece c of row n at c ^ (n & 7)).  Thread
+// `tid` of `nthr` fills items tid, tid + nthr, ...; each batch issues all of
+// its loads before any conversion, so the fill costs a few L2 round trips.
+template <int FMT>
+STRATA_DEVFN void fill_tokens(uint8_t* bsm, const uint16_t* __restrict__ hidden, int T, int H,
+                              int NB, int tid, int nthr) {
+  constexpr int kBatch = 4;
+  const int ng = H / 16, total = NB * ng;
+  for (int i0 = tid; i0 < total; i0 += kBatch * nthr) {
+    uint4 a[kBatch], b[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int idx = i0 + u * nthr;
+      const int n = idx / ng, g = idx - n * ng;
+      a[u] = b[u] = make_uint4(0, 0, 0, 0);
+      if (idx < total && n < T) {
+        a[u] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 16 * g);
+        b[u] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 16 * g + 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int idx = i0 + u * nthr;
+      if (idx >= total) break;
+      const int n = idx / ng, g = idx - n * ng;
+      const uint32_t w[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
+      uint16_t e[16];
+#pragma unroll
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint16_t bf = (uint16_t)((kk & 1) ? (w[kk >> 1] >> 16) : (w[kk >> 1] & 0xffffu));
+        e[group_slot<FMT>(kk)] = bf16_to_f16_bits(bf);
+      }
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = (uint32_t)e[2 * j] | ((uint32_t)e[2 * j + 1] << 16);
+      const int pc = (g & 3) * 2;
+      uint8_t* row = bsm + (size_t)(g >> 2) * (NB * 128) + n * 128;
+      *reinterpret_cast<uint4*>(row + ((pc ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(row + (((pc + 1) ^ (n & 7)) << 4)) =
+          make_uint4(o[4], o[5], o[6], o[7]);
+    }
+  }
+}
+
+struct TcTile {
+  int e, rb, s0, n;
+  int tok[16];  // gate/up: token of each of the expert's pairs
+};
+
+// The CTA's tiles: round robin for gate/up (B is shared by all tiles),
+// contiguous ranges for down (consecutive tiles share an expert's h block).
+struct TcSched {
+  int tb, tstep, tcount;
+};
+template <int MODE>
+STRATA_DEVFN TcSched tc_sched(int ntot) {
+  TcSched q;
+  if (MODE == 0) {
+    q.tb = blockIdx.x;
+    q.tstep = gridDim.x;
+    q.tcount = ntot > q.tb ? (ntot - q.tb + q.tstep - 1) / q.tstep : 0;
+  } else {
+    q.tb = (int)((long long)ntot * blockIdx.x / gridDim.x);
+    q.tstep = 1;
+    q.tcount = (int)((long long)ntot * (blockIdx.x + 1) / gridDim.x) - q.tb;
+  }
+  return q;
+}
+
+// ---------------------------------------------------------------- kernel
+template <int MODE, int FMT>
+__global__ void __launch_bounds__(kTcThreads, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down codes
+                 const __grid_constant__ CUtensorMap mc1,  // up codes   | h [P, I]
+                 const __grid_constant__ CUtensorMap ms0,  // gate scales | unused
+                 const __grid_constant__ CUtensorMap ms1,  // up scales   | unused
+                 const TcParams p) {
+  constexpr int CBR = tc_cbr<FMT>();
+  constexpr int PIECE_K = (FMT == STRATA_FMT_Q2_32) ? 64 : 32;  // K per 16-byte code piece
+  constexpr int NPC = CBR / 16;                                  // pieces per full chunk
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const TcLayout L = tc_layout(MODE, FMT, p.NB, p.H, p.I, p.S, p.maxT);
+  const int S = p.S;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
+  uint64_t* empty = full + kTcMaxStages;
+  uint64_t* tfull = empty + kTcMaxStages;
+  uint64_t* tempty = tfull + kTcTS;
+  uint64_t* afull = tempty + kTcTS;
+  uint64_t* aempty = afull + 2;
+  uint64_t* sfull = aempty + 2;
+  uint64_t* sempty = sfull + 2;
+  uint64_t* bfull = sempty + 2;
+  uint64_t* bempty = bfull + 2;
+  uint64_t* tbl_ready = bempty + 2;
+  uint64_t* done = tbl_ready + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  TcTile* tbl = reinterpret_cast<TcTile*>(smem + L.tbl);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = p.H, I = p.I, T = p.T;
+  const int K = (MODE == 0) ? H : I;
+  const int nch = (K + kTcKC - 1) / kTcKC;
+  const int tpe = (MODE == 0) ? I / 64 : H / 128;  // tiles per expert
+  const Planes PL = plane_offsets(FMT, H, I);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 128);
+    }
+    for (int t = 0; t < kTcTS; ++t) {
+      mbar_init(&tfull[t], 128);
+      mbar_init(&tempty[t], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&afull[a], 1);
+      mbar_init(&aempty[a], 128);
+      mbar_init(&sfull[a], 1);
+      mbar_init(&sempty[a], 128 * kTcGroups);
+      mbar_init(&bfull[a], 1);
+      mbar_init(&bempty[a], 1);
+    }
+    mbar_init(tbl_ready, 128);
+    mbar_init(done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == kTcMmaWarp) {
+    tmem_alloc(tmem_slot, kTcTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == kTcProdWarp * 32) {
+    prefetch_tensormap(&mc0);
+    prefetch_tensormap(&mc1);
+    if constexpr (MODE == 0) {
+      prefetch_tensormap(&ms0);
+      prefetch_tensormap(&ms1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  // Dependents are released only after this CTA holds its tensor memory (a
+  // dependent CTA that allocated first on this SM and then waited for this
+  // grid would never get it back), and, for gate/up, after the routing
+  // tables it reads are complete: the down grid reads them before its wait.
+  if constexpr (MODE == 0) pdl_wait_prior();
+  pdl_trigger();
+
+  // ---- the CTA's tiles
+  int U = p.shared_mode ? 1 : p.active[0];
+  if (U < 0 || U > p.E) {
+    if (threadIdx.x == 0) dev_flag(p.status, STRATA_DEV_BOUNDS);
+    U = 0;
+  }
+  const TcSched sq = tc_sched<MODE>(U * tpe);
+  int tcount = sq.tcount;
+  if (tcount > p.maxT) {
+    if (threadIdx.x == 0) dev_flag(p.status, STRATA_DEV_BOUNDS);
+    tcount = p.maxT;
+  }
+  // expert of the CTA's i-th tile, straight from the routing tables
+  auto tile_e = [&](int i, int& rb) {
+    const int j = sq.tb + i * sq.tstep;
+    const int u = j / tpe;
+    rb = j - u * tpe;
+    if (p.shared_mode) return 0;
+    const int e = p.active[1 + u];
+    return (e < 0 || e >= p.E) ? 0 : e;
+  };
+
+  if (warp == kTcProdWarp) {
+    // ------------------------------------------------ TMA producer
+    if (elect_one()) {
+      int gc = 0, bseq = -1, prev_e = -1;
+      auto issue = [&](int e, int rb, int c) {
+        const int s = gc % S;
+        mbar_wait_guarded(&empty[s], ((gc / S) & 1) ^ 1, p.status, abort_flag);
+        uint8_t* st = smem + s * L.stage_bytes;
+        if constexpr (MODE == 0) {
+          mbar_arrive_expect_tx(&full[s], L.stage_bytes);
+          tma_load_3d(st, &mc0, c * CBR, rb * 64, e, &full[s]);
+          tma_load_3d(st + 64 * CBR, &mc1, c * CBR, rb * 64, e, &full[s]);
+          tma_load_3d(st + L.codes_bytes, &ms0, c * 8, rb * 64, e, &full[s]);
+          tma_load_3d(st + L.codes_bytes + 1024, &ms1, c * 8, rb * 64, e, &full[s]);
+        } else {
+          mbar_arrive_expect_tx(&full[s], L.codes_bytes);
+          tma_load_3d(st, &mc0, c * CBR, rb * 128, e, &full[s]);
+        }
+        ++gc;
+      };
+      for (int i = 0; i < tcount; ++i) {
+        int rb;
+        const int e = tile_e(i, rb);
+        int pre = 0;
+        if constexpr (MODE == 1) {
+          // the tile's scales: rows rb*128.. of the down plane, all of K
+          const int sb = i & 1;
+          mbar_wait_guarded(&sempty[sb], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
+          mbar_arrive_expect_tx(&sfull[sb], 8u * I);
+          bulk_g2s(smem + L.sbuf + sb * L.s_bytes,
+                   p.wbase + (uint64_t)e * p.stride + PL.scales[2] +
+                       (uint64_t)rb * 128u * (uint64_t)(I / 16),
+                   8u * I, &sfull[sb]);
+          // first tile: the weight chunks go out before the wait for h
+          pre = (i == 0) ? min(nch, S) : 0;
+          for (int c = 0; c < pre; ++c) issue(e, rb, c);
+          if (i == 0 || e != prev_e) {
+            ++bseq;
+            if (bseq == 0) pdl_wait_prior();  // h is written by the preceding grid
+            const int b = bseq & 1;
+            const int s0 = p.shared_mode ? 0 : p.offsets[e];
+            mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
+            const uint32_t ab = (uint32_t)p.NB * 128u;
+            mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
+            for (int a = 0; a < I / 64; ++a)
+              tma_load_2d(smem + L.b + b * L.b_bytes + a * ab, &mc1, 64 * a, s0, &bfull[b]);
+          }
+        }
+        for (int c = pre; c < nch; ++c) issue(e, rb, c);
+        prev_e = e;
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---- everyone else: the gate/up B operand, then (epilogue warps) the
+    // tile table
+    if constexpr (MODE == 0) {
+      // the producer warp is not among the fillers: renumber the warps after it
+      const int ftid = warp < kTcProdWarp ? (int)threadIdx.x : (int)threadIdx.x - 32;
+      fill_tokens<FMT>(smem + L.b, p.hidden, T, H, p.NB, ftid, (kTcWarps - 1) * 32);
+      fence_proxy_async_smem();
+      named_bar_sync(2, (kTcWarps - 1) * 32);
+    }
+    if (warp < 4) {
+      const int r = threadIdx.x;
+      for (int i = r; i < tcount; i += 128) {
+        TcTile& t = tbl[i];
+        t.e = tile_e(i, t.rb);
+        if (p.shared_mode) {
+          t.s0 = 0;
+          t.n = T;
+        } else {
+          t.s0 = p.offsets[t.e];
+          t.n = p.offsets[t.e + 1] - t.s0;
+          if (p.active[1 + (sq.tb + i * sq.tstep) / tpe] != t.e) {  // invalid expert id
+            dev_flag(p.status, STRATA_DEV_BOUNDS);
+            t.n = 0;
+          }
+        }
+        if (t.n < 0 || t.n > p.NB) {
+          dev_flag(p.status, STRATA_DEV_BOUNDS);
+          t.n = t.n < 0 ? 0 : p.NB;
+        }
+      }
+      named_bar_sync(1, 128);
+      if constexpr (MODE == 0) {
+        for (int x = r; x < tcount * 16; x += 128) {
+          TcTile& t = tbl[x >> 4];
+          const int j = x & 15;
+          if (j < t.n) {
+            int tk = p.shared_mode ? j : p.perm[t.s0 + j] / p.k;
+            if (tk < 0 || tk >= T) {
+              dev_flag(p.status, STRATA_DEV_BOUNDS);
+              tk = 0;
+            }
+            t.tok[j] = tk;
+          }
+        }
+      }
+      mbar_arrive(tbl_ready);
+    }
+  }
+
+  if (warp < 4) {
+    // ------------------------------------------------ epilogue
+    mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
+    const int r = threadIdx.x;  // tile row = TMEM lane
+    float* xch = reinterpret_cast<float*>(smem + L.xch);
+    for (int i = 0; i < tcount; ++i) {
+      const TcTile& ti = tbl[i];
+      const int a = i & 1;
+      mbar_wait_guarded(&afull[a], (i >> 1) & 1, p.status, abort_flag);
+      tc_fence_after();
+      uint32_t v[16];
+      tmem_ld16(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)(a * 32), v);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(&aempty[a]);
+      if constexpr (MODE == 0) {
+        float* xr = xch + r * 17;  // rows 0-63 gate, 64-127 up
+#pragma unroll
+        for (int j = 0; j < 16; ++j) xr[j] = __uint_as_float(v[j]);
+        named_bar_sync(1, 128);
+        for (int idx = r; idx < ti.n * 64; idx += 128) {
+          const int j = idx >> 6, l = idx & 63;
+          const int t = ti.tok[j];
+          const float gv = xch[l * 17 + t], uv = xch[(64 + l) * 17 + t];
+          const float h = silu_f32(gv) * uv;
+          const int ii = ti.rb * 64 + l;
+          const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
+          p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(__float2half_rn(h));
+        }
+        named_bar_sync(1, 128);
+      } else {
+        const int row = ti.rb * 128 + r;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < ti.n) p.y[(size_t)(ti.s0 + j) * H + row] = __uint_as_float(v[j]);
+      }
+    }
+  } else if (warp < kTcProdWarp) {
+    // ------------------------------------------------ decoders
+    const int g = (warp - 4) >> 2;
+    const int qd = warp & 3;
+    const int r = 32 * qd + lane;  // tile row = TMEM lane
+    const uint32_t swz = ((uint32_t)(r * CBR) >> 7) & (uint32_t)(NPC - 1);
+    const uint32_t tl = tmem_base + ((uint32_t)(32 * qd) << 16) + kTcACol0;
+    const Q4Table T4 = q4_table();
+    int gc = 0;
+    for (int i = 0; i < tcount; ++i) {
+      const uint8_t* srow = nullptr;
+      if constexpr (MODE == 1) {
+        mbar_wait_guarded(&sfull[i & 1], (i >> 1) & 1, p.status, abort_flag);
+        srow = smem + L.sbuf + (i & 1) * L.s_bytes + r * (I / 16);
+      }
+      for (int c = 0; c < nch; ++c, ++gc) {
+        if (gc % kTcGroups != g) continue;
+        const int s = gc % S;
+        mbar_wait_guarded(&full[s], (gc / S) & 1, p.status, abort_flag);
+        const uint8_t* st = smem + s * L.stage_bytes;
+        const int kv = min(kTcKC, K - c * kTcKC);  // 256, or 128 for a ragged last chunk
+        const int np = kv / PIECE_K;
+        uint4 cw[NPC];
+#pragma unroll
+        for (int pc = 0; pc < NPC; ++pc)
+          cw[pc] = (pc < np) ? lds128(st + r * CBR + ((pc ^ swz) << 4)) : make_uint4(0, 0, 0, 0);
+        uint32_t sc[4];
+        if constexpr (MODE == 0) {
+          const uint4 v = lds128(st + L.codes_bytes + r * 16);
+          sc[0] = v.x;
+          sc[1] = v.y;
+          sc[2] = v.z;
+          sc[3] = v.w;
+        } else {
+          const uint2 lo = lds64(srow + c * 16);
+          sc[0] = lo.x;
+          sc[1] = lo.y;
+          sc[2] = 0;
+          sc[3] = 0;
+          if (kv > 128) {
+            const uint2 hi = lds64(srow + c * 16 + 8);
+            sc[2] = hi.x;
+            sc[3] = hi.y;
+          }
+        }
+        // The stage is released before its loads are consumed: order those
+        // generic-proxy reads before the producer's next TMA (async-proxy)
+        // write into the stage, which the barrier alone does not.
+        fence_proxy_async_smem();
+        mbar_arrive(&empty[s]);
+        const int t = gc % kTcTS;
+        mbar_wait_guarded(&tempty[t], ((gc / kTcTS) & 1) ^ 1, p.status, abort_flag);
+        tc_fence_after();
+        const uint32_t ta = tl + (uint32_t)t * 128u;
+        if constexpr (FMT == STRATA_FMT_Q2_32) {
+#pragma unroll
+          for (int pc = 0; pc < NPC; ++pc) {
+            if (pc < np) {
+              uint32_t R[32];
+              const uint32_t d0 = dup_lo(sc[pc]), d1 = dup_hi(sc[pc]);
+              dq_q2_word(cw[pc].x, d0, R);
+              dq_q2_word(cw[pc].y, d0, R + 8);
+              dq_q2_word(cw[pc].z, d1, R + 16);
+              dq_q2_word(cw[pc].w, d1, R + 24);
+              tmem_st32(ta + pc * 32, R);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int pc = 0; pc < NPC; ++pc) {
+            if (pc < np) {
+              uint32_t R[16], R0[8], R1[8];
+              const __half2 d2 =
+                  u32_as_h2((pc & 1) ? dup_hi(sc[pc >> 1]) : dup_lo(sc[pc >> 1]));
+              dq_q4_group(cw[pc].x, cw[pc].y, d2, T4, R0);
+              dq_q4_group(cw[pc].z, cw[pc].w, d2, T4, R1);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                R[j] = R0[j];
+                R[8 + j] = R1[j];
+              }
+              tmem_st16(ta + pc * 16, R);
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&tfull[t]);
+      }
+      if constexpr (MODE == 1) {
+        fence_proxy_async_smem();  // same for the scale block and its next bulk copy
+        mbar_arrive(&sempty[i & 1]);
+      }
+    }
+  } else if (warp == kTcMmaWarp) {
+    // ------------------------------------------------ MMA issue (one thread)
+    if constexpr (MODE == 1) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
+    if (elect_one()) {
+      const uint32_t idesc = idesc_f16_f32(16);
+      const uint32_t sbo = p.NB == 16 ? 1024u : 0u;
+      const uint32_t ab = (uint32_t)p.NB * 128u;
+      // descriptor start-address steps (16-byte units): one 64-K atom, one K16 step
+      const uint64_t d_atom = ab >> 4, d_k16 = 32 >> 4;
+      int gc = 0, bseq = -1, prev_e = -1;
+      for (int i = 0; i < tcount; ++i) {
+        uint32_t bbase = smem_addr(smem + L.b);
+        int b = 0;
+        if constexpr (MODE == 1) {
+          const int e = tbl[i].e;
+          if (i == 0 || e != prev_e) {
+            ++bseq;
+            mbar_wait_guarded(&bfull[bseq & 1], (bseq >> 1) & 1, p.status, abort_flag);
+            tc_fence_after();
+          }
+          prev_e = e;
+          b = bseq & 1;
+          bbase += (uint32_t)b * L.b_bytes;
+        }
+        const int a = i & 1;
+        mbar_wait_guarded(&aempty[a], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(a * 32);
+        // B descriptor of the chunk's first K16 step; the steps inside a
+        // chunk are constant offsets from it (the loop is unrolled)
+        uint64_t bd = smem_desc_k128_sbo(bbase, sbo);
+        for (int c = 0; c < nch; ++c, ++gc, bd += 4 * d_atom) {
+          const int t = gc % kTcTS;
+          mbar_wait_guarded(&tfull[t], (gc / kTcTS) & 1, p.status, abort_flag);
+          tc_fence_after();
+          const bool half = K - c * kTcKC < kTcKC;  // ragged last chunk: 128 K
+          const uint32_t at = tmem_base + kTcACol0 + (uint32_t)t * 128u;
+#pragma unroll
+          for (int kk = 0; kk < kTcKC / 16; ++kk) {
+            if (kk < kTcKC / 32 || !half)
+              mma_f16_ts(d, at + (uint32_t)kk * 8u, bd + (kk >> 2) * d_atom + (kk & 3) * d_k16,
+                         idesc, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&tempty[t]);
+        }
+        mma_commit(&afull[a]);
+        if constexpr (MODE == 1) {
+          if (i + 1 == tcount || tbl[i + 1].e != tbl[i].e) mma_commit(&bempty[b]);
+        }
+      }
+      mma_commit(done);
+      // every MMA retired before the tensor memory is released (bounded)
+      mbar_wait_bounded(done, 0, p.status);
+    }
+    __syncwarp();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kTcMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTcTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------- host side
+namespace {
+
+// Tiles per CTA at most (the tile-table capacity): every expert active.
+int tc_max_tiles(int mode, int E, int H, int I, int grid) {
+  const long long ntot = (long long)E * (mode == 0 ? I / 64 : H / 128);
+  return (int)std::max<long long>(1, (ntot + grid - 1) / grid);
+}
+
+// Shared-memory stages that fit, rounded down to a multiple of the decoder
+// group count: chunk c uses stage c % S and group c % kTcGroups, so every
+// use of a stage belongs to one group and its barrier phases are awaited in
+// order (a waiter two phases ahead would see its parity as complete).
+int tc_stages(int mode, int fmt, int NB, int H, int I, int maxT) {
+  const TcLayout L0 = tc_layout(mode, fmt, NB, H, I, 0, maxT);
+  const long long room = (long long)kTcSmemBudget - 1024 - (long long)L0.total;
+  if (room <= 0) return 0;
+  const int s = (int)std::min<long long>(kTcMaxStages, room / L0.stage_bytes);
+  return s - s % kTcGroups;
+}
+
+template <int MODE, int FMT>
+cudaError_t launch_tc(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& m2,
+                      const CUtensorMap& m3, const TcParams& prm, int grid, cudaStream_t st) {
+  auto kern = decode_tc_kernel<MODE, FMT>;
+  const size_t smem = 1024 + tc_layout(MODE, FMT, prm.NB, prm.H, prm.I, prm.S, prm.maxT).total;
+  cudaError_t e =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, m0, m1, m2, m3, prm);
+}
+
+}  // namespace
+
+bool decode_tc_supported(int T, int H, int I, int E, int fmt, int grid) {
+  if (T < 1 || T > kDecodeMaxTokens || H % 256 || I % 128 || grid < 1) return false;
+  const int NB = T <= 8 ? 8 : 16;
+  return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, E, H, I, grid)) >= kTcGroups &&
+         tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, E, H, I, grid)) >= kTcGroups;
+}
+
+cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
+  const int E = a.shared_mode ? 1 : a.E;
+  if (!decode_tc_supported(a.T, a.H, a.I, E, a.fmt, a.num_sms)) return cudaErrorNotSupported;
+  const int NB = a.T <= 8 ? 8 : 16;
+  const long long P = a.shared_mode ? a.T : (long long)a.T * a.k;
+  const Planes PL = plane_offsets(a.fmt, a.H, a.I);
+  const bool q2 = a.fmt == STRATA_FMT_Q2_32;
+  const cuuint32_t cbr = q2 ? kTcKC / 4 : kTcKC / 2;
+  const CUtensorMapSwizzle sw = cbr == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const cuuint64_t rowH = codes_row_bytes(a.fmt, a.H), rowI = codes_row_bytes(a.fmt, a.I);
+  CUtensorMap mg, mu, msg, msu, md, mh;
+  {
+    const cuuint64_t dims[3] = {rowH, (cuuint64_t)a.I, (cuuint64_t)E};
+    const cuuint64_t str[2] = {rowH, a.stride};
+    const cuuint32_t box[3] = {cbr, 64, 1};
+    if (!make_tmap(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[0], dims, str, box, sw) ||
+        !make_tmap(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[1], dims, str, box, sw))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {(cuuint64_t)a.H / 32, (cuuint64_t)a.I, (cuuint64_t)E};
+    const cuuint64_t str[2] = {(cuuint64_t)a.H / 16, a.stride};
+    const cuuint32_t box[3] = {8, 64, 1};
+    if (!make_tmap(&msg, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, a.wbase + PL.scales[0], dims, str, box,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap(&msu, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, a.wbase + PL.scales[1], dims, str, box,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[3] = {rowI, (cuuint64_t)a.H, (cuuint64_t)E};
+    const cuuint64_t str[2] = {rowI, a.stride};
+    const cuuint32_t box[3] = {cbr, 128, 1};
+    if (!make_tmap(&md, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[2], dims, str, box, sw))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)a.I, (cuuint64_t)P};
+    const cuuint64_t str[1] = {(cuuint64_t)a.I * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)NB};
+    if (!make_tmap(&mh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.hbuf, dims, str, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  TcParams prm;
+  prm.hidden = a.hidden;
+  prm.T = a.T;
+  prm.H = a.H;
+  prm.I = a.I;
+  prm.E = E;
+  prm.k = a.k;
+  prm.wbase = a.wbase;
+  prm.stride = a.stride;
+  prm.offsets = a.offsets;
+  prm.perm = a.perm;
+  prm.active = a.active;
+  prm.shared_mode = a.shared_mode;
+  prm.hbuf = a.hbuf;
+  prm.y = a.y;
+  prm.status = a.status;
+  prm.NB = NB;
+  cudaError_t e;
+  prm.maxT = tc_max_tiles(0, E, a.H, a.I, a.num_sms);
+  prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);
+  if (q2)
+    e = launch_tc<0, STRATA_FMT_Q2_32>(mg, mu, msg, msu, prm, a.num_sms, st);
+  else
+    e = launch_tc<0, STRATA_FMT_Q4CB_32>(mg, mu, msg, msu, prm, a.num_sms, st);
+  if (e != cudaSuccess) return e;
+  prm.maxT = tc_max_tiles(1, E, a.H, a.I, a.num_sms);
+  prm.S = tc_stages(1, a.fmt, NB, a.H, a.I, prm.maxT);
+  if (q2) return launch_tc<1, STRATA_FMT_Q2_32>(md, mh, md, md, prm, a.num_sms, st);
+  return launch_tc<1, STRATA_FMT_Q4CB_32>(md, mh, md, md, prm, a.num_sms, st);
+}
+
+}  // namespace strata

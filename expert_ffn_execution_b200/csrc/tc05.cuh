@@ -71,6 +71,16 @@ STRATA_DEVFN void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
       : "memory");
 }
 
+// 3-D tiled load (c0 innermost), no multicast.
+STRATA_DEVFN void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+      : "memory");
+}
+
 STRATA_DEVFN void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -108,6 +118,31 @@ STRATA_DEVFN void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 STRATA_DEVFN void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Register -> tensor memory: 32 lanes x 32 bits, N consecutive columns per
+// thread (thread i of the warp writes lane base + i).
+STRATA_DEVFN void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+STRATA_DEVFN void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+STRATA_DEVFN void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 // ---------------------------------------------------------------- MMA
 // Shared-memory matrix descriptor, K-major operand in the 128-byte swizzled
 // layout: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte
@@ -119,6 +154,18 @@ STRATA_DEVFN uint64_t smem_desc_k128(uint32_t saddr) {
   d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: 8 rows x 128 B
   d |= (uint64_t)1 << 46;                         // version
   d |= (uint64_t)2 << 61;                         // SWIZZLE_128B
+  return d;
+}
+
+// Same, with an explicit stride byte offset between 8-row groups (0 makes
+// rows 8-15 of an N = 16 operand repeat rows 0-7).
+STRATA_DEVFN uint64_t smem_desc_k128_sbo(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
   return d;
 }
 
@@ -141,6 +188,18 @@ STRATA_DEVFN void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, ui
       : "memory");
 }
 
+// Same with the A operand (128 rows x 16 K, two fp16 per 32-bit column, row
+// m in lane m) read from tensor memory at a_tmem.
+STRATA_DEVFN void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on `bar` once all previously issued tcgen05 operations of this
 // thread have completed.
 STRATA_DEVFN void mma_commit(uint64_t* bar) {
@@ -148,6 +207,15 @@ STRATA_DEVFN void mma_commit(uint64_t* bar) {
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_addr(bar))
       : "memory");
+}
+
+// Programmatic dependent launch: wait for the preceding grid's completion
+// (and memory), and let the next grid's CTAs be scheduled.
+STRATA_DEVFN void pdl_wait_prior() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+STRATA_DEVFN void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+STRATA_DEVFN void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 STRATA_DEVFN bool elect_one() {

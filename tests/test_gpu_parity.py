@@ -163,7 +163,8 @@ def check_layer(r: Run, sample=None):
     return err
 
 
-@pytest.mark.parametrize("config,T", [(0, 1), (1, 4), (3, 1), (3, 4), (4, 1), (4, 4)])
+@pytest.mark.parametrize("config,T", [(0, 1), (1, 4), (3, 1), (3, 4), (4, 1), (4, 4), (4, 8),
+                                      (4, 16)])
 def test_decode_layer_parity(config, T):
     r = Run(config, T).run()
     err = check_layer(r)
@@ -185,9 +186,10 @@ def test_decode_small_expert_count_and_k1():
     check_layer(r)
 
 
-def test_decode_deterministic():
-    a = Run(1, 4).run()
-    b = Run(1, 4).run()
+@pytest.mark.parametrize("config,T", [(1, 4), (4, 8)])
+def test_decode_deterministic(config, T):
+    a = Run(config, T).run()
+    b = Run(config, T).run()
     for x, y in ((a.ids, b.ids), (a.perm, b.perm), (a.y, b.y), (a.out, b.out)):
         assert torch.equal(x, y)
 
