@@ -154,13 +154,24 @@ STRATA_DEVFN void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t
 // normalises a row gets the same bits.
 STRATA_DEVFN float rms_inv_warp(const float* __restrict__ xr, int H, float eps) {
   const int lane = threadIdx.x & 31;
+  constexpr int kBatch = 8;  // loads in flight per lane; the FMA order is unchanged
   float ss = 0.f;
-  for (int h = lane * 4; h < H; h += 128) {
-    const float4 v = *reinterpret_cast<const float4*>(xr + h);
-    ss = fmaf(v.x, v.x, ss);
-    ss = fmaf(v.y, v.y, ss);
-    ss = fmaf(v.z, v.z, ss);
-    ss = fmaf(v.w, v.w, ss);
+  for (int h0 = lane * 4; h0 < H; h0 += 128 * kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int h = h0 + 128 * u;
+      v[u] = (h < H) ? *reinterpret_cast<const float4*>(xr + h) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (h0 + 128 * u < H) {
+        ss = fmaf(v[u].x, v[u].x, ss);
+        ss = fmaf(v[u].y, v[u].y, ss);
+        ss = fmaf(v[u].z, v[u].z, ss);
+        ss = fmaf(v[u].w, v[u].w, ss);
+      }
+    }
   }
   ss = warp_sum(ss);
   return 1.0f / sqrtf(ss / (float)H + eps);

@@ -40,7 +40,7 @@
 
 namespace strata {
 
-constexpr int kTcGroups = 2;                      // decoder groups (4 warps each)
+constexpr int kTcGroups = 3;                      // decoder groups (4 warps each)
 constexpr int kTcProdWarp = 4 + 4 * kTcGroups;     // TMA producer warp
 constexpr int kTcMmaWarp = kTcProdWarp + 1;        // TMEM allocation + MMA warp
 constexpr int kTcWarps = kTcMmaWarp + 1;
@@ -434,13 +434,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
 
   if (warp < 4) {
     // ------------------------------------------------ epilogue
-    mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
+    mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
     const int r = threadIdx.x;  // tile row = TMEM lane
     float* xch = reinterpret_cast<float*>(smem + L.xch);
     for (int i = 0; i < tcount; ++i) {
       const TcTile& ti = tbl[i];
       const int a = i & 1;
-      mbar_wait_guarded(&afull[a], (i >> 1) & 1, p.status, abort_flag);
+      mbar_wait_backoff(&afull[a], (i >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
       uint32_t v[16];
       tmem_ld16(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)(a * 32), v);

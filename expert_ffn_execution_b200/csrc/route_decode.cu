@@ -69,22 +69,59 @@ __global__ void __launch_bounds__(kRlThreads) route_logits_kernel(RouteArgs a, f
   // 2. the tokens (written by the preceding grid)
   pdl_wait_prior();
   pdl_trigger();
+  const int nq = T * HR / 4;  // 4-element groups of this CTA's rows (HR % 16 == 0)
+  constexpr int kQ = 4;       // groups per thread in flight
   if (a.x) {
+    const float* __restrict__ x = a.x;
     for (int t = warp; t < T; t += kRlThreads / 32) {
-      const float inv = rms_inv_warp(a.x + (size_t)t * H, H, a.eps);
+      const float inv = rms_inv_warp(x + (size_t)t * H, H, a.eps);
       if (lane == 0) sinv[t] = inv;
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < T * HR; i += kRlThreads) {
-      const int t = i / HR, r = i - t * HR;
-      const uint16_t b = float_to_bf16_bits(a.x[(size_t)t * H + h0 + r] * sinv[t]);
-      xs[t * (HR + 8) + r] = b;
-      if (es == 0) a.hidden_out[(size_t)t * H + h0 + r] = b;
+    uint16_t* __restrict__ hout = a.hidden_out;
+    for (int q0 = threadIdx.x; q0 < nq; q0 += kRlThreads * kQ) {
+      float4 v[kQ];
+#pragma unroll
+      for (int u = 0; u < kQ; ++u) {
+        const int q = q0 + u * kRlThreads;
+        const int t = (4 * q) / HR, r = 4 * q - t * HR;
+        v[u] = q < nq ? *reinterpret_cast<const float4*>(x + (size_t)t * H + h0 + r)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < kQ; ++u) {
+        const int q = q0 + u * kRlThreads;
+        if (q < nq) {
+          const int t = (4 * q) / HR, r = 4 * q - t * HR;
+          const float inv = sinv[t];
+          const uint32_t lo = float_to_bf16_bits(v[u].x * inv) |
+                              ((uint32_t)float_to_bf16_bits(v[u].y * inv) << 16);
+          const uint32_t hi = float_to_bf16_bits(v[u].z * inv) |
+                              ((uint32_t)float_to_bf16_bits(v[u].w * inv) << 16);
+          *reinterpret_cast<uint2*>(xs + t * (HR + 8) + r) = make_uint2(lo, hi);
+          if (es == 0) *reinterpret_cast<uint2*>(hout + (size_t)t * H + h0 + r) = make_uint2(lo, hi);
+        }
+      }
     }
   } else {
-    for (int i = threadIdx.x; i < T * HR; i += kRlThreads) {
-      const int t = i / HR, r = i - t * HR;
-      xs[t * (HR + 8) + r] = a.hidden[(size_t)t * H + h0 + r];
+    const uint16_t* __restrict__ hin = a.hidden;
+    for (int q0 = threadIdx.x; q0 < nq; q0 += kRlThreads * kQ) {
+      uint2 v[kQ];
+#pragma unroll
+      for (int u = 0; u < kQ; ++u) {
+        const int q = q0 + u * kRlThreads;
+        const int t = (4 * q) / HR, r = 4 * q - t * HR;
+        v[u] = q < nq ? *reinterpret_cast<const uint2*>(hin + (size_t)t * H + h0 + r)
+                      : make_uint2(0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kQ; ++u) {
+        const int q = q0 + u * kRlThreads;
+        if (q < nq) {
+          const int t = (4 * q) / HR, r = 4 * q - t * HR;
+          *reinterpret_cast<uint2*>(xs + t * (HR + 8) + r) = v[u];
+        }
+      }
     }
   }
   asm volatile("cp.async.wait_group 0;" ::: "memory");
@@ -144,12 +181,40 @@ __global__ void __launch_bounds__(kRsThreads) route_select_kernel(RouteArgs a, c
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait_prior();
   pdl_trigger();
-  for (int i = threadIdx.x; i < T * E; i += kRsThreads) {
-    float s = 0.f;
-    for (int h = 0; h < HS; ++h) s += part[(size_t)h * T * E + i];
-    if (a.bias) s += a.bias[i % E];
-    lg[i] = s;
-    if (a.logits_opt) a.logits_opt[i] = s;
+  // logits = sum of the HS partials in order, + bias; all loads of a thread
+  // are issued before any store (part, bias and the outputs may not alias)
+  {
+    const float* __restrict__ pp = part;
+    const float* __restrict__ bias = a.bias;
+    float* __restrict__ lopt = a.logits_opt;
+    const int n4 = T * E / 4;
+    for (int g = threadIdx.x; g < n4; g += kRsThreads) {
+      float4 v[8];
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < HS) v[h] = *reinterpret_cast<const float4*>(pp + (size_t)h * T * E + 4 * g);
+      float bb[4] = {0.f, 0.f, 0.f, 0.f};
+      if (bias) {
+        const int e = (4 * g) % E;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) bb[j] = bias[e + j];
+      }
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < 8; ++h)
+        if (h < HS) {
+          s[0] += v[h].x;
+          s[1] += v[h].y;
+          s[2] += v[h].z;
+          s[3] += v[h].w;
+        }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (bias) s[j] += bb[j];
+        lg[4 * g + j] = s[j];
+        if (lopt) lopt[4 * g + j] = s[j];
+      }
+    }
   }
   __syncthreads();
   for (int t = warp; t < T; t += kRsThreads / 32) {
@@ -216,8 +281,11 @@ static cudaError_t launch_route_t(const RouteArgs& a, float* part, cudaStream_t 
 }
 
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st) {
+  // vector accesses: W_r and the partials 16-byte, x 16-byte, hidden 8-byte aligned
   if (!route_decode_supported(a.T, a.H, a.E, a.k) || !a.part ||
-      reinterpret_cast<uintptr_t>(a.wr) % 16 || reinterpret_cast<uintptr_t>(a.part) % 16)
+      reinterpret_cast<uintptr_t>(a.wr) % 16 || reinterpret_cast<uintptr_t>(a.part) % 16 ||
+      (a.x && (reinterpret_cast<uintptr_t>(a.x) % 16 || reinterpret_cast<uintptr_t>(a.hidden_out) % 8)) ||
+      (!a.x && reinterpret_cast<uintptr_t>(a.hidden) % 8))
     return cudaErrorNotSupported;
   const bool two = a.T > 8;
   if (a.E <= 256)

@@ -43,6 +43,27 @@ STRATA_DEVFN bool mbar_wait_guarded(uint64_t* bar, uint32_t parity, int32_t* sta
   return true;
 }
 
+// Same, polling with a nanosleep backoff: for warps off the critical path
+// (epilogue, table), so that their polling does not take issue slots from
+// the warps that share their scheduler.
+STRATA_DEVFN bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, int32_t* status,
+                                    volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  uint32_t ns = 64;
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort_flag = 1;
+      dev_flag(status, STRATA_DEV_TIMEOUT);
+      return false;
+    }
+    __nanosleep(ns);
+    if (ns < 512) ns <<= 1;
+  }
+  return true;
+}
+
 // Add expected transaction bytes to the current phase without arriving.
 STRATA_DEVFN void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
