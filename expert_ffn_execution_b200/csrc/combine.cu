@@ -5,17 +5,14 @@
 namespace strata {
 
 // hidden[t,h] = bf16_rne(x[t,h] * (1 / sqrt(mean_h x^2 + eps))), one CTA per
-// token; the RMS comes from rms_inv_warp (the same bits as the fused routing
-// kernel).
+// token; the RMS comes from rms_inv_rows<256> (the same bits as the fused
+// routing kernel).
 __global__ void __launch_bounds__(256)
 rmsnorm_kernel(const float* __restrict__ x, int H, float eps, uint16_t* __restrict__ out) {
+  __shared__ float red[8];
   __shared__ float s_inv;
   const float* xr = x + (size_t)blockIdx.x * H;
-  if (threadIdx.x < 32) {
-    const float inv = rms_inv_warp(xr, H, eps);
-    if (threadIdx.x == 0) s_inv = inv;
-  }
-  __syncthreads();
+  rms_inv_rows<256>(xr, 1, H, eps, red, &s_inv);
   const float inv = s_inv;
   uint16_t* orow = out + (size_t)blockIdx.x * H;
   for (int h = threadIdx.x * 4; h < H; h += blockDim.x * 4) {
@@ -47,9 +44,11 @@ STRATA_DEVFN void load8(const void* base, int dtype, size_t idx, float (&v)[8]) 
 
 // acc = sum_j w_j * y[inv[t*k+j]] (j ascending, separate multiply and add,
 // no contraction), + shared_y; out = bf16(acc); residual_out = residual + acc.
-// grid (T, ceil(H / (8 * 128))): each thread owns 8 consecutive features and
-// issues the loads of four expert rows before accumulating them in order.
-constexpr int kCombThreads = 128;
+// grid (T, ceil(H / (8 * 64))): each thread owns 8 consecutive features; the
+// loads of up to 8 expert rows, the shared row and the residual are in
+// flight together before the accumulation, which keeps the fixed order.
+constexpr int kCombThreads = 64;
+constexpr int kCombBatch = 8;
 __global__ void __launch_bounds__(kCombThreads)
 combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restrict__ inv,
                const float* __restrict__ w, const void* __restrict__ shared_y, int shared_dtype,
@@ -69,13 +68,21 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
   __syncthreads();
   const int h = (blockIdx.y * kCombThreads + threadIdx.x) * 8;
   if (h >= H) return;
+  float sv[8], rv[8];
+  if (shared_y) load8(shared_y, shared_dtype, (size_t)t * H + h, sv);
+  if (residual_out) {
+    const float4 r0 = *reinterpret_cast<const float4*>(residual + (size_t)t * H + h);
+    const float4 r1 = *reinterpret_cast<const float4*>(residual + (size_t)t * H + h + 4);
+    rv[0] = r0.x; rv[1] = r0.y; rv[2] = r0.z; rv[3] = r0.w;
+    rv[4] = r1.x; rv[5] = r1.y; rv[6] = r1.z; rv[7] = r1.w;
+  }
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int j0 = 0; j0 < k; j0 += 4) {
-    float v[4][8];
+  for (int j0 = 0; j0 < k; j0 += kCombBatch) {
+    float v[kCombBatch][8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kCombBatch; ++u) {
       const int j = j0 + u;
       const int pos = (j < k) ? s_pos[j] : -1;
       if (pos >= 0) {
@@ -87,7 +94,7 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
       }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < kCombBatch; ++u) {
       const int j = j0 + u;
       if (j < k && s_pos[j] >= 0) {
         const float wj = s_w[j];
@@ -97,10 +104,8 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
     }
   }
   if (shared_y) {
-    float v[8];
-    load8(shared_y, shared_dtype, (size_t)t * H + h, v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], v[i]);
+    for (int i = 0; i < 8; ++i) acc[i] = __fadd_rn(acc[i], sv[i]);
   }
   uint32_t o[4];
 #pragma unroll
@@ -108,16 +113,11 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
     o[i] = float_to_bf16_bits(acc[2 * i]) | (uint32_t(float_to_bf16_bits(acc[2 * i + 1])) << 16);
   *reinterpret_cast<uint4*>(out + (size_t)t * H + h) = make_uint4(o[0], o[1], o[2], o[3]);
   if (residual_out) {
-    const float* r = residual + (size_t)t * H + h;
-    const float4 r0 = *reinterpret_cast<const float4*>(r);
-    const float4 r1 = *reinterpret_cast<const float4*>(r + 4);
-    const float4 o0 = make_float4(__fadd_rn(r0.x, acc[0]), __fadd_rn(r0.y, acc[1]),
-                                  __fadd_rn(r0.z, acc[2]), __fadd_rn(r0.w, acc[3]));
-    const float4 o1 = make_float4(__fadd_rn(r1.x, acc[4]), __fadd_rn(r1.y, acc[5]),
-                                  __fadd_rn(r1.z, acc[6]), __fadd_rn(r1.w, acc[7]));
     float* ro = residual_out + (size_t)t * H + h;
-    *reinterpret_cast<float4*>(ro) = o0;
-    *reinterpret_cast<float4*>(ro + 4) = o1;
+    *reinterpret_cast<float4*>(ro) = make_float4(__fadd_rn(rv[0], acc[0]), __fadd_rn(rv[1], acc[1]),
+                                                 __fadd_rn(rv[2], acc[2]), __fadd_rn(rv[3], acc[3]));
+    *reinterpret_cast<float4*>(ro + 4) = make_float4(__fadd_rn(rv[4], acc[4]), __fadd_rn(rv[5], acc[5]),
+                                                     __fadd_rn(rv[6], acc[6]), __fadd_rn(rv[7], acc[7]));
   }
 }
 

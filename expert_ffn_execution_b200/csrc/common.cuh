@@ -149,32 +149,54 @@ STRATA_DEVFN void mma_16816_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// 1 / sqrt(mean(x^2) + eps) of one row, computed by one warp in a fixed order
-// (lane-strided float4 partial sums, then a butterfly), so every kernel that
-// normalises a row gets the same bits.
-STRATA_DEVFN float rms_inv_warp(const float* __restrict__ xr, int H, float eps) {
-  const int lane = threadIdx.x & 31;
-  constexpr int kBatch = 8;  // loads in flight per lane; the FMA order is unchanged
-  float ss = 0.f;
-  for (int h0 = lane * 4; h0 < H; h0 += 128 * kBatch) {
-    float4 v[kBatch];
+// 1 / sqrt(mean(x^2) + eps) of T rows by a whole CTA of NTH threads, in a
+// fixed order, so every kernel that normalises a row gets the same bits:
+// thread i accumulates elements 4i..4i+3, 4i+4*NTH.., ... of a row with fmaf
+// in that order; warp butterfly sums; the warp partials are added in warp
+// order.  Loads of several rows are in flight together.  red holds
+// >= T * NTH/32 floats and inv_out T floats (shared memory); ends with a
+// __syncthreads.
+template <int NTH>
+STRATA_DEVFN void rms_inv_rows(const float* __restrict__ x, int T, int H, float eps, float* red,
+                               float* inv_out) {
+  constexpr int NW = NTH / 32;
+  constexpr int kMaxV = 16;  // float4 loads in flight per thread
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int per = (H + 4 * NTH - 1) / (4 * NTH);  // float4 per thread per row
+  const int rows = per >= kMaxV ? 1 : kMaxV / per;  // rows per batch
+  for (int t0 = 0; t0 < T; t0 += rows) {
+    float4 v[kMaxV];
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const int h = h0 + 128 * u;
-      v[u] = (h < H) ? *reinterpret_cast<const float4*>(xr + h) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int u = 0; u < kMaxV; ++u) {
+      const int r = u / per, j = u - r * per;  // per >= 1
+      const int t = t0 + r, h = 4 * tid + 4 * NTH * j;
+      v[u] = (r < rows && t < T && h < H && u < rows * per)
+                 ? *reinterpret_cast<const float4*>(x + (size_t)t * H + h)
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    for (int r = 0; r < rows && t0 + r < T; ++r) {
+      float ss = 0.f;
 #pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      if (h0 + 128 * u < H) {
-        ss = fmaf(v[u].x, v[u].x, ss);
-        ss = fmaf(v[u].y, v[u].y, ss);
-        ss = fmaf(v[u].z, v[u].z, ss);
-        ss = fmaf(v[u].w, v[u].w, ss);
+      for (int u = 0; u < kMaxV; ++u) {
+        if (u / per == r && u < rows * per && 4 * tid + 4 * NTH * (u - r * per) < H) {
+          ss = fmaf(v[u].x, v[u].x, ss);
+          ss = fmaf(v[u].y, v[u].y, ss);
+          ss = fmaf(v[u].z, v[u].z, ss);
+          ss = fmaf(v[u].w, v[u].w, ss);
+        }
       }
+      ss = warp_sum(ss);
+      if (lane == 0) red[(t0 + r) * NW + wid] = ss;
     }
   }
-  ss = warp_sum(ss);
-  return 1.0f / sqrtf(ss / (float)H + eps);
+  __syncthreads();
+  if (tid < T) {
+    float ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) ss += red[tid * NW + w];
+    inv_out[tid] = 1.0f / sqrtf(ss / (float)H + eps);
+  }
+  __syncthreads();
 }
 
 }  // namespace strata

@@ -73,11 +73,7 @@ __global__ void __launch_bounds__(kRlThreads) route_logits_kernel(RouteArgs a, f
   constexpr int kQ = 4;       // groups per thread in flight
   if (a.x) {
     const float* __restrict__ x = a.x;
-    for (int t = warp; t < T; t += kRlThreads / 32) {
-      const float inv = rms_inv_warp(x + (size_t)t * H, H, a.eps);
-      if (lane == 0) sinv[t] = inv;
-    }
-    __syncthreads();
+    rms_inv_rows<kRlThreads>(x, T, H, a.eps, red, sinv);  // red is free until the MMA
     uint16_t* __restrict__ hout = a.hidden_out;
     for (int q0 = threadIdx.x; q0 < nq; q0 += kRlThreads * kQ) {
       float4 v[kQ];
@@ -228,8 +224,8 @@ __global__ void __launch_bounds__(kRsThreads) route_select_kernel(RouteArgs a, c
     }
   }
   __syncthreads();
-  if (a.counts)
-    block_bucket(sid, T * k, E, scnt, scr, a.counts, a.offsets, a.perm, a.inv, a.active);
+  if (a.counts && warp == 0)
+    warp_bucket(sid, T * k, E, scnt, a.counts, a.offsets, a.perm, a.inv, a.active);
 }
 
 // ---------------------------------------------------------------- launchers

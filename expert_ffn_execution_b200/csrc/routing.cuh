@@ -1,4 +1,4 @@
-// routing.cuh -- block-level top-k and bucketing shared by the standalone
+// routing.cuh -- warp-level top-k and bucketing shared by the standalone
 // router/bucket kernels and the fused decode routing kernel, so every path
 // produces the same bits.
 #pragma once
@@ -7,54 +7,133 @@
 
 namespace strata {
 
+// Order-preserving 32-bit key of a float logit (-0 counts as +0), and back.
+STRATA_DEVFN uint32_t logit_key(float v) {
+  const uint32_t u = __float_as_uint(v == 0.f ? 0.f : v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+STRATA_DEVFN float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Top-k of one token's logits (shared memory, E <= 32 * NPL) by one warp:
 // the k largest, ties to the lower index, in descending order;
-// w_j = exp(l_j - l_max) / sum_chosen exp(l_i - l_max).  Lane j < k returns
-// the j-th id and weight.
+// w_j = exp(l_j - l_max) / sum_chosen exp(l_i - l_max), summed in rank order.
+// Lane j < k returns the j-th id and weight.  Each round takes the warp's
+// largest key and, among the lanes holding it, the lowest index, with two
+// redux.sync reductions; only the winning lane rescans its values.
 template <int NPL>
 STRATA_DEVFN void warp_topk(const float* lg, int E, int k, int& out_id, float& out_w) {
   const int lane = threadIdx.x & 31;
-  float v[NPL];
+  uint32_t key[NPL];
   uint32_t taken = 0;
 #pragma unroll
   for (int j = 0; j < NPL; ++j) {
     const int e = lane + 32 * j;
-    v[j] = (e < E) ? lg[e] : -INFINITY;
+    key[j] = (e < E) ? logit_key(lg[e]) : 0u;
     if (e >= E) taken |= 1u << j;
   }
-  float lmax = 0.f, sum = 0.f, my_l = 0.f;
-  int my_id = -1;
-  for (int r = 0; r < k; ++r) {
-    float bv = -INFINITY;
-    int bi = 0x7fffffff;
+  uint32_t bk = 0;
+  int bi = 0x7fffffff;
+  auto rescan = [&]() {
+    bk = 0;
+    bi = 0x7fffffff;
 #pragma unroll
     for (int j = 0; j < NPL; ++j) {
       const int e = lane + 32 * j;
-      if (!(taken & (1u << j)) && (v[j] > bv || (v[j] == bv && e < bi))) {
-        bv = v[j];
+      if (!(taken & (1u << j)) && (bi == 0x7fffffff || key[j] > bk)) {
+        bk = key[j];
         bi = e;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
+  };
+  rescan();
+  float lmax = 0.f, sum = 0.f, my_l = 0.f;
+  int my_id = -1;
+  for (int r = 0; r < k; ++r) {
+    const uint32_t m = __reduce_max_sync(0xffffffffu, bk);
+    const uint32_t cand = (bi != 0x7fffffff && bk == m) ? (uint32_t)bi : 0x7fffffffu;
+    const int win = (int)__reduce_min_sync(0xffffffffu, cand);
+    if (win < E && (win & 31) == lane) {
+      taken |= 1u << (win >> 5);
+      rescan();
     }
-    if (bi < E && (bi & 31) == lane) taken |= 1u << (bi >> 5);
+    const float bv = key_logit(m);
     if (r == 0) lmax = bv;
     const float ex = expf(bv - lmax);
     sum += ex;
     if (lane == r) {
-      my_id = (bi < E) ? bi : -1;
+      my_id = (win < E) ? win : -1;
       my_l = ex;
     }
   }
   out_id = my_id;
   out_w = my_l / sum;
+}
+
+// Counting sort of P (token, slot) pairs by expert, stable in pair order, by
+// one warp.  sid[P] holds the pairs' experts (-1: invalid, dropped) in shared
+// memory; scnt is shared scratch of E ints.  P <= 2^20, E <= 2047.
+STRATA_DEVFN void warp_bucket(const int* sid, int P, int E, int* scnt,
+                              int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                              int32_t* __restrict__ active) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int e = lane; e < E; e += 32) scnt[e] = 0;
+  __syncwarp();
+  for (int p = lane; p < P; p += 32)
+    if (sid[p] >= 0) atomicAdd(&scnt[sid[p]], 1);
+  __syncwarp();
+  // each lane owns a contiguous run of experts; one scan of (pairs << 11 | non-empty)
+  const int per = (E + 31) / 32;
+  const int e0 = lane * per, e1 = min(E, e0 + per);
+  uint32_t mine = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = scnt[e];
+    mine += ((uint32_t)c << 11) + (c > 0 ? 1u : 0u);
+  }
+  uint32_t incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t excl = incl - mine;
+  int off = (int)(excl >> 11), apos = (int)(excl & 2047u);
+  for (int e = e0; e < e1; ++e) {
+    const int c = scnt[e];
+    counts[e] = c;
+    offsets[e] = off;
+    if (c > 0) active[1 + apos++] = e;
+    scnt[e] = off;  // becomes the expert's next free sorted position
+    off += c;
+  }
+  if (lane == 31) {
+    offsets[E] = (int)(incl >> 11);
+    active[0] = (int)(incl & 2047u);
+  }
+  __syncwarp();
+  // ranks in pair order, 32 pairs at a time
+  for (int p0 = 0; p0 < P; p0 += 32) {
+    const int p = p0 + lane;
+    const int e = (p < P) ? sid[p] : -2;
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    int base = 0;
+    if (p < P && e >= 0) base = scnt[e];
+    __syncwarp();
+    if (p < P) {
+      if (e >= 0) {
+        const int pos = base + __popc(same & lt);
+        perm[pos] = p;
+        inv[p] = pos;
+        if ((same & lt) == 0) scnt[e] = base + __popc(same);
+      } else {
+        inv[p] = -1;
+      }
+    }
+    __syncwarp();
+  }
 }
 
 // Block-wide exclusive scan of one int per thread; `scratch` holds >= 33 ints.
@@ -83,56 +162,6 @@ STRATA_DEVFN int block_excl_scan_any(int v, int* scratch, int* total) {
   const int r = before + x - v;
   __syncthreads();
   return r;
-}
-
-// Counting sort of P (token, slot) pairs by expert, stable in pair order, by
-// one CTA.  sid[P] holds the pairs' experts (-1: invalid, dropped) in shared
-// memory; scnt is shared scratch of E ints, scr of >= 33 ints.
-STRATA_DEVFN void block_bucket(const int* sid, int P, int E, int* scnt, int* scr,
-                               int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                               int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                               int32_t* __restrict__ active) {
-  for (int e = threadIdx.x; e < E; e += blockDim.x) scnt[e] = 0;
-  __syncthreads();
-  for (int p = threadIdx.x; p < P; p += blockDim.x)
-    if (sid[p] >= 0) atomicAdd(&scnt[sid[p]], 1);
-  __syncthreads();
-  // each thread owns a contiguous run of experts
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int e0 = threadIdx.x * per;
-  int mine = 0, act = 0;
-  for (int e = e0; e < e0 + per && e < E; ++e) {
-    mine += scnt[e];
-    act += scnt[e] > 0;
-  }
-  int total = 0, nact = 0;
-  int off = block_excl_scan_any(mine, scr, &total);
-  int apos = block_excl_scan_any(act, scr, &nact);
-  for (int e = e0; e < e0 + per && e < E; ++e) {
-    const int c = scnt[e];
-    counts[e] = c;
-    offsets[e] = off;
-    if (c > 0) active[1 + apos++] = e;
-    scnt[e] = off;  // becomes the expert's first sorted position
-    off += c;
-  }
-  if (threadIdx.x == 0) {
-    offsets[E] = total;
-    active[0] = nact;
-  }
-  __syncthreads();
-  for (int p = threadIdx.x; p < P; p += blockDim.x) {
-    const int e = sid[p];
-    if (e < 0) {
-      inv[p] = -1;
-      continue;
-    }
-    int rank = 0;
-    for (int p2 = 0; p2 < p; ++p2) rank += (sid[p2] == e);
-    const int pos = scnt[e] + rank;
-    perm[pos] = p;
-    inv[p] = pos;
-  }
 }
 
 }  // namespace strata
