@@ -12,7 +12,8 @@ from ._binding import (DECODE_MAX_T, DEV_BOUNDS, DEV_TIMEOUT, DTYPE_F16, DTYPE_F
                        moe_rmsnorm, moe_route, moe_route_workspace_size, moe_router_topk,
                        moe_router_topk_workspace_size,
                        moe_shared_expert, moe_shared_expert_workspace_size, qweights,
-                       status_string, strata_expert_bytes, strata_read_status)
+                       status_string, strata_expert_bytes, strata_read_status,
+                       strata_selftest_wait)
 from .layer import ExpertWeights, MoELayer
 
 __all__ = [n for n in dir() if not n.startswith("_")]

@@ -45,6 +45,7 @@ _SIGS = {
     "strata_status_string": (ctypes.c_char_p, [_I]),
     "strata_expert_bytes": (_U64, [_I, _I, _I]),
     "strata_read_status": (_I, [_P, _P]),
+    "strata_selftest_wait": (_I, [_U64, _I, _P, _P, _P]),
     "moe_rmsnorm": (_I, [_P, _I, _I, _F, _P, _P]),
     "moe_router_topk_workspace_size": (_U64, [_I, _I, _I, _I]),
     "moe_router_topk": (_I, [_P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _U64, _P, _P]),
@@ -120,6 +121,12 @@ def _qw(w):
 
 
 # ---------------------------------------------------------------- helpers
+def strata_selftest_wait(budget_cycles, complete, dev_status, dev_out, stream=None, check=True):
+    rc = load().strata_selftest_wait(int(budget_cycles), 1 if complete else 0, _ptr(dev_status),
+                                     _ptr(dev_out), _stream(stream))
+    return _check("strata_selftest_wait", rc) if check else rc
+
+
 def abi_version() -> int:
     return load().strata_abi_version()
 

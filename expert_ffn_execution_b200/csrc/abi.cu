@@ -148,6 +148,14 @@ int32_t strata_read_status(const int32_t* dev_status, void* stream) {
   return STRATA_OK;
 }
 
+int32_t strata_selftest_wait(uint64_t budget_cycles, int32_t complete, int32_t* dev_status,
+                             int32_t* dev_out, void* stream) {
+  if (budget_cycles > 4000000000ull || !dev_status || !dev_out || !aligned(dev_out, 4))
+    return STRATA_EINVAL;
+  return from_cuda(launch_wait_selftest((long long)budget_cycles, complete ? 1 : 0, dev_status,
+                                        dev_out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps, uint16_t* hidden,
                     void* stream) {
   if (T < 0 || H < 32 || H > 16384 || H % 8 || !(eps >= 0.f)) return STRATA_EINVAL;

@@ -63,6 +63,8 @@ bool route_decode_supported(int T, int H, int E, int k);
 uint64_t route_decode_workspace_bytes(int T, int H, int E);
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
 
+cudaError_t launch_wait_selftest(long long budget, int complete, int32_t* status, int32_t* out,
+                                 cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int T, int H, float eps, uint16_t* out, cudaStream_t st);
 uint64_t router_workspace_bytes(int T, int H, int E, int k);
 cudaError_t launch_router_topk(const uint16_t* hidden, const uint16_t* wr, const float* bias,

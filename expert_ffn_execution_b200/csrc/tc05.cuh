@@ -13,11 +13,12 @@ namespace strata {
 // STRATA_DEV_TIMEOUT into the status word and returns false.
 constexpr long long kWaitCycles = 4000000000LL;
 
-STRATA_DEVFN bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t* status) {
+STRATA_DEVFN bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t* status,
+                                   long long budget = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > budget) {
       dev_flag(status, STRATA_DEV_TIMEOUT);
       return false;
     }
@@ -28,13 +29,13 @@ STRATA_DEVFN bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t* sta
 // Same, but a CTA-wide abort flag in shared memory short-circuits every later
 // wait once one has timed out, so a broken pipeline ends quickly.
 STRATA_DEVFN bool mbar_wait_guarded(uint64_t* bar, uint32_t parity, int32_t* status,
-                                    volatile int* abort_flag) {
+                                    volatile int* abort_flag, long long budget = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   if (*abort_flag) return false;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > budget) {
       *abort_flag = 1;
       dev_flag(status, STRATA_DEV_TIMEOUT);
       return false;
@@ -47,13 +48,14 @@ STRATA_DEVFN bool mbar_wait_guarded(uint64_t* bar, uint32_t parity, int32_t* sta
 // (epilogue, table), so that their polling does not take issue slots from
 // the warps that share their scheduler.
 STRATA_DEVFN bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, int32_t* status,
-                                    volatile int* abort_flag) {
+                                    volatile int* abort_flag, long long budget = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
+  if (*abort_flag) return false;
   const long long t0 = clock64();
   uint32_t ns = 64;
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitCycles) {
+    if (clock64() - t0 > budget) {
       *abort_flag = 1;
       dev_flag(status, STRATA_DEV_TIMEOUT);
       return false;

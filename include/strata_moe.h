@@ -124,6 +124,22 @@ STRATA_API uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t int
  * STRATA_EBOUNDS (the first set bit, timeout first) or STRATA_ECUDA. */
 STRATA_API int32_t strata_read_status(const int32_t* dev_status, void* stream);
 
+/* Failure-detection self-test of the bounded device waits (the pages have
+ * no counterpart: it checks this library's own error path).  One CTA waits
+ * on an mbarrier with the same bounded waits every kernel uses, first the
+ * pipeline's (abort-flag guarded) wait, then the epilogue's backoff wait.
+ * complete != 0: the barrier's phase is completed first, both waits succeed,
+ * dev_out = {1, 1} and dev_status is untouched.  complete == 0: nothing ever
+ * arrives; the first wait gives up after budget_cycles SM cycles (kernels
+ * use about 4e9, 2 s), ORs STRATA_DEV_TIMEOUT into *dev_status and raises
+ * the CTA's abort flag, the second wait then returns at once, dev_out =
+ * {0, 0}; strata_read_status reports STRATA_ETIMEOUT and the context stays
+ * usable.  Nothing faults, traps or hangs.
+ *   dev_status int32 device word; dev_out int32[2] device.
+ *   budget_cycles <= 4e9, else STRATA_EINVAL.  Asynchronous on `stream`. */
+STRATA_API int32_t strata_selftest_wait(uint64_t budget_cycles, int32_t complete,
+                             int32_t* dev_status, int32_t* dev_out, void* stream);
+
 /* ---------------------------------------------------------------- calls */
 
 /* RMSNorm with unit gain, the layer's input normalisation:
