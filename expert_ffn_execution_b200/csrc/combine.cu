@@ -57,25 +57,28 @@ combine_kernel(const void* __restrict__ y, int y_dtype, const int32_t* __restric
   const int t = blockIdx.x;
   __shared__ int s_pos[32];
   __shared__ float s_w[32];
-  // launched as a programmatic dependent: every input comes from earlier grids
-  pdl_wait_prior();
-  pdl_trigger();
+  const int h = (blockIdx.y * kCombThreads + threadIdx.x) * 8;
+  // Launched as a programmatic dependent.  The routing tables and the
+  // residual come from grids that finished before the preceding one let its
+  // dependents start, so they are read before the wait; the expert outputs
+  // y and shared_y come from the preceding grids and are read after it.
   if (threadIdx.x < k) {
     const int p = t * k + threadIdx.x;
     s_pos[threadIdx.x] = inv[p];
     s_w[threadIdx.x] = w[p];
   }
-  __syncthreads();
-  const int h = (blockIdx.y * kCombThreads + threadIdx.x) * 8;
-  if (h >= H) return;
   float sv[8], rv[8];
-  if (shared_y) load8(shared_y, shared_dtype, (size_t)t * H + h, sv);
-  if (residual_out) {
+  if (residual_out && h < H) {
     const float4 r0 = *reinterpret_cast<const float4*>(residual + (size_t)t * H + h);
     const float4 r1 = *reinterpret_cast<const float4*>(residual + (size_t)t * H + h + 4);
     rv[0] = r0.x; rv[1] = r0.y; rv[2] = r0.z; rv[3] = r0.w;
     rv[4] = r1.x; rv[5] = r1.y; rv[6] = r1.z; rv[7] = r1.w;
   }
+  pdl_wait_prior();
+  pdl_trigger();
+  __syncthreads();
+  if (h >= H) return;
+  if (shared_y) load8(shared_y, shared_dtype, (size_t)t * H + h, sv);
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;

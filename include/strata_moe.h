@@ -262,7 +262,13 @@ STRATA_API int32_t moe_shared_expert(const uint16_t* hidden, const strata_qweigh
  *   shared_y [T,H] or NULL, shared_dtype as y_dtype
  *   residual fp32 [T,H] or NULL (required if residual_out != NULL)
  *   out      bf16 [T,H];  residual_out fp32 [T,H] or NULL (may alias residual)
- * H multiple of 8; all row pointers 16-byte aligned. */
+ * H multiple of 8; all row pointers 16-byte aligned.
+ * The kernel is a programmatic dependent launch: it reads inv, topk_w and
+ * residual before waiting for the preceding kernel of the stream, and y and
+ * shared_y after.  So inv, topk_w and residual must not be written by the
+ * immediately preceding kernel if that kernel releases its dependents early
+ * (griddepcontrol.launch_dependents); this library's expert kernels write
+ * only y / shared_y, and ordinary kernels release nothing early. */
 STRATA_API int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* inv,
                     const float* topk_w, const void* shared_y,
                     int32_t shared_dtype, const float* residual, int32_t T,
