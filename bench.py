@@ -13,7 +13,8 @@ resident in HBM, device-timed with CUDA events over exactly --steps steps
 between a barrier + synchronize on both sides (max over ranks).  `e2e` is the
 same metric with each step's input copied host->device from pinned memory
 and its result copied back inside the timed region.  `roofline` is the
-moe_experts stage (decode gate/up and down kernels) measured live with
+moe_experts stage (decode: the counter reset and the fused gate/up + down
+kernel, or the gate/up and down kernels) measured live with
 external CUDA events captured in the step graphs, against algorithmic bytes.
 
 --impl reference times the CPU oracle (the only reference implementation this
@@ -229,8 +230,9 @@ class DecodeStack:
 
 def kernels_per_layer(T, k, shared):
     """Kernel launches the library enqueues per layer.  Decode (T <= 16):
-    moe_route 2 (logits with RMSNorm; top-k and bucket), experts 2 (gate/up,
-    down), shared expert 2, combine 1.  Prefill: moe_route 7 (RMSNorm,
+    moe_route 2 (logits with RMSNorm; top-k and bucket), experts 2 (counter
+    reset and the fused gate/up + down kernel, or gate/up and down), shared
+    expert 2, combine 1.  Prefill: moe_route 7 (RMSNorm,
     router GEMM, top-k, bucket histogram, column scan, offsets, scatter),
     experts 4 (plan, gather, gate/up GEMM, down GEMM), shared expert 4,
     combine 1."""
@@ -377,7 +379,7 @@ def run_ours(args):
             "e2e": {"value": round(e2e, 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4},
             "gpu_launches": kernels_per_layer(T, k, cfg.shared_fmt is not None) * L * args.steps,
-            "roofline": ({"kernel": "moe_experts decode stage (gate/up + down kernels)",
+            "roofline": ({"kernel": "moe_experts decode stage (fused gate/up + down kernel)",
                           "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                           "unit": "GB/s", "frac": round(achieved / hbm, 4),
                           "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, burst)"

@@ -50,7 +50,8 @@ bool decode_supported(const strata_qweights* w) {
 
 uint64_t experts_ws(const strata_qweights* w, int T, int k, int shared) {
   const int P = shared ? T : T * k;
-  if (T <= kDecodeMaxTokens) return up256((uint64_t)P * w->inter * 2);
+  // decode: h fp16 [P, I], then one progress counter per active expert
+  if (T <= kDecodeMaxTokens) return up256((uint64_t)P * w->inter * 2) + up256((uint64_t)P * 4);
   return prefill_workspace_bytes(T, w->hidden, w->inter, shared ? 1 : w->num_experts, shared ? 1 : k,
                                  shared);
 }
@@ -77,11 +78,15 @@ int32_t run_experts(const uint16_t* hidden, const strata_qweights* w, const int3
     a.active = active;
     a.shared_mode = shared;
     a.hbuf = reinterpret_cast<uint16_t*>(ws);
+    const int P = shared ? T : T * k;
+    a.sync = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) +
+                                        up256((uint64_t)P * w->inter * 2));
     a.y = reinterpret_cast<float*>(y);
     a.status = status;
     a.num_sms = num_sms_of_current_device();
     (void)ws_bytes;
-    if (decode_tc_supported(T, w->hidden, w->inter, shared ? 1 : E, w->fmt, a.num_sms))
+    const int Umax = shared ? 1 : std::min(E, P);
+    if (decode_tc_supported(T, w->hidden, w->inter, Umax, w->fmt, a.num_sms))
       return from_cuda(launch_experts_decode_tc(a, st));
     if (decode_smem_bytes(T, w->hidden) > 200u * 1024u) return STRATA_EUNSUPPORTED;
     return from_cuda(launch_experts_decode(a, st));
@@ -432,14 +437,17 @@ int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router, c
 // all free HBM up front (weights plus a cache pool), where a cudaMalloc in the
 // middle of a step would fail and a cudaFree would synchronise the device.
 // The call allocates nothing: no cudaMalloc, cudaFree or allocating library
-// routine.  Its only scratch is the fp16 SwiGLU activation h [T*k, I].
+// routine.  Its scratch is the fp16 SwiGLU activation h [T*k, I] and the
+// per-expert progress counters of the fused decode kernel.
 //
 // Every call on a device shares the one array, which keeps the last call's
-// contents.  Nothing in it must start at zero: the down kernel reads only the
-// h rows that the gate/up kernel of the same call wrote.  Calls whose kernels
-// overlap on the GPU (other streams, other host threads) race on the array.
+// contents.  Nothing in it must start at zero: the down tiles read only the
+// h rows that the gate/up tiles of the same call wrote, and each call zeroes
+// its counters before the kernel that uses them.  Calls whose kernels overlap
+// on the GPU (other streams, other host threads) race on the array.
 namespace {
-constexpr uint64_t kStaticScratchBytes = 2ull << 20;  // T*k*I <= 1,048,576 fp16
+constexpr uint64_t kStaticHBytes = 2ull << 20;  // T*k*I <= 1,048,576 fp16
+constexpr uint64_t kStaticScratchBytes = kStaticHBytes + 4096;  // + T*k <= 512 counters
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_experts_static_scratch[kStaticScratchBytes];
@@ -471,7 +479,7 @@ extern "C" int32_t moe_experts_static_scratch(const uint16_t* hidden, const stra
   if (!valid_weights(w) || T < 0 || k < 1 || k > w->num_experts || k > 32) return STRATA_EINVAL;
   if (w->num_experts > 1024) return STRATA_EINVAL;
   // sizes beyond the array (or beyond the decode path) are rejected up front
-  if (T > kDecodeMaxTokens || (uint64_t)T * k * w->inter * 2 > kStaticScratchBytes)
+  if (T > kDecodeMaxTokens || (uint64_t)T * k * w->inter * 2 > kStaticHBytes)
     return STRATA_EUNSUPPORTED;
   if (T == 0) return STRATA_OK;
   if (!hidden || !offsets || !perm || !active || !y) return STRATA_EINVAL;

@@ -116,6 +116,21 @@ STRATA_DEVFN bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same, but the thread may be suspended (off the issue slots) until the
+// phase completes or up to kSuspendHintNs have passed.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+STRATA_DEVFN bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait for phase `parity` of the barrier.
 STRATA_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
   for (uint32_t i = 0; i < kWaitLimit; ++i)

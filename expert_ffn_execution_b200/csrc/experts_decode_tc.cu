@@ -10,18 +10,39 @@
 // through shared memory, whose bandwidth would otherwise cap the path.  Codes
 // and scales arrive by TMA into a ring of shared-memory stages.
 //
-// Two kernels per call, chained by programmatic dependent launch:
-//   gate/up  tiles of 64 rows of I: lanes 0-63 decode the gate rows, lanes
-//            64-127 the same up rows.  B = every token of the call, so a tile
-//            computes all T columns and the epilogue keeps the tokens routed
-//            to the tile's expert: h = SwiGLU(gate, up) -> fp16 [P, I] in
-//            sorted pair order, K permuted within 16-groups the way the down
-//            kernel's decode orders K.
-//   down     tiles of 128 rows of H of one expert.  B = that expert's h rows
-//            (TMA from h); y fp32 [P, H] in sorted order.
+// Two kinds of tile:
+//   gate/up  64 rows of I: lanes 0-63 decode the gate rows, lanes 64-127 the
+//            same up rows.  B = every token of the call, so a tile computes
+//            all T columns and the epilogue keeps the tokens routed to the
+//            tile's expert: h = SwiGLU(gate, up) -> fp16 [P, I] in sorted pair
+//            order, K permuted within 16-groups the way the down tiles'
+//            decode orders K.
+//   down     128 rows of H of one expert.  B = that expert's h rows (TMA from
+//            h); y fp32 [P, H] in sorted order.
+// and three kernel forms (MODE):
+//   2  fused: one launch runs both kinds.  Each CTA takes its gate/up tiles
+//      round robin, then a share of the down tiles chosen so that every CTA
+//      has about the same weighted work (a gate/up tile costs H, a down tile
+//      I plus a fixed overhead, in 64-column units).  Down tiles are dealt in
+//      rounds counted back from each CTA's last tile, from the end of the
+//      expert order: the experts whose gate/up tiles finish last become the
+//      last tile of many CTAs rather than all tiles of a few, and the extra
+//      down tiles of CTAs with fewer gate/up tiles come from the experts that
+//      are ready first.  A down
+//      tile's h block is loaded once its expert's gate/up tiles are all done:
+//      each gate/up epilogue publishes its h rows and then counts itself in a
+//      per-expert counter (release); the producer polls it (acquire, bounded)
+//      before the TMA.  The counters are zeroed by a one-thread-block kernel
+//      launched just before, so the workspace needs no initial contents.
+//   0, 1  gate/up alone, then down alone (chained by programmatic dependent
+//      launch): used when the fused form's shared memory leaves too few
+//      stages.
+// Every CTA of a fused grid is resident at once (one per SM, grid <= SMs),
+// and a CTA's gate/up tiles depend on nothing outside it, so the waits on the
+// counters always end; they are bounded all the same.
 //
 // One persistent CTA per SM with a static tile list.  Warps:
-//   0-3   epilogue: tcgen05.ld of their TMEM lane quarter
+//   0-3   epilogue: tcgen05.ld of their TMEM lane quarter (and the tile table)
 //   4..   decoders: kTcGroups groups of four warps taking K chunks in turn;
 //         a thread owns one tile row (= TMEM lane), reads its codes from
 //         the swizzled stage (conflict-free), decodes to fp16 and stores them
@@ -51,6 +72,9 @@ constexpr int kTcACol0 = 64;      // A stage t at columns 64 + 128 t (accumulato
 constexpr int kTcTmemCols = 512;
 constexpr int kTcMaxStages = 16;
 constexpr int kTcSmemBudget = 227 * 1024;
+constexpr int kTcFusedMinStages = 9;  // fewer: run the two-kernel form
+constexpr int kTcDownOverhead = 4;    // per-down-tile cost beyond its K, 64-column units
+constexpr int kTcMaxGrid = 1024;      // the fused tile dealing keeps one int per CTA
 // Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
 // only after the MMAs of its previous one retired, so with at least as many
 // stages as groups no waiter runs two phases ahead of a stage's barrier.
@@ -68,9 +92,15 @@ struct TcParams {
   uint16_t* hbuf;  // gate/up output, down input: fp16 [P, I]
   float* y;        // down output: fp32 [P, H]
   int32_t* status;
+  int32_t* sync;   // fused form: finished gate/up tiles per active expert (zeroed)
   int S;           // shared-memory stages (a multiple of kTcGroups)
   int NB;          // B rows: 8 (T <= 8; rows 8-15 of the MMA repeat them) or 16
   int maxT;        // capacity of the tile table: tiles per CTA at most
+};
+
+struct TcTile {
+  int e, rb, s0, n, u;  // expert, row block, first sorted slot, pairs, active index
+  int tok[16];          // gate/up: token of each of the expert's pairs
 };
 
 template <int FMT>
@@ -78,38 +108,87 @@ __host__ __device__ constexpr int tc_cbr() {  // code bytes per row per chunk
   return FMT == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
 }
 
+// ---------------------------------------------------------------- fused dealing
+// Gate/up tiles go round robin: CTA c has q + (c < r) of them (ntA = qG + r).
+// Down tiles: CTA c gets bstart(c+1) - bstart(c), where bstart(c) =
+// clamp(floor(F(c) / (G costB)), 0, ntB) and F(c) = c Tot - G costA A(c),
+// A(c) = c q + min(c, r) the gate/up tiles of CTAs below c and Tot the
+// weighted total: each CTA's weighted work is then Tot / G within one down
+// tile.  F is linear with F(0) = 0 and F(G) = G ntB costB; its slope above r
+// is positive, below r possibly negative (then those CTAs get no down tile),
+// so bstart is non-decreasing and ends at ntB.
+struct TcDeal {
+  int G, ntA, ntB, q, r;
+  long long costA, costB, tot;
+};
+
+__host__ __device__ inline TcDeal tc_deal(int G, int U, int H, int I) {
+  TcDeal d;
+  d.G = G;
+  d.ntA = U * (I / 64);
+  d.ntB = U * (H / 128);
+  d.q = d.ntA / G;
+  d.r = d.ntA - d.q * G;
+  d.costA = H / 64;
+  d.costB = I / 64 + kTcDownOverhead;
+  d.tot = (long long)d.ntA * d.costA + (long long)d.ntB * d.costB;
+  return d;
+}
+
+__host__ __device__ inline int tc_deal_bstart(const TcDeal& d, int c) {
+  const long long a = (long long)c * d.q + (c < d.r ? c : d.r);
+  const long long F = (long long)c * d.tot - (long long)d.G * d.costA * a;
+  if (F <= 0) return 0;
+  const long long s = F / ((long long)d.G * d.costB);
+  return (int)(s < d.ntB ? s : d.ntB);
+}
+
+// Most tiles a CTA gets for any U <= Umax (the tile-table capacity):
+// ceil(ntA / G) gate/up tiles plus at most slope / (G costB) + 1 down tiles.
+__host__ __device__ inline int tc_deal_max_tiles(int G, int Umax, int H, int I) {
+  const TcDeal d = tc_deal(G, Umax, H, I);
+  const long long nb = ((long long)G * d.costA + (long long)d.ntB * d.costB) / (G * d.costB) + 2;
+  return (d.ntA + G - 1) / G + (int)nb;
+}
+
 struct TcLayout {
-  uint32_t codes_bytes, stage_bytes, b, b_bytes, sbuf, s_bytes, xch, tbl, bars, total;
+  uint32_t codes_bytes, stage_bytes, b, b_bytes, hb, hb_bytes, sbuf, s_bytes, xch, tbl, bars,
+      total;
 };
 
 __host__ __device__ inline uint32_t up1k(uint32_t x) { return (x + 1023u) & ~1023u; }
 
-// Shared memory, from a 1024-byte aligned base: S stages | B (gate/up: one
-// token block; down: two h blocks) | down: two per-tile scale blocks |
-// gate/up: the SwiGLU exchange buffer | the tile table (maxT entries of 80
-// bytes) | barriers.
+// Shared memory, from a 1024-byte aligned base: S stages | gate/up: the token
+// block | down: two h blocks | down: two per-tile scale blocks | gate/up: the
+// SwiGLU exchange buffer (also the fused form's dealing scratch) | the tile
+// table | barriers.  Every TMA destination is 1024-byte aligned.
 __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, int I, int S,
                                               int maxT) {
   TcLayout L;
+  const bool gu = mode != 1, dn = mode != 0;
   const uint32_t cbr = fmt == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
   L.codes_bytes = 128u * cbr;
-  L.stage_bytes = L.codes_bytes + (mode == 0 ? 128u * 16u : 0u);
+  L.stage_bytes = L.codes_bytes + (gu ? 128u * 16u : 0u);
   uint32_t off = (uint32_t)S * L.stage_bytes;
   L.b = off;
-  L.b_bytes = (uint32_t)NB * (uint32_t)(mode == 0 ? H : I) * 2u;
-  off += (mode == 0 ? 1u : 2u) * L.b_bytes;
+  L.b_bytes = gu ? (uint32_t)NB * (uint32_t)H * 2u : 0u;
+  off += L.b_bytes;
+  L.hb = off;
+  L.hb_bytes = dn ? (uint32_t)NB * (uint32_t)I * 2u : 0u;
+  off += 2u * L.hb_bytes;
   L.sbuf = off;
-  L.s_bytes = mode == 1 ? up1k(8u * (uint32_t)I) : 0u;
+  L.s_bytes = dn ? up1k(8u * (uint32_t)I) : 0u;
   off += 2u * L.s_bytes;
   L.xch = off;
-  off += mode == 0 ? up1k(2u * 64u * 17u * 4u) : 0u;
+  off += gu ? up1k(2u * 64u * 17u * 4u) : 0u;
   L.tbl = off;
-  off += up1k(80u * (uint32_t)maxT);
+  off += up1k((uint32_t)sizeof(TcTile) * (uint32_t)maxT);
   L.bars = off;
   off += 1024u;
   L.total = off;
   return L;
 }
+static_assert(2 * 64 * 17 * 4 >= 4 * kTcMaxGrid, "dealing scratch fits the exchange buffer");
 
 // ---------------------------------------------------------------- decode
 // One Q2 word (16 codes, element j at bits 2j) -> R[i] = fp16x2 (element i,
@@ -198,39 +277,18 @@ STRATA_DEVFN void fill_tokens(uint8_t* bsm, const uint16_t* __restrict__ hidden,
   }
 }
 
-struct TcTile {
-  int e, rb, s0, n;
-  int tok[16];  // gate/up: token of each of the expert's pairs
-};
-
-// The CTA's tiles: round robin for gate/up (B is shared by all tiles),
-// contiguous ranges for down (consecutive tiles share an expert's h block).
-struct TcSched {
-  int tb, tstep, tcount;
-};
-template <int MODE>
-STRATA_DEVFN TcSched tc_sched(int ntot) {
-  TcSched q;
-  if (MODE == 0) {
-    q.tb = blockIdx.x;
-    q.tstep = gridDim.x;
-    q.tcount = ntot > q.tb ? (ntot - q.tb + q.tstep - 1) / q.tstep : 0;
-  } else {
-    q.tb = (int)((long long)ntot * blockIdx.x / gridDim.x);
-    q.tstep = 1;
-    q.tcount = (int)((long long)ntot * (blockIdx.x + 1) / gridDim.x) - q.tb;
-  }
-  return q;
-}
 
 // ---------------------------------------------------------------- kernel
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down codes
-                 const __grid_constant__ CUtensorMap mc1,  // up codes   | h [P, I]
-                 const __grid_constant__ CUtensorMap ms0,  // gate scales | unused
-                 const __grid_constant__ CUtensorMap ms1,  // up scales   | unused
+decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
+                 const __grid_constant__ CUtensorMap mu,   // up codes
+                 const __grid_constant__ CUtensorMap msg,  // gate scales
+                 const __grid_constant__ CUtensorMap msu,  // up scales
+                 const __grid_constant__ CUtensorMap md,   // down codes
+                 const __grid_constant__ CUtensorMap mh,   // h [P, I]
                  const TcParams p) {
+  constexpr bool kGU = MODE != 1, kDN = MODE != 0;
   constexpr int CBR = tc_cbr<FMT>();
   constexpr int PIECE_K = (FMT == STRATA_FMT_Q2_32) ? 64 : 32;  // K per 16-byte code piece
   constexpr int NPC = CBR / 16;                                  // pieces per full chunk
@@ -257,10 +315,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.H, I = p.I, T = p.T;
-  const int K = (MODE == 0) ? H : I;
-  const int nch = (K + kTcKC - 1) / kTcKC;
-  const int tpe = (MODE == 0) ? I / 64 : H / 128;  // tiles per expert
+  const int nchA = H / kTcKC;                // H % 256 == 0
+  const int nchB = (I + kTcKC - 1) / kTcKC;  // I % 128 == 0: the last chunk may be 128 wide
+  const int tpeA = I / 64, tpeB = H / 128;   // tiles per expert
   const Planes PL = plane_offsets(FMT, H, I);
+  const int G = gridDim.x, cta = blockIdx.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -289,11 +348,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
     tmem_relinquish();
   }
   if (threadIdx.x == kTcProdWarp * 32) {
-    prefetch_tensormap(&mc0);
-    prefetch_tensormap(&mc1);
-    if constexpr (MODE == 0) {
-      prefetch_tensormap(&ms0);
-      prefetch_tensormap(&ms1);
+    if constexpr (kGU) {
+      prefetch_tensormap(&mg);
+      prefetch_tensormap(&mu);
+      prefetch_tensormap(&msg);
+      prefetch_tensormap(&msu);
+    }
+    if constexpr (kDN) {
+      prefetch_tensormap(&md);
+      prefetch_tensormap(&mh);
     }
   }
   tc_fence_before();
@@ -302,90 +365,147 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
   const uint32_t tmem_base = *tmem_slot;
   // Dependents are released only after this CTA holds its tensor memory (a
   // dependent CTA that allocated first on this SM and then waited for this
-  // grid would never get it back), and, for gate/up, after the routing
-  // tables it reads are complete: the down grid reads them before its wait.
-  if constexpr (MODE == 0) pdl_wait_prior();
+  // grid would never get it back), and, when gate/up tiles run here, after
+  // the routing tables it reads are complete: a down-only grid reads them
+  // before its wait.
+  if constexpr (kGU) pdl_wait_prior();
   pdl_trigger();
 
-  // ---- the CTA's tiles
+  // ---- the CTA's tiles: nA gate/up tiles, then nB down tiles
   int U = p.shared_mode ? 1 : p.active[0];
-  if (U < 0 || U > p.E) {
+  const int Pn = p.shared_mode ? 1 : T * p.k;
+  if (U < 0 || U > p.E || U > Pn) {
     if (threadIdx.x == 0) dev_flag(p.status, STRATA_DEV_BOUNDS);
     U = 0;
   }
-  const TcSched sq = tc_sched<MODE>(U * tpe);
-  int tcount = sq.tcount;
-  if (tcount > p.maxT) {
-    if (threadIdx.x == 0) dev_flag(p.status, STRATA_DEV_BOUNDS);
-    tcount = p.maxT;
+  int nA = 0, nB = 0, b0 = 0;
+  TcDeal deal{};
+  if constexpr (MODE == 0) {
+    const int ntA = U * tpeA;
+    nA = ntA > cta ? (ntA - cta + G - 1) / G : 0;
+  } else if constexpr (MODE == 1) {
+    const int ntB = U * tpeB;  // contiguous ranges: consecutive tiles share an h block
+    b0 = (int)((long long)ntB * cta / G);
+    nB = (int)((long long)ntB * (cta + 1) / G) - b0;
+  } else {
+    deal = tc_deal(G, U, H, I);
+    nA = deal.q + (cta < deal.r ? 1 : 0);
+    nB = tc_deal_bstart(deal, cta + 1) - tc_deal_bstart(deal, cta);
   }
-  // expert of the CTA's i-th tile, straight from the routing tables
-  auto tile_e = [&](int i, int& rb) {
-    const int j = sq.tb + i * sq.tstep;
-    const int u = j / tpe;
-    rb = j - u * tpe;
+  if (nA + nB > p.maxT) {
+    if (threadIdx.x == 0) dev_flag(p.status, STRATA_DEV_BOUNDS);
+    nA = min(nA, p.maxT);
+    nB = p.maxT - nA;
+  }
+  const int tcount = nA + nB;
+  // expert of an active-list index, straight from the routing tables
+  auto expert_of = [&](int u) {
     if (p.shared_mode) return 0;
     const int e = p.active[1 + u];
     return (e < 0 || e >= p.E) ? 0 : e;
+  };
+  // gate/up tile i: round robin over the grid
+  auto tile_a = [&](int i, int& u, int& rb) {
+    const int j = cta + i * G;
+    u = j / tpeA;
+    rb = j - u * tpeA;
+  };
+  // down tile i of the down-only form: a contiguous range
+  auto tile_b1 = [&](int i, int& u, int& rb) {
+    const int j = b0 + (i - nA);
+    u = j / tpeB;
+    rb = j - u * tpeB;
   };
 
   if (warp == kTcProdWarp) {
     // ------------------------------------------------ TMA producer
     if (elect_one()) {
       int gc = 0, bseq = -1, prev_e = -1;
-      auto issue = [&](int e, int rb, int c) {
+      auto next_stage = [&](uint32_t tx) {
         const int s = gc % S;
         mbar_wait_guarded(&empty[s], ((gc / S) & 1) ^ 1, p.status, abort_flag);
-        uint8_t* st = smem + s * L.stage_bytes;
-        if constexpr (MODE == 0) {
-          mbar_arrive_expect_tx(&full[s], L.stage_bytes);
-          tma_load_3d(st, &mc0, c * CBR, rb * 64, e, &full[s]);
-          tma_load_3d(st + 64 * CBR, &mc1, c * CBR, rb * 64, e, &full[s]);
-          tma_load_3d(st + L.codes_bytes, &ms0, c * 8, rb * 64, e, &full[s]);
-          tma_load_3d(st + L.codes_bytes + 1024, &ms1, c * 8, rb * 64, e, &full[s]);
-        } else {
-          mbar_arrive_expect_tx(&full[s], L.codes_bytes);
-          tma_load_3d(st, &mc0, c * CBR, rb * 128, e, &full[s]);
-        }
+        mbar_arrive_expect_tx(&full[s], tx);
         ++gc;
+        return s;
+      };
+      // the expert's h rows [s0, s0 + NB) into the next B buffer
+      auto load_h = [&](int e) {
+        ++bseq;
+        const int b = bseq & 1;
+        const int s0 = p.shared_mode ? 0 : p.offsets[e];
+        mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
+        const uint32_t ab = (uint32_t)p.NB * 128u;
+        mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
+        for (int a = 0; a < I / 64; ++a)
+          tma_load_2d(smem + L.hb + b * L.hb_bytes + a * ab, &mh, 64 * a, s0, &bfull[b]);
       };
       for (int i = 0; i < tcount; ++i) {
-        int rb;
-        const int e = tile_e(i, rb);
-        int pre = 0;
-        if constexpr (MODE == 1) {
+        if (kGU && (MODE == 0 || i < nA)) {
+          int u, rb;
+          tile_a(i, u, rb);
+          const int e = expert_of(u);
+          for (int c = 0; c < nchA; ++c) {
+            const int s = next_stage(L.codes_bytes + 128u * 16u);
+            uint8_t* st = smem + s * L.stage_bytes;
+            tma_load_3d(st, &mg, c * CBR, rb * 64, e, &full[s]);
+            tma_load_3d(st + 64 * CBR, &mu, c * CBR, rb * 64, e, &full[s]);
+            tma_load_3d(st + L.codes_bytes, &msg, c * 8, rb * 64, e, &full[s]);
+            tma_load_3d(st + L.codes_bytes + 1024, &msu, c * 8, rb * 64, e, &full[s]);
+          }
+          continue;
+        }
+        if constexpr (kDN) {
+          const int ib = i - nA;  // down-tile sequence number
+          int u, rb;
+          if constexpr (MODE == 1) {
+            tile_b1(i, u, rb);
+          } else {
+            if (ib == 0) mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
+            u = tbl[i].u;
+            rb = tbl[i].rb;
+          }
+          const int e = expert_of(u);
           // the tile's scales: rows rb*128.. of the down plane, all of K
-          const int sb = i & 1;
-          mbar_wait_guarded(&sempty[sb], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
+          const int sb = ib & 1;
+          mbar_wait_guarded(&sempty[sb], ((ib >> 1) & 1) ^ 1, p.status, abort_flag);
           mbar_arrive_expect_tx(&sfull[sb], 8u * I);
           bulk_g2s(smem + L.sbuf + sb * L.s_bytes,
                    p.wbase + (uint64_t)e * p.stride + PL.scales[2] +
                        (uint64_t)rb * 128u * (uint64_t)(I / 16),
                    8u * I, &sfull[sb]);
-          // first tile: the weight chunks go out before the wait for h
-          pre = (i == 0) ? min(nch, S) : 0;
-          for (int c = 0; c < pre; ++c) issue(e, rb, c);
-          if (i == 0 || e != prev_e) {
-            ++bseq;
-            if (bseq == 0) pdl_wait_prior();  // h is written by the preceding grid
-            const int b = bseq & 1;
-            const int s0 = p.shared_mode ? 0 : p.offsets[e];
-            mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
-            const uint32_t ab = (uint32_t)p.NB * 128u;
-            mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
-            for (int a = 0; a < I / 64; ++a)
-              tma_load_2d(smem + L.b + b * L.b_bytes + a * ab, &mc1, 64 * a, s0, &bfull[b]);
+          auto issue_b = [&](int c) {
+            const int s = next_stage(L.codes_bytes);
+            tma_load_3d(smem + s * L.stage_bytes, &md, c * CBR, rb * 128, e, &full[s]);
+          };
+          const bool new_h = ib == 0 || e != prev_e;
+          if constexpr (MODE == 1) {
+            // first tile: the weight chunks go out before the wait for h
+            const int pre = (ib == 0) ? min(nchB, S) : 0;
+            for (int c = 0; c < pre; ++c) issue_b(c);
+            if (new_h) {
+              if (bseq < 0) pdl_wait_prior();  // h is written by the preceding grid
+              load_h(e);
+            }
+            for (int c = pre; c < nchB; ++c) issue_b(c);
+          } else {
+            for (int c = 0; c < nchB; ++c) issue_b(c);
+            if (new_h) {
+              // the expert's h is complete once each of its gate/up tiles
+              // has counted itself; then read it through the async proxy
+              gmem_wait_geq(p.sync + u, tpeA, p.status, abort_flag);
+              fence_proxy_async_global();
+              load_h(e);
+            }
           }
+          prev_e = e;
         }
-        for (int c = pre; c < nch; ++c) issue(e, rb, c);
-        prev_e = e;
       }
     }
     __syncwarp();
   } else {
     // ---- everyone else: the gate/up B operand, then (epilogue warps) the
     // tile table
-    if constexpr (MODE == 0) {
+    if constexpr (kGU) {
       // the producer warp is not among the fillers: renumber the warps after it
       const int ftid = warp < kTcProdWarp ? (int)threadIdx.x : (int)threadIdx.x - 32;
       fill_tokens<FMT>(smem + L.b, p.hidden, T, H, p.NB, ftid, (kTcWarps - 1) * 32);
@@ -394,16 +514,47 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
     }
     if (warp < 4) {
       const int r = threadIdx.x;
+      int* bcnt = reinterpret_cast<int*>(smem + L.xch);  // fused: down tiles of every CTA
+      if constexpr (MODE == 2) {
+        for (int c2 = r; c2 < G; c2 += 128)
+          bcnt[c2] = tc_deal_bstart(deal, c2 + 1) - tc_deal_bstart(deal, c2);
+        named_bar_sync(1, 128);
+      }
       for (int i = r; i < tcount; i += 128) {
         TcTile& t = tbl[i];
-        t.e = tile_e(i, t.rb);
+        int u, rb;
+        if (kGU && (MODE == 0 || i < nA)) {
+          tile_a(i, u, rb);
+        } else if (MODE == 1) {
+          tile_b1(i, u, rb);
+        } else {
+          // rounds are counted back from each CTA's last tile (k2 = 0) and
+          // take the down tiles from the end of the expert order: k2 = 0 is
+          // every CTA's last tile, from the experts that become ready last;
+          // the rounds only CTAs with fewer gate/up tiles reach take the
+          // experts that are ready first.  Tile = every tile of the rounds
+          // before k2, then the k2-th tiles of the CTAs below this one.
+          const int k2 = bcnt[cta] - 1 - (i - nA);
+          int jp = 0;
+          for (int c2 = 0; c2 < G; ++c2) {
+            const int b = bcnt[c2];
+            jp += min(b, k2) + ((c2 < cta && b > k2) ? 1 : 0);
+          }
+          const int j = deal.ntB - 1 - jp;
+          u = j / tpeB;
+          rb = j - u * tpeB;
+        }
+        t.u = u;
+        t.rb = rb;
+        t.e = expert_of(u);
         if (p.shared_mode) {
           t.s0 = 0;
           t.n = T;
         } else {
           t.s0 = p.offsets[t.e];
           t.n = p.offsets[t.e + 1] - t.s0;
-          if (p.active[1 + (sq.tb + i * sq.tstep) / tpe] != t.e) {  // invalid expert id
+          const int eraw = p.active[1 + u];
+          if (eraw < 0 || eraw >= p.E) {  // invalid expert id
             dev_flag(p.status, STRATA_DEV_BOUNDS);
             t.n = 0;
           }
@@ -414,8 +565,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
         }
       }
       named_bar_sync(1, 128);
-      if constexpr (MODE == 0) {
-        for (int x = r; x < tcount * 16; x += 128) {
+      if constexpr (kGU) {
+        for (int x = r; x < nA * 16; x += 128) {
           TcTile& t = tbl[x >> 4];
           const int j = x & 15;
           if (j < t.n) {
@@ -447,7 +598,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(&aempty[a]);
-      if constexpr (MODE == 0) {
+      if (kGU && (MODE == 0 || i < nA)) {
         float* xr = xch + r * 17;  // rows 0-63 gate, 64-127 up
 #pragma unroll
         for (int j = 0; j < 16; ++j) xr[j] = __uint_as_float(v[j]);
@@ -461,8 +612,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
           const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
           p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(__float2half_rn(h));
         }
+        if constexpr (MODE == 2) {
+          // publish this thread's h stores (to the TMA reads of other CTAs)
+          fence_proxy_async_global();
+          __threadfence();
+        }
         named_bar_sync(1, 128);
-      } else {
+        if constexpr (MODE == 2) {
+          if (r == 0) atomicAdd(p.sync + ti.u, 1);  // after every thread's fence
+        }
+      } else if constexpr (kDN) {
         const int row = ti.rb * 128 + r;
 #pragma unroll
         for (int j = 0; j < 16; ++j)
@@ -479,10 +638,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
     const Q4Table T4 = q4_table();
     int gc = 0;
     for (int i = 0; i < tcount; ++i) {
+      const bool isA = kGU && (MODE == 0 || i < nA);
+      const int ib = i - nA;
+      const int K = isA ? H : I;
+      const int nch = isA ? nchA : nchB;
       const uint8_t* srow = nullptr;
-      if constexpr (MODE == 1) {
-        mbar_wait_guarded(&sfull[i & 1], (i >> 1) & 1, p.status, abort_flag);
-        srow = smem + L.sbuf + (i & 1) * L.s_bytes + r * (I / 16);
+      if (!isA) {
+        mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
+        srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
       }
       for (int c = 0; c < nch; ++c, ++gc) {
         if (gc % kTcGroups != g) continue;
@@ -496,7 +659,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
         for (int pc = 0; pc < NPC; ++pc)
           cw[pc] = (pc < np) ? lds128(st + r * CBR + ((pc ^ swz) << 4)) : make_uint4(0, 0, 0, 0);
         uint32_t sc[4];
-        if constexpr (MODE == 0) {
+        if (isA) {
           const uint4 v = lds128(st + L.codes_bytes + r * 16);
           sc[0] = v.x;
           sc[1] = v.y;
@@ -558,9 +721,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
         tc_fence_before();
         mbar_arrive(&tfull[t]);
       }
-      if constexpr (MODE == 1) {
+      if (!isA) {
         fence_proxy_async_smem();  // same for the scale block and its next bulk copy
-        mbar_arrive(&sempty[i & 1]);
+        mbar_arrive(&sempty[ib & 1]);
       }
     }
   } else if (warp == kTcMmaWarp) {
@@ -574,19 +737,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
       const uint64_t d_atom = ab >> 4, d_k16 = 32 >> 4;
       int gc = 0, bseq = -1, prev_e = -1;
       for (int i = 0; i < tcount; ++i) {
+        const bool isA = kGU && (MODE == 0 || i < nA);
         uint32_t bbase = smem_addr(smem + L.b);
         int b = 0;
-        if constexpr (MODE == 1) {
+        if (!isA) {
+          if (MODE == 2 && i == nA) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
           const int e = tbl[i].e;
-          if (i == 0 || e != prev_e) {
+          if (i == nA || e != prev_e) {
             ++bseq;
             mbar_wait_guarded(&bfull[bseq & 1], (bseq >> 1) & 1, p.status, abort_flag);
             tc_fence_after();
           }
           prev_e = e;
           b = bseq & 1;
-          bbase += (uint32_t)b * L.b_bytes;
+          bbase = smem_addr(smem + L.hb) + (uint32_t)b * L.hb_bytes;
         }
+        const int K = isA ? H : I;
+        const int nch = isA ? nchA : nchB;
         const int a = i & 1;
         mbar_wait_guarded(&aempty[a], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
         tc_fence_after();
@@ -609,7 +776,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
           mma_commit(&tempty[t]);
         }
         mma_commit(&afull[a]);
-        if constexpr (MODE == 1) {
+        if (!isA) {
           if (i + 1 == tcount || tbl[i + 1].e != tbl[i].e) mma_commit(&bempty[b]);
         }
       }
@@ -627,12 +794,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mc0,  // gate codes | down 
   }
 }
 
+// Zeroes the fused form's counters.  It releases its dependent (the fused
+// grid, which may then set up) at once, but writes only after the grid before
+// it, which may be a fused grid still counting, has finished; the fused grid
+// reads the counters after waiting for this one.
+__global__ void __launch_bounds__(128) tc_sync_reset_kernel(int32_t* sync, int n) {
+  pdl_trigger();
+  pdl_wait_prior();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) sync[i] = 0;
+}
+
 // ---------------------------------------------------------------- host side
 namespace {
 
-// Tiles per CTA at most (the tile-table capacity): every expert active.
-int tc_max_tiles(int mode, int E, int H, int I, int grid) {
-  const long long ntot = (long long)E * (mode == 0 ? I / 64 : H / 128);
+// Tiles per CTA at most (the tile-table capacity) with at most Umax active
+// experts.
+int tc_max_tiles(int mode, int Umax, int H, int I, int grid) {
+  if (mode == 2) return tc_deal_max_tiles(grid, Umax, H, I);
+  const long long ntot = (long long)Umax * (mode == 0 ? I / 64 : H / 128);
   return (int)std::max<long long>(1, (ntot + grid - 1) / grid);
 }
 
@@ -648,77 +827,103 @@ int tc_stages(int mode, int fmt, int NB, int H, int I, int maxT) {
   return s - s % kTcGroups;
 }
 
+void pdl_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, int threads,
+                size_t smem, cudaStream_t st) {
+  cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(threads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+}
+
 template <int MODE, int FMT>
-cudaError_t launch_tc(const CUtensorMap& m0, const CUtensorMap& m1, const CUtensorMap& m2,
-                      const CUtensorMap& m3, const TcParams& prm, int grid, cudaStream_t st) {
+cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, cudaStream_t st) {
   auto kern = decode_tc_kernel<MODE, FMT>;
   const size_t smem = 1024 + tc_layout(MODE, FMT, prm.NB, prm.H, prm.I, prm.S, prm.maxT).total;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
+  cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, m0, m1, m2, m3, prm);
+  pdl_config(cfg, attr, grid, kTcThreads, smem, st);
+  return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], prm);
+}
+
+cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  pdl_config(cfg, attr, 1, 128, 0, st);
+  return cudaLaunchKernelEx(&cfg, tc_sync_reset_kernel, sync, n);
+}
+
+bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
+  return grid <= kTcMaxGrid &&
+         tc_stages(2, fmt, NB, H, I, tc_max_tiles(2, Umax, H, I, grid)) >= kTcFusedMinStages;
 }
 
 }  // namespace
 
-bool decode_tc_supported(int T, int H, int I, int E, int fmt, int grid) {
-  if (T < 1 || T > kDecodeMaxTokens || H % 256 || I % 128 || grid < 1) return false;
+bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid) {
+  if (T < 1 || T > kDecodeMaxTokens || H % 256 || I % 128 || grid < 1 || Umax < 1) return false;
   const int NB = T <= 8 ? 8 : 16;
-  return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, E, H, I, grid)) >= kTcGroups &&
-         tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, E, H, I, grid)) >= kTcGroups;
+  return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, Umax, H, I, grid)) >= kTcGroups &&
+         tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, Umax, H, I, grid)) >= kTcGroups;
+}
+
+bool decode_tc_fused(int T, int H, int I, int Umax, int fmt, int grid) {
+  return decode_tc_supported(T, H, I, Umax, fmt, grid) &&
+         tc_fused_fits(T <= 8 ? 8 : 16, H, I, Umax, fmt, grid);
 }
 
 cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   const int E = a.shared_mode ? 1 : a.E;
-  if (!decode_tc_supported(a.T, a.H, a.I, E, a.fmt, a.num_sms)) return cudaErrorNotSupported;
-  const int NB = a.T <= 8 ? 8 : 16;
   const long long P = a.shared_mode ? a.T : (long long)a.T * a.k;
+  const int Umax = a.shared_mode ? 1 : (int)std::min<long long>(a.E, P);
+  if (!decode_tc_supported(a.T, a.H, a.I, Umax, a.fmt, a.num_sms)) return cudaErrorNotSupported;
+  const int NB = a.T <= 8 ? 8 : 16;
   const Planes PL = plane_offsets(a.fmt, a.H, a.I);
   const bool q2 = a.fmt == STRATA_FMT_Q2_32;
   const cuuint32_t cbr = q2 ? kTcKC / 4 : kTcKC / 2;
   const CUtensorMapSwizzle sw = cbr == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   const cuuint64_t rowH = codes_row_bytes(a.fmt, a.H), rowI = codes_row_bytes(a.fmt, a.I);
-  CUtensorMap mg, mu, msg, msu, md, mh;
+  CUtensorMap m[6];  // gate codes, up codes, gate scales, up scales, down codes, h
   {
     const cuuint64_t dims[3] = {rowH, (cuuint64_t)a.I, (cuuint64_t)E};
     const cuuint64_t str[2] = {rowH, a.stride};
     const cuuint32_t box[3] = {cbr, 64, 1};
-    if (!make_tmap(&mg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[0], dims, str, box, sw) ||
-        !make_tmap(&mu, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[1], dims, str, box, sw))
+    if (!make_tmap(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[0], dims, str, box,
+                   sw) ||
+        !make_tmap(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[1], dims, str, box,
+                   sw))
       return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[3] = {(cuuint64_t)a.H / 32, (cuuint64_t)a.I, (cuuint64_t)E};
     const cuuint64_t str[2] = {(cuuint64_t)a.H / 16, a.stride};
     const cuuint32_t box[3] = {8, 64, 1};
-    if (!make_tmap(&msg, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, a.wbase + PL.scales[0], dims, str, box,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !make_tmap(&msu, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, a.wbase + PL.scales[1], dims, str, box,
-                   CU_TENSOR_MAP_SWIZZLE_NONE))
+    if (!make_tmap(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, a.wbase + PL.scales[0], dims, str,
+                   box, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tmap(&m[3], CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, a.wbase + PL.scales[1], dims, str,
+                   box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[3] = {rowI, (cuuint64_t)a.H, (cuuint64_t)E};
     const cuuint64_t str[2] = {rowI, a.stride};
     const cuuint32_t box[3] = {cbr, 128, 1};
-    if (!make_tmap(&md, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[2], dims, str, box, sw))
+    if (!make_tmap(&m[4], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[2], dims, str, box,
+                   sw))
       return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)a.I, (cuuint64_t)P};
     const cuuint64_t str[1] = {(cuuint64_t)a.I * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)NB};
-    if (!make_tmap(&mh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.hbuf, dims, str, box,
+    if (!make_tmap(&m[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.hbuf, dims, str, box,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
@@ -738,19 +943,27 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.hbuf = a.hbuf;
   prm.y = a.y;
   prm.status = a.status;
+  prm.sync = a.sync;
   prm.NB = NB;
   cudaError_t e;
-  prm.maxT = tc_max_tiles(0, E, a.H, a.I, a.num_sms);
+  if (a.sync && tc_fused_fits(NB, a.H, a.I, Umax, a.fmt, a.num_sms)) {
+    prm.maxT = tc_max_tiles(2, Umax, a.H, a.I, a.num_sms);
+    prm.S = tc_stages(2, a.fmt, NB, a.H, a.I, prm.maxT);
+    if ((e = launch_sync_reset(a.sync, Umax, st)) != cudaSuccess) return e;
+    if (q2) return launch_tc<2, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
+    return launch_tc<2, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+  }
+  prm.maxT = tc_max_tiles(0, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);
   if (q2)
-    e = launch_tc<0, STRATA_FMT_Q2_32>(mg, mu, msg, msu, prm, a.num_sms, st);
+    e = launch_tc<0, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
   else
-    e = launch_tc<0, STRATA_FMT_Q4CB_32>(mg, mu, msg, msu, prm, a.num_sms, st);
+    e = launch_tc<0, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
   if (e != cudaSuccess) return e;
-  prm.maxT = tc_max_tiles(1, E, a.H, a.I, a.num_sms);
+  prm.maxT = tc_max_tiles(1, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(1, a.fmt, NB, a.H, a.I, prm.maxT);
-  if (q2) return launch_tc<1, STRATA_FMT_Q2_32>(md, mh, md, md, prm, a.num_sms, st);
-  return launch_tc<1, STRATA_FMT_Q4CB_32>(md, mh, md, md, prm, a.num_sms, st);
+  if (q2) return launch_tc<1, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
+  return launch_tc<1, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
 }
 
 }  // namespace strata

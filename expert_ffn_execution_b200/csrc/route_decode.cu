@@ -16,7 +16,7 @@
 //                 into part[hs][t][e].
 //   route_select  one CTA: logits = sum over hs in order + bias, then the
 //                 per-token top-k (one warp per token) and the stable counting
-//                 sort of the T*k pairs.
+//                 sort of the T*k pairs (the whole CTA).
 // Every sum runs in a fixed order, so the results do not depend on timing.
 #include "routing.cuh"
 #include "tc05.cuh"
@@ -224,8 +224,7 @@ __global__ void __launch_bounds__(kRsThreads) route_select_kernel(RouteArgs a, c
     }
   }
   __syncthreads();
-  if (a.counts && warp == 0)
-    warp_bucket(sid, T * k, E, scnt, a.counts, a.offsets, a.perm, a.inv, a.active);
+  if (a.counts) block_bucket(sid, T * k, E, scnt, scr, a.counts, a.offsets, a.perm, a.inv, a.active);
 }
 
 // ---------------------------------------------------------------- launchers

@@ -1,6 +1,6 @@
-// routing.cuh -- warp-level top-k and bucketing shared by the standalone
-// router/bucket kernels and the fused decode routing kernel, so every path
-// produces the same bits.
+// routing.cuh -- the top-k (one warp per token) shared by the router kernels,
+// so every routing path produces the same bits, the block-wide bucketing of
+// the decode routing kernel, and a block-wide scan.
 #pragma once
 
 #include "decode.cuh"
@@ -71,35 +71,36 @@ STRATA_DEVFN void warp_topk(const float* lg, int E, int k, int& out_id, float& o
   out_w = my_l / sum;
 }
 
+// Block-wide exclusive scan of one int per thread; `scratch` holds >= 33 ints.
+STRATA_DEVFN int block_excl_scan_any(int v, int* scratch, int* total);
+
 // Counting sort of P (token, slot) pairs by expert, stable in pair order, by
-// one warp.  sid[P] holds the pairs' experts (-1: invalid, dropped) in shared
-// memory; scnt is shared scratch of E ints.  P <= 2^20, E <= 2047.
-STRATA_DEVFN void warp_bucket(const int* sid, int P, int E, int* scnt,
-                              int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                              int32_t* __restrict__ active) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int e = lane; e < E; e += 32) scnt[e] = 0;
-  __syncwarp();
-  for (int p = lane; p < P; p += 32)
+// the whole block (every thread calls it).  sid[P] holds the pairs' experts
+// (-1: invalid, dropped) in shared memory; scnt is shared scratch of E ints,
+// scr of 33.  P <= 2^20, E <= 2047.  Each thread owns a contiguous run of
+// experts; one block scan of (pairs << 11 | non-empty) gives both the sorted
+// offsets and the positions in the active list.  Warp 0 then ranks the
+// pairs, 32 at a time, in pair order.
+STRATA_DEVFN void block_bucket(const int* sid, int P, int E, int* scnt, int* scr,
+                               int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                               int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                               int32_t* __restrict__ active) {
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const int lane = tid & 31;
+  for (int e = tid; e < E; e += nth) scnt[e] = 0;
+  __syncthreads();
+  for (int p = tid; p < P; p += nth)
     if (sid[p] >= 0) atomicAdd(&scnt[sid[p]], 1);
-  __syncwarp();
-  // each lane owns a contiguous run of experts; one scan of (pairs << 11 | non-empty)
-  const int per = (E + 31) / 32;
-  const int e0 = lane * per, e1 = min(E, e0 + per);
+  __syncthreads();
+  const int per = (E + nth - 1) / nth;
+  const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
   uint32_t mine = 0;
   for (int e = e0; e < e1; ++e) {
     const int c = scnt[e];
     mine += ((uint32_t)c << 11) + (c > 0 ? 1u : 0u);
   }
-  uint32_t incl = mine;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const uint32_t excl = incl - mine;
+  int tot = 0;
+  const uint32_t excl = (uint32_t)block_excl_scan_any((int)mine, scr, &tot);
   int off = (int)(excl >> 11), apos = (int)(excl & 2047u);
   for (int e = e0; e < e1; ++e) {
     const int c = scnt[e];
@@ -109,34 +110,35 @@ STRATA_DEVFN void warp_bucket(const int* sid, int P, int E, int* scnt,
     scnt[e] = off;  // becomes the expert's next free sorted position
     off += c;
   }
-  if (lane == 31) {
-    offsets[E] = (int)(incl >> 11);
-    active[0] = (int)(incl & 2047u);
+  if (tid == 0) {
+    offsets[E] = (int)((uint32_t)tot >> 11);
+    active[0] = (int)((uint32_t)tot & 2047u);
   }
-  __syncwarp();
-  // ranks in pair order, 32 pairs at a time
-  for (int p0 = 0; p0 < P; p0 += 32) {
-    const int p = p0 + lane;
-    const int e = (p < P) ? sid[p] : -2;
-    const uint32_t same = __match_any_sync(0xffffffffu, e);
-    int base = 0;
-    if (p < P && e >= 0) base = scnt[e];
-    __syncwarp();
-    if (p < P) {
-      if (e >= 0) {
-        const int pos = base + __popc(same & lt);
-        perm[pos] = p;
-        inv[p] = pos;
-        if ((same & lt) == 0) scnt[e] = base + __popc(same);
-      } else {
-        inv[p] = -1;
+  __syncthreads();
+  if (tid < 32) {
+    const uint32_t lt = (1u << lane) - 1u;
+    for (int p0 = 0; p0 < P; p0 += 32) {
+      const int p = p0 + lane;
+      const int e = (p < P) ? sid[p] : -2;
+      const uint32_t same = __match_any_sync(0xffffffffu, e);
+      int base = 0;
+      if (p < P && e >= 0) base = scnt[e];
+      __syncwarp();
+      if (p < P) {
+        if (e >= 0) {
+          const int pos = base + __popc(same & lt);
+          perm[pos] = p;
+          inv[p] = pos;
+          if ((same & lt) == 0) scnt[e] = base + __popc(same);
+        } else {
+          inv[p] = -1;
+        }
       }
+      __syncwarp();
     }
-    __syncwarp();
   }
 }
 
-// Block-wide exclusive scan of one int per thread; `scratch` holds >= 33 ints.
 STRATA_DEVFN int block_excl_scan_any(int v, int* scratch, int* total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
   int x = v;

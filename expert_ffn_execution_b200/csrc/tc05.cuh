@@ -10,14 +10,16 @@ namespace strata {
 
 // ---------------------------------------------------------------- bounded waits
 // A wait gives up after ~kWaitCycles SM cycles (about 2 s), ORs
-// STRATA_DEV_TIMEOUT into the status word and returns false.
+// STRATA_DEV_TIMEOUT into the status word and returns false.  Between its
+// checks of the budget (and of the abort flag) the waiting thread sleeps in
+// mbarrier.try_wait until the phase completes or the suspend hint runs out.
 constexpr long long kWaitCycles = 4000000000LL;
 
 STRATA_DEVFN bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, int32_t* status,
                                    long long budget = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity)) {
     if (clock64() - t0 > budget) {
       dev_flag(status, STRATA_DEV_TIMEOUT);
       return false;
@@ -33,7 +35,7 @@ STRATA_DEVFN bool mbar_wait_guarded(uint64_t* bar, uint32_t parity, int32_t* sta
   if (mbar_try_wait(bar, parity)) return true;
   if (*abort_flag) return false;
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity)) {
     if (*abort_flag) return false;
     if (clock64() - t0 > budget) {
       *abort_flag = 1;
@@ -44,16 +46,24 @@ STRATA_DEVFN bool mbar_wait_guarded(uint64_t* bar, uint32_t parity, int32_t* sta
   return true;
 }
 
-// Same, polling with a nanosleep backoff: for warps off the critical path
-// (epilogue, table), so that their polling does not take issue slots from
-// the warps that share their scheduler.
+// The wait of the warps off the critical path (epilogue, table).  It was a
+// nanosleep backoff; with the suspending try_wait above it is the same wait.
 STRATA_DEVFN bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, int32_t* status,
                                     volatile int* abort_flag, long long budget = kWaitCycles) {
-  if (mbar_try_wait(bar, parity)) return true;
-  if (*abort_flag) return false;
+  return mbar_wait_guarded(bar, parity, status, abort_flag, budget);
+}
+
+// Wait until a global counter written by other CTAs of the grid reaches
+// `target` (acquire at GPU scope), polling with a nanosleep backoff; bounded
+// like the waits above.
+STRATA_DEVFN bool gmem_wait_geq(const int32_t* ptr, int target, int32_t* status,
+                                volatile int* abort_flag, long long budget = kWaitCycles) {
   const long long t0 = clock64();
-  uint32_t ns = 64;
-  while (!mbar_try_wait(bar, parity)) {
+  uint32_t ns = 32;
+  while (true) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    if (v >= target) return true;
     if (*abort_flag) return false;
     if (clock64() - t0 > budget) {
       *abort_flag = 1;
@@ -61,9 +71,13 @@ STRATA_DEVFN bool mbar_wait_backoff(uint64_t* bar, uint32_t parity, int32_t* sta
       return false;
     }
     __nanosleep(ns);
-    if (ns < 512) ns <<= 1;
+    if (ns < 256) ns <<= 1;
   }
-  return true;
+}
+
+// Generic-proxy global accesses <-> async-proxy (TMA) global accesses.
+STRATA_DEVFN void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Add expected transaction bytes to the current phase without arriving.
