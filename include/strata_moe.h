@@ -207,7 +207,9 @@ STRATA_API int32_t moe_route(const float* x, int32_t T, int32_t H, float eps,
  * with fp32 accumulation (the SwiGLU expert FFN; the pages' experts are run by
  * the GPU when resident, Strata review "success idea one" step 2).
  *   y: [P,H] in SORTED order.  T <= STRATA_DECODE_MAX_T: fp32 (decode path,
- *      weight-streaming dequant-GEMV).  T > STRATA_DECODE_MAX_T: fp16 (prefill
+ *      weight-streaming dequant-GEMV; gate/up and down tiles run in one
+ *      kernel, after a one-CTA kernel that zeroes the per-expert counters
+ *      it keeps in the workspace).  T > STRATA_DECODE_MAX_T: fp16 (prefill
  *      path, tcgen05 grouped GEMM over dequantised fp16 tiles).
  *   offsets/perm/active: as written by moe_bucket for the same (T, k, E).
  * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket. */
@@ -225,7 +227,8 @@ STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
  * HBM (weights plus a cache pool), where a cudaMalloc during a step would fail
  * and a cudaFree would synchronise the device.  The call allocates nothing (no
  * cudaMalloc, cudaFree or allocating library routine); its scratch, the fp16
- * activations h [T*k, I], lives in one file-scope 2 MiB array of the library.
+ * activations h [T*k, I] (up to 2 MiB) and T*k progress counters, lives in one
+ * file-scope array of the library.
  *   Limit: T <= STRATA_DECODE_MAX_T and T*k*I <= 1,048,576 (2 MiB of fp16);
  *   beyond it the call returns STRATA_EUNSUPPORTED and launches nothing.
  *   Set-up: the first call on each device, with that device current, looks
@@ -233,9 +236,10 @@ STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
  *   that first call before any stream capture.  A failed lookup returns
  *   STRATA_ECUDA.
  *   Sharing: all calls on a device use the same array, which keeps the last
- *   call's contents; no part of it has to start at zero (each call reads only
- *   the h rows it wrote).  Calls that overlap on the GPU (other streams, other
- *   host threads) race on the array: serialise them.
+ *   call's contents; no part of it has to start at zero (each call zeroes its
+ *   counters before use and reads only the h rows it wrote).  Calls that
+ *   overlap on the GPU (other streams, other host threads) race on the
+ *   array: serialise them.
  * Other arguments, the output y (fp32 [T*k, H], sorted order) and the other
  * errors are those of moe_experts. */
 STRATA_API int32_t moe_experts_static_scratch(const uint16_t* hidden, const strata_qweights* w,
