@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(kRlThreads) route_logits_kernel(RouteArgs a, f
 
 template <int NPL>
 __global__ void __launch_bounds__(kRsThreads) route_select_kernel(RouteArgs a, const float* part) {
-  extern __shared__ __align__(16) uint8_t smem[];
+  extern __shared__ __align__(128) uint8_t smem[];
   const int T = a.T, E = a.E, k = a.k;
   const int HS = route_hsplit(a.H, E);
   float* lg = reinterpret_cast<float*>(smem);

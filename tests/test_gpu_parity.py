@@ -186,6 +186,22 @@ def test_decode_small_expert_count_and_k1():
     check_layer(r)
 
 
+def test_decode_large_down_scales():
+    """Down-projection block scales of 82..328 (2^14 times the C1 range, on
+    both sides of 128): the 2-bit decode's fp16 products d*(c-1.5) stay in
+    range and parity holds as for ordinary scales.  Gate/up scales stay as
+    generated so that h stays well inside fp16."""
+    r = Run(1, 4)
+    planes, _ = mi.plane_layout(r.c.fmt, r.H, r.I)
+    _, off, n, _, _, _ = [pl for pl in planes if pl[0] == "down" and pl[5] == "scales"][0]
+    d = r.inp.experts[:, off:off + n].view(torch.float16)
+    d.mul_(2.0 ** 14)
+    big = (d.abs() >= 128).float().mean().item()
+    assert 0.2 < big < 0.9, big  # both forms are exercised
+    r.run()
+    check_layer(r)
+
+
 @pytest.mark.parametrize("config,T", [(1, 4), (4, 8)])
 def test_decode_deterministic(config, T):
     a = Run(config, T).run()
