@@ -79,9 +79,8 @@ STRATA_DEVFN float warp_sum(float v) {
 namespace strata {
 
 // ---------------------------------------------------------------- mbarrier / bulk copy
-// Every wait is bounded: after kWaitLimit polls it gives up, ORs
-// STRATA_DEV_TIMEOUT into the status word and returns false.
-constexpr uint32_t kWaitLimit = 1u << 26;
+// The bounded waits built on these (a cycle budget, STRATA_DEV_TIMEOUT on
+// expiry) are in tc05.cuh.
 
 STRATA_DEVFN uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -129,14 +128,6 @@ STRATA_DEVFN bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
       : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
-}
-
-// Bounded wait for phase `parity` of the barrier.
-STRATA_DEVFN bool mbar_wait(uint64_t* bar, uint32_t parity, int32_t* status) {
-  for (uint32_t i = 0; i < kWaitLimit; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  dev_flag(status, STRATA_DEV_TIMEOUT);
-  return false;
 }
 
 // 1-D bulk copy global -> this CTA's shared memory; completion is counted on

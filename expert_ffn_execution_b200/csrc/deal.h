@@ -1,0 +1,75 @@
+// deal.h -- how the fused decode kernel deals its tiles to the CTAs of one
+// grid.  Plain integer arithmetic, compiled for the device by the kernel and
+// for the host by the library and by a CPU test of the dealing itself.
+#pragma once
+
+#ifdef __CUDACC__
+#define STRATA_HD __host__ __device__
+#else
+#define STRATA_HD
+#endif
+
+namespace strata {
+
+constexpr int kTcDownOverhead = 4;  // per-down-tile cost beyond its K, 64-column units
+
+// Gate/up tiles go round robin: CTA c has q + (c < r) of them (ntA = qG + r).
+// Down tiles: CTA c gets bstart(c+1) - bstart(c), where bstart(c) =
+// clamp(floor(F(c) / (G costB)), 0, ntB) and F(c) = c Tot - G costA A(c),
+// A(c) = c q + min(c, r) the gate/up tiles of CTAs below c and Tot the
+// weighted total: each CTA's weighted work is then Tot / G within one down
+// tile.  F is linear with F(0) = 0 and F(G) = G ntB costB; its slope above r
+// is positive, below r possibly negative (then those CTAs get no down tile),
+// so bstart is non-decreasing and ends at ntB.
+struct TcDeal {
+  int G, ntA, ntB, q, r;
+  long long costA, costB, tot;
+};
+
+STRATA_HD inline TcDeal tc_deal(int G, int U, int H, int I) {
+  TcDeal d;
+  d.G = G;
+  d.ntA = U * (I / 64);
+  d.ntB = U * (H / 128);
+  d.q = d.ntA / G;
+  d.r = d.ntA - d.q * G;
+  d.costA = H / 64;
+  d.costB = I / 64 + kTcDownOverhead;
+  d.tot = (long long)d.ntA * d.costA + (long long)d.ntB * d.costB;
+  return d;
+}
+
+STRATA_HD inline int tc_deal_bstart(const TcDeal& d, int c) {
+  const long long a = (long long)c * d.q + (c < d.r ? c : d.r);
+  const long long F = (long long)c * d.tot - (long long)d.G * d.costA * a;
+  if (F <= 0) return 0;
+  const long long s = F / ((long long)d.G * d.costB);
+  return (int)(s < d.ntB ? s : d.ntB);
+}
+
+// Most tiles a CTA gets for any U <= Umax (the tile-table capacity):
+// ceil(ntA / G) gate/up tiles plus at most slope / (G costB) + 1 down tiles.
+STRATA_HD inline int tc_deal_max_tiles(int G, int Umax, int H, int I) {
+  const TcDeal d = tc_deal(G, Umax, H, I);
+  const long long nb = ((long long)G * d.costA + (long long)d.ntB * d.costB) / (G * d.costB) + 2;
+  return (d.ntA + G - 1) / G + (int)nb;
+}
+
+// Down tile (expert-major index) of the kk-th down tile of CTA `cta`, given
+// every CTA's down-tile count bcnt[G].  Rounds are counted back from each
+// CTA's last tile (k2 = 0) and take the down tiles from the end of the
+// expert order: k2 = 0 is every CTA's last tile, from the experts that become
+// ready last; the rounds only CTAs with fewer gate/up tiles reach take the
+// experts that are ready first.  Index = every tile of the rounds before k2,
+// then the k2-th tiles of the CTAs below this one, counted from the end.
+STRATA_HD inline int tc_deal_down_tile(const TcDeal& d, const int* bcnt, int cta, int kk) {
+  const int k2 = bcnt[cta] - 1 - kk;
+  int jp = 0;
+  for (int c2 = 0; c2 < d.G; ++c2) {
+    const int b = bcnt[c2];
+    jp += (b < k2 ? b : k2) + ((c2 < cta && b > k2) ? 1 : 0);
+  }
+  return d.ntB - 1 - jp;
+}
+
+}  // namespace strata

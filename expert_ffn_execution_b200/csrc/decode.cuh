@@ -26,7 +26,6 @@ cudaError_t launch_experts_decode(const DecodeArgs& a, cudaStream_t st);
 size_t decode_smem_bytes(int T, int H);
 // Umax: most active experts of a call (1 for the shared expert, else min(E, T*k)).
 bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid);
-bool decode_tc_fused(int T, int H, int I, int Umax, int fmt, int grid);
 cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st);
 
 struct PrefillArgs {

@@ -55,6 +55,7 @@
 // per-tile scales, per-expert h block).  Every wait is bounded.
 #include <algorithm>
 
+#include "deal.h"
 #include "decode.cuh"
 #include "tc05.cuh"
 #include "tmap.h"
@@ -73,7 +74,6 @@ constexpr int kTcTmemCols = 512;
 constexpr int kTcMaxStages = 16;
 constexpr int kTcSmemBudget = 227 * 1024;
 constexpr int kTcFusedMinStages = 9;  // fewer: run the two-kernel form
-constexpr int kTcDownOverhead = 4;    // per-down-tile cost beyond its K, 64-column units
 constexpr int kTcMaxGrid = 1024;      // the fused tile dealing keeps one int per CTA
 // Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
 // only after the MMAs of its previous one retired, so with at least as many
@@ -106,49 +106,6 @@ struct TcTile {
 template <int FMT>
 __host__ __device__ constexpr int tc_cbr() {  // code bytes per row per chunk
   return FMT == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
-}
-
-// ---------------------------------------------------------------- fused dealing
-// Gate/up tiles go round robin: CTA c has q + (c < r) of them (ntA = qG + r).
-// Down tiles: CTA c gets bstart(c+1) - bstart(c), where bstart(c) =
-// clamp(floor(F(c) / (G costB)), 0, ntB) and F(c) = c Tot - G costA A(c),
-// A(c) = c q + min(c, r) the gate/up tiles of CTAs below c and Tot the
-// weighted total: each CTA's weighted work is then Tot / G within one down
-// tile.  F is linear with F(0) = 0 and F(G) = G ntB costB; its slope above r
-// is positive, below r possibly negative (then those CTAs get no down tile),
-// so bstart is non-decreasing and ends at ntB.
-struct TcDeal {
-  int G, ntA, ntB, q, r;
-  long long costA, costB, tot;
-};
-
-__host__ __device__ inline TcDeal tc_deal(int G, int U, int H, int I) {
-  TcDeal d;
-  d.G = G;
-  d.ntA = U * (I / 64);
-  d.ntB = U * (H / 128);
-  d.q = d.ntA / G;
-  d.r = d.ntA - d.q * G;
-  d.costA = H / 64;
-  d.costB = I / 64 + kTcDownOverhead;
-  d.tot = (long long)d.ntA * d.costA + (long long)d.ntB * d.costB;
-  return d;
-}
-
-__host__ __device__ inline int tc_deal_bstart(const TcDeal& d, int c) {
-  const long long a = (long long)c * d.q + (c < d.r ? c : d.r);
-  const long long F = (long long)c * d.tot - (long long)d.G * d.costA * a;
-  if (F <= 0) return 0;
-  const long long s = F / ((long long)d.G * d.costB);
-  return (int)(s < d.ntB ? s : d.ntB);
-}
-
-// Most tiles a CTA gets for any U <= Umax (the tile-table capacity):
-// ceil(ntA / G) gate/up tiles plus at most slope / (G costB) + 1 down tiles.
-__host__ __device__ inline int tc_deal_max_tiles(int G, int Umax, int H, int I) {
-  const TcDeal d = tc_deal(G, Umax, H, I);
-  const long long nb = ((long long)G * d.costA + (long long)d.ntB * d.costB) / (G * d.costB) + 2;
-  return (d.ntA + G - 1) / G + (int)nb;
 }
 
 struct TcLayout {
@@ -528,19 +485,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         } else if (MODE == 1) {
           tile_b1(i, u, rb);
         } else {
-          // rounds are counted back from each CTA's last tile (k2 = 0) and
-          // take the down tiles from the end of the expert order: k2 = 0 is
-          // every CTA's last tile, from the experts that become ready last;
-          // the rounds only CTAs with fewer gate/up tiles reach take the
-          // experts that are ready first.  Tile = every tile of the rounds
-          // before k2, then the k2-th tiles of the CTAs below this one.
-          const int k2 = bcnt[cta] - 1 - (i - nA);
-          int jp = 0;
-          for (int c2 = 0; c2 < G; ++c2) {
-            const int b = bcnt[c2];
-            jp += min(b, k2) + ((c2 < cta && b > k2) ? 1 : 0);
-          }
-          const int j = deal.ntB - 1 - jp;
+          const int j = tc_deal_down_tile(deal, bcnt, cta, i - nA);
           u = j / tpeB;
           rb = j - u * tpeB;
         }
@@ -872,11 +817,6 @@ bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid) {
   const int NB = T <= 8 ? 8 : 16;
   return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, Umax, H, I, grid)) >= kTcGroups &&
          tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, Umax, H, I, grid)) >= kTcGroups;
-}
-
-bool decode_tc_fused(int T, int H, int I, int Umax, int fmt, int grid) {
-  return decode_tc_supported(T, H, I, Umax, fmt, grid) &&
-         tc_fused_fits(T <= 8 ? 8 : 16, H, I, Umax, fmt, grid);
 }
 
 cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
