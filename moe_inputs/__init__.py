@@ -99,6 +99,11 @@ CONFIGS = {
     4: LayerConfig("C4", 4096, 256, 2048, 6, FMT_Q4CB, (0.0005, 0.002), (1, 4, 8192),
                    zipf_s=1.0, shared_fmt=FMT_Q4CB, shared_d_range=(0.0005, 0.002),
                    x_bf16=True, notes="large experts, 4-bit codebook"),
+    # the other reading of config 3: every expert, routed and shared, in the
+    # 4-bit codebook format at E = 512 (reported beside C3, not a parity gate)
+    5: LayerConfig("C3b", 2560, 512, 640, 10, FMT_Q4CB, (0.0005, 0.002), (1, 4),
+                   zipf_s=1.1, shared_fmt=FMT_Q4CB, shared_d_range=(0.0005, 0.002),
+                   notes="C3 with 4-bit-codebook routed experts"),
 }
 
 
