@@ -209,7 +209,9 @@ STRATA_API int32_t moe_route(const float* x, int32_t T, int32_t H, float eps,
  *   y: [P,H] in SORTED order.  T <= STRATA_DECODE_MAX_T: fp32 (decode path,
  *      weight-streaming dequant-GEMV; gate/up and down tiles run in one
  *      kernel, after a one-CTA kernel that zeroes the per-expert counters
- *      it keeps in the workspace).  T > STRATA_DECODE_MAX_T: fp16 (prefill
+ *      it keeps in the workspace, or, where that kernel's shared memory
+ *      leaves too few stages, in a gate/up and a down kernel).
+ *      T > STRATA_DECODE_MAX_T: fp16 (prefill
  *      path, tcgen05 grouped GEMM over dequantised fp16 tiles).
  *   offsets/perm/active: as written by moe_bucket for the same (T, k, E).
  * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket. */
