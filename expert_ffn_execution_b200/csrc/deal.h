@@ -17,10 +17,13 @@ constexpr int kTcDownOverhead = 4;  // per-down-tile cost beyond its K, 64-colum
 // Down tiles: CTA c gets bstart(c+1) - bstart(c), where bstart(c) =
 // clamp(floor(F(c) / (G costB)), 0, ntB) and F(c) = c Tot - G costA A(c),
 // A(c) = c q + min(c, r) the gate/up tiles of CTAs below c and Tot the
-// weighted total: each CTA's weighted work is then Tot / G within one down
-// tile.  F is linear with F(0) = 0 and F(G) = G ntB costB; its slope above r
-// is positive, below r possibly negative (then those CTAs get no down tile),
-// so bstart is non-decreasing and ends at ntB.
+// weighted total.  F(c) / G is how far the CTAs below c fall short of their
+// share c Tot / G after their gate/up tiles; down tiles make it up, so each
+// CTA where F >= 0 at both ends carries Tot / G within one down tile.  F is
+// piecewise linear with F(0) = 0 and F(G) = G ntB costB; its slope above r is
+// positive, below r possibly negative, and where it is negative (the CTAs
+// below already carry more than their share) a CTA gets no down tile, so
+// bstart is non-decreasing and ends at ntB.
 struct TcDeal {
   int G, ntA, ntB, q, r;
   long long costA, costB, tot;

@@ -1,8 +1,10 @@
 // Exhaustive host check of the fused decode kernel's tile dealing (deal.h):
 // for many grid sizes, active-expert counts and shapes, every down tile is
 // dealt to exactly one (CTA, slot), the cut points are non-decreasing and
-// end at the tile count, and no CTA gets more tiles than the table capacity
-// computed for any larger expert count.  Prints "ok <cases>" or the first
+// end at the tile count, every CTA outside the clamped range carries the mean
+// weighted work within one down tile (inside it, none gets a down tile), and
+// no CTA gets more tiles than the
+// table capacity computed for any larger expert count.  Prints "ok <cases>" or the first
 // failure, and exits non-zero on a failure.
 #include <cstdio>
 #include <vector>
@@ -28,8 +30,27 @@ static int check(int G, int U, int Umax, int H, int I) {
     }
     bc[c] = bs[c + 1] - bs[c];
   }
+  // balance: where F >= 0 at both ends of CTA c's range (no clamp), its
+  // weighted work is within one down tile of Tot / G; where F(c+1) < 0 (the
+  // CTAs up to c already carry more than their share) it has no down tile
   for (int c = 0; c < G; ++c) {
     const int nA = d.q + (c < d.r ? 1 : 0);
+    const auto F = [&](int x) {
+      const long long a = (long long)x * d.q + (x < d.r ? x : d.r);
+      return (long long)x * d.tot - (long long)d.G * d.costA * a;
+    };
+    const long long work = (long long)nA * d.costA + (long long)bc[c] * d.costB;  // x G below
+    if (F(c) >= 0 && F(c + 1) >= 0 && bs[c + 1] < d.ntB) {
+      const long long dev = work * G - d.tot;
+      if (dev <= -(long long)G * d.costB || dev >= (long long)G * d.costB) {
+        std::printf("FAIL balance G=%d U=%d c=%d work=%lld tot/G=%lld/%d\n", G, U, c, work, d.tot, G);
+        return 1;
+      }
+    }
+    if (F(c + 1) < 0 && bc[c] != 0) {
+      std::printf("FAIL clamped G=%d U=%d c=%d\n", G, U, c);
+      return 1;
+    }
     if (nA + bc[c] > cap) {
       std::printf("FAIL capacity G=%d U=%d Umax=%d c=%d: %d + %d > %d\n", G, U, Umax, c, nA,
                   bc[c], cap);
