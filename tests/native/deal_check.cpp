@@ -68,8 +68,8 @@ static int check(int G, int U, int Umax, int H, int I) {
 }
 
 int main() {
-  const int shapes[][2] = {{2560, 640}, {256, 128}, {512, 384}, {4096, 1024},
-                           {2048, 1408}, {7168, 2048}};
+  const int shapes[][2] = {{2560, 640}, {256, 128}, {512, 256}, {512, 384}, {4096, 1024},
+                           {4096, 2048}, {2048, 1408}, {7168, 2048}};
   const int grids[] = {1, 2, 3, 7, 64, 132, 148, 160, 1024};
   const int pmax[] = {1, 4, 16, 40, 64, 160, 512};
   long cases = 0;
