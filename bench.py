@@ -1,27 +1,36 @@
 #!/usr/bin/env python3
 """Benchmark of the routed-expert FFN layer on B200.
 
-Default workload (the headline configuration): 48 stacked MoE layers of the
-hidden-2560 / 512-expert / width-640 / top-10 shape with 2-bit (Q2_32) expert
-weights, 37.75 GB resident in HBM, T = 4 tokens per step (one token plus
-three speculative drafts verified together).  One step = for each layer
-RMSNorm -> router/top-k -> bucket -> experts -> combine + residual add, each
-layer a call sequence of the library's C ABI, captured into a CUDA graph.
+Default run: two lines, the headline last.
+  1. config 2: one prefill layer (T = 8192 tokens, 81,920 token-expert pairs)
+     of the hidden-2560 / 512-expert / width-640 / top-10 shape with 2-bit
+     (Q2_32) experts; its roofline is the tensor-core grouped GEMM.
+  2. config 1, the headline: 48 stacked layers of that shape (37.75 GB of
+     2-bit experts resident in HBM), T = 4 tokens per step (one token plus
+     three speculative drafts verified together); its roofline is the
+     weight-streaming experts stage against HBM bandwidth.
+One step = for each layer RMSNorm -> router/top-k -> bucket -> experts ->
+combine + residual add, each layer a call sequence of the library's C ABI,
+captured into a CUDA graph.
 
-Prints one JSON line (rank 0).  `value` is whole-job tokens/s with the inputs
-resident in HBM, device-timed with CUDA events over exactly --steps steps
-between a barrier + synchronize on both sides (max over ranks).  `e2e` is the
-same metric with each step's input copied host->device from pinned memory
-and its result copied back inside the timed region.  `roofline` is the
-moe_experts stage (decode: the counter reset and the fused gate/up + down
-kernel, or the gate/up and down kernels) measured live with
-external CUDA events captured in the step graphs, against algorithmic bytes.
+Each line is one JSON object (rank 0).  `value` is whole-job tokens/s with the
+inputs resident in HBM, device-timed with CUDA events over exactly --steps
+steps between a barrier + synchronize on both sides (max over ranks).  `e2e`
+is the same metric with each step's input copied host->device from pinned
+memory and its result copied back inside the timed region.  `roofline` is the
+moe_experts stage measured live with external CUDA events captured in the
+step graphs, against its algorithmic bytes (decode) or flops (prefill).
+`parity` compares one graph-replayed step, layer by layer, with the CPU
+oracle (teacher-forced: each layer's recorded GPU input): RMSNorm within one
+bf16 ulp, top-k ids exact except listed near-ties, layer output per-token
+relative L2 <= 5e-3.  `cpu_baseline` is the oracle's own time on those same
+checked layers (decode) or sampled tokens (prefill), on the host's cores.
 
 --impl reference times the CPU oracle (the only reference implementation this
-layer has) on the host cores, on a bounded sample of the same workload.
-Multi-GPU (torchrun): every rank holds its own copy of the model and runs its
-own token batches (replicas, weak scaling); there is no collective on the
-data path.
+layer has) on the host cores, on a bounded sample of the headline workload,
+the same way.  Multi-GPU (torchrun): every rank holds its own copy of the
+model and runs its own token batches (replicas, weak scaling); there is no
+collective on the data path.
 """
 from __future__ import annotations
 
@@ -34,6 +43,7 @@ import sys
 import tempfile
 import time
 
+import numpy as np
 import torch
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -44,8 +54,12 @@ import moe_inputs as mi  # noqa: E402
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_SUSTAINED = 1400.0
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 peak"
 NCU_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+DEFAULT_LINES = "2:8192,1:4"   # config:T, run in this order; the last is the headline
+OUT_REL_L2 = 5e-3
+NEAR_TIE_REL = 1e-5
 
 
 def peaks():
@@ -60,9 +74,9 @@ def peaks():
 def sustained_tflops():
     try:
         with open(PEAKS_FILE) as f:
-            return float(json.load(f)["bf16_tflops_sustained"])
+            return float(json.load(f)["bf16_tflops_sustained"]), "measured"
     except Exception:
-        return 1400.0
+        return FALLBACK_BF16_SUSTAINED, "fallback"
 
 
 def dist_env():
@@ -91,6 +105,14 @@ def max_over_ranks(values, device):
 def job_tokens_per_s(tokens_per_step_per_rank, steps, world, ms):
     """Whole-job throughput: the tokens all ranks processed / the job time."""
     return tokens_per_step_per_rank * steps * world / (ms * 1e-3)
+
+
+def parse_lines(spec):
+    out = []
+    for item in spec.split(","):
+        c, t = item.split(":")
+        out.append((int(c), int(t)))
+    return out
 
 
 class Clocks:
@@ -148,7 +170,23 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def u16(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
 # ---------------------------------------------------------------- model
+class Record:
+    """Per-layer snapshots of one step: the layer input (residual stream),
+    the normalised hidden rows, the routing and the MoE output."""
+
+    def __init__(self, L, T, H, k, dev):
+        self.x = torch.empty(L, T, H, dtype=torch.float32, device=dev)
+        self.hidden = torch.empty(L, T, H, dtype=torch.bfloat16, device=dev)
+        self.ids = torch.empty(L, T, k, dtype=torch.int32, device=dev)
+        self.w = torch.empty(L, T, k, dtype=torch.float32, device=dev)
+        self.out = torch.empty(L, T, H, dtype=torch.bfloat16, device=dev)
+
+
 class DecodeStack:
     """L layers of one configuration, weights generated on the device."""
 
@@ -160,6 +198,7 @@ class DecodeStack:
         c = self.c
         self.H, self.E, self.I, self.k = c.H, c.E, c.I, c.k
         self.ebytes = mi.expert_bytes(c.fmt, c.H, c.I)
+        self.sbytes = mi.expert_bytes(c.shared_fmt, c.H, c.I) if c.shared_fmt else 0
         self.wr, self.bias, self.experts, self.qw, self.shared, self.sqw = [], [], [], [], [], []
         for l in range(layers):
             inp = mi.make_layer(config, T, layer=l, device=device, with_experts=False)
@@ -201,9 +240,8 @@ class DecodeStack:
                 sm.moe_shared_expert_workspace_size(self.sqw[0], T) if self.sqw[0] else 0)
         self.ws = torch.empty(int(n) + 256, dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        self.launches_per_step = None
 
-    def step(self, x_in, x_out, active_bufs=None, events=None):
+    def step(self, x_in, x_out, active_bufs, events=None, record: Record | None = None):
         """Enqueue one step (all layers): x_out = x_in after L layers."""
         sm, T, H, E, k = self.sm, self.T, self.H, self.E, self.k
         st = self.status
@@ -212,6 +250,8 @@ class DecodeStack:
         for l in range(self.L):
             nxt = x_out if l == self.L - 1 else (self.xa if (l % 2 == 0) else self.xb)
             act = active_bufs[l]
+            if record is not None:
+                record.x[l].copy_(cur)
             sm.moe_route(cur, T, H, self.c.eps, self.wr[l], self.bias[l], E, k, self.hidden,
                          self.ids, self.w, self.counts, self.offsets, self.perm, self.inv, act,
                          ws, wn, st)
@@ -225,38 +265,146 @@ class DecodeStack:
                 sm.moe_shared_expert(self.hidden, self.sqw[l], T, self.shy, ws, wn, st)
             sm.moe_combine(self.y, self.ydtype, self.inv, self.w, self.shy, self.ydtype, cur, T, k,
                            H, self.out, nxt, st)
+            if record is not None:
+                record.hidden[l].copy_(self.hidden)
+                record.ids[l].copy_(self.ids)
+                record.w[l].copy_(self.w)
+                record.out[l].copy_(self.out)
             cur = nxt
 
 
 def kernels_per_layer(T, k, shared):
     """Kernel launches the library enqueues per layer.  Decode (T <= 16):
     moe_route 2 (logits with RMSNorm; top-k and bucket), experts 2 (counter
-    reset and the fused gate/up + down kernel, or gate/up and down), shared
-    expert 2, combine 1.  Prefill: moe_route 7 (RMSNorm,
-    router GEMM, top-k, bucket histogram, column scan, offsets, scatter),
-    experts 4 (plan, gather, gate/up GEMM, down GEMM), shared expert 4,
-    combine 1."""
+    reset and the fused gate/up + down kernel), shared expert 2, combine 1.
+    Prefill: moe_route 7 (RMSNorm, router GEMM, top-k, bucket histogram,
+    column scan, offsets, scatter), experts 4 (plan, gather, gate/up GEMM,
+    down GEMM), shared expert 4, combine 1."""
     if T <= 16:
         return 2 + 2 + 1 + (2 if shared else 0)
     return 7 + 4 + 1 + (4 if shared else 0)
 
 
-def run_ours(args):
-    ws_, rank, local = dist_env()
-    if ws_ > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    cfg = mi.CONFIGS[args.config]
-    T = args.tokens or cfg.Ts[0]
-    L = args.layers or cfg.layers
-    stack = DecodeStack(args.config, T, L, dev)
+# ---------------------------------------------------------------- oracle side
+def oracle_layer_inputs(stack, l, ids_needed):
+    """Router weights, bias and the blobs of the experts `ids_needed` of
+    layer l of a device stack, on the host."""
+    wr = u16(stack.wr[l])
+    bias = None if stack.bias[l] is None else stack.bias[l].cpu().numpy()
+    blobs = {int(e): stack.experts[l][int(e)].cpu().numpy() for e in np.unique(ids_needed)}
+    sh = None if stack.shared[l] is None else stack.shared[l][0].cpu().numpy()
+    return wr, bias, blobs, sh
+
+
+def rel_l2_rows(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return np.sqrt(((a - b) ** 2).sum(-1)) / np.maximum(np.sqrt((b ** 2).sum(-1)), 1e-30)
+
+
+def _routing_compare(ref_logits, gpu_ids, k):
+    """(exact tokens, near-tie tokens accepted, mismatched tokens) of the GPU
+    ids against the oracle's logits; the tie band is NEAR_TIE_REL."""
+    from tests.harness import check_routing
+    ok, near, bad = check_routing(ref_logits, gpu_ids, k)
+    return near, bad
+
+
+def _near_ties(ref_logits, k, t_offset=0, max_list=16):
+    from tests.harness import near_tie_report
+    return [{"token": t + t_offset, "rank": r, "rel_gap": g}
+            for t, r, g in near_tie_report(ref_logits, None, k, max_list)]
+
+
+def parity_and_oracle_time(stack, rec, args):
+    """Layer-by-layer check of one recorded step against the oracle, and the
+    oracle's own time on that work (the CPU baseline).  Decode: whole layers
+    (every token), teacher-forced on the recorded GPU input of each layer, in
+    layer order until --cpu-seconds of oracle time.  Prefill: router and
+    top-k on every token; the layer on a stratified sample of tokens."""
+    import oracle
+    from tests.harness import parallel_rows, stratified_tokens
+    c, T, H, E, k, L = stack.c, stack.T, stack.H, stack.E, stack.k, stack.L
+    eps = c.eps
+    max_err, ulp_ok, mismatched, near, near_ties, checked = 0.0, True, [], [], [], 0
+    spent, tok_done = 0.0, 0
+    threads = oracle.num_threads()
+    for l in range(L):
+        x_l = rec.x[l].cpu().numpy()
+        hid = u16(rec.hidden[l])
+        gids = rec.ids[l].cpu().numpy()
+        out = oracle.bf16_bits_to_f32(u16(rec.out[l]))
+        ref_h = oracle.rmsnorm(x_l, eps)
+        a = oracle.bf16_bits_to_f32(hid).astype(np.float64)
+        b = oracle.bf16_bits_to_f32(ref_h).astype(np.float64)
+        ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b), 1e-30))) - 7)
+        ulp_ok &= bool(np.all(np.abs(a - b) <= ulp))
+        wr = u16(stack.wr[l])
+        bias = None if stack.bias[l] is None else stack.bias[l].cpu().numpy()
+        ref_lg = np.concatenate(parallel_rows(
+            lambda lo, hi: oracle.router_logits(hid[lo:hi], wr, bias), T, 256))
+        n_l, bad_l = _routing_compare(ref_lg, gids, k)
+        mismatched += [(l, t) for t in bad_l]
+        near += [(l, t) for t in n_l]
+        near_ties += [dict(layer=l, **d) for d in _near_ties(ref_lg, k)]
+        if stack.decode:
+            toks = np.arange(T)
+        else:
+            toks = stratified_tokens(stack.counts.cpu().numpy(), stack.offsets.cpu().numpy(),
+                                     stack.perm.cpu().numpy(), k, T, n=args.prefill_sample,
+                                     seed=l)
+        oracle_ids, _ = oracle.topk(ref_lg[toks], k)
+        _, _, blobs, sh = oracle_layer_inputs(stack, l, np.concatenate([oracle_ids.ravel(),
+                                                                        gids[toks].ravel()]))
+        # the timed oracle call: the whole layer on these tokens, routed by
+        # the oracle itself
+        t0 = time.perf_counter()
+        ref = oracle.moe_layer(hid[toks], wr, bias, E, k, c.fmt, stack.I, blobs,
+                               shared_fmt=c.shared_fmt or 0, shared_blob=sh)
+        spent += time.perf_counter() - t0
+        tok_done += len(toks)
+        if not np.array_equal(ref["ids"], gids[toks]):
+            # near-tie tokens: compare the output with the GPU's own choice
+            ref = oracle.moe_layer(hid[toks], wr, bias, E, k, c.fmt, stack.I, blobs,
+                                   shared_fmt=c.shared_fmt or 0, shared_blob=sh,
+                                   forced_ids=gids[toks])
+        err = rel_l2_rows(out[toks], ref["out_f32"])
+        max_err = max(max_err, float(err.max()))
+        checked += 1
+        if spent >= args.cpu_seconds and l + 1 < L:
+            break
+    parity = {"layers_checked": checked, "layers": L,
+              "tokens_checked_per_layer": int(len(toks)),
+              "routing_tokens_per_layer": T,
+              "rmsnorm_within_1ulp": ulp_ok,
+              "ids_exact": not mismatched and not near,
+              "near_tie_tokens_accepted": [{"layer": a, "token": b} for a, b in near][:32],
+              "mismatched_tokens": [{"layer": a, "token": b} for a, b in mismatched][:32],
+              "near_ties_listed": near_ties[:32],
+              "max_rel_l2": max_err, "bar_rel_l2": OUT_REL_L2,
+              "pass": ulp_ok and not mismatched and max_err <= OUT_REL_L2}
+    if stack.decode:
+        per_layer = spent / checked
+        cpu = {"value": round(T / (per_layer * L), 4), "unit": "tokens/s",
+               "cores": min(threads, T), "kind": "oracle",
+               "sample": f"{checked} of {L} layers of the checked step (every token, T={T}), "
+                         f"scaled to a {L}-layer step ({per_layer:.3f} s per layer)"}
+    else:
+        cpu = {"value": round(tok_done / spent / L, 4), "unit": "tokens/s",
+               "cores": min(threads, int(len(toks))), "kind": "oracle",
+               "sample": f"the layer on {tok_done} sampled tokens of T={T} "
+                         f"({spent:.2f} s), scaled to {L} layer(s)"}
+    return parity, cpu
+
+
+# ---------------------------------------------------------------- one bench line
+def run_line(args, config, T, L, ws_, rank, dev):
+    cfg = mi.CONFIGS[config]
+    stack = DecodeStack(config, T, L, dev)
     prefill = T > stack.sm.DECODE_MAX_T
     H, E, k = stack.H, stack.E, stack.k
-    G = min(args.steps, args.graphs)
-    # distinct seeded inputs per graph, per rank
-    xs = [mi.gen_x(T, H, replica_input_seed(args.config, rank, g), dev, cfg.x_bf16)
+    G = max(1, min(args.steps, args.graphs))
+    xs = [mi.gen_x(T, H, replica_input_seed(config, rank, g), dev, cfg.x_bf16)
           for g in range(G)]
     x_out = [torch.empty(T, H, dtype=torch.float32, device=dev) for _ in range(G)]
     actives = [[torch.empty(E + 1, dtype=torch.int32, device=dev) for _ in range(L)]
@@ -288,7 +436,6 @@ def run_ours(args):
     torch.cuda.synchronize()
     if int(stack.status.item()) != 0:
         raise SystemExit(f"device status {int(stack.status.item())} after warm-up")
-    # the bucket of the last layer accounts for every (token, slot) pair
     if int(stack.offsets[E].item()) != T * k:
         raise SystemExit(f"bucket total {int(stack.offsets[E].item())} != T*k = {T * k}")
 
@@ -297,7 +444,7 @@ def run_ours(args):
             torch.distributed.barrier()
 
     # device-timed region
-    clocks = Clocks(local)
+    clocks = Clocks(dev.index)
     clocks.start()
     barrier()
     torch.cuda.synchronize()
@@ -317,8 +464,7 @@ def run_ours(args):
         durs.append(events[0][l][0].elapsed_time(events[0][l][1]) * 1e-3)
         U = int(actives[0][l][0].item())
         bytes_.append(U * stack.ebytes + T * H * 2 + T * k * H * 4)
-    # prefill: algorithmic flops of the expert GEMMs (routed + shared)
-    flops = 6.0 * H * stack.I * T * k + (6.0 * H * stack.I * T if cfg.shared_fmt else 0.0)
+    flops = 6.0 * H * stack.I * T * k
     # end-to-end: pinned host input -> device, step, result -> pinned host
     hx = [xs[g].cpu().pin_memory() for g in range(G)]
     hout = [torch.empty(T, H, dtype=torch.float32).pin_memory() for _ in range(G)]
@@ -342,48 +488,67 @@ def run_ours(args):
     value = job_tokens_per_s(T, args.steps, ws_, ms)
     e2e = job_tokens_per_s(T, args.steps, ws_, e2e_ms)
     hbm, bf16, src = peaks()
-    bf16_sus = sustained_tflops()
+    bf16_sus, sus_src = sustained_tflops()
     avg_dur = sum(durs) / len(durs)
     avg_bytes = sum(bytes_) / len(bytes_)
     achieved = avg_bytes / avg_dur / 1e9
-    if prefill:
-        achieved_tf = flops / avg_dur / 1e12
+    achieved_tf = flops / avg_dur / 1e12
     traffic = None
     try:
         with open(NCU_TRAFFIC_FILE) as f:
-            tr = json.load(f)
-        traffic = tr.get(f"C{args.config}_T{T}")
+            traffic = json.load(f).get(f"C{config}_T{T}")
     except Exception:
         pass
+    # parity of the graph-replayed step: one more replay of graph 0's step,
+    # captured with per-layer snapshot copies, must give graph 0's output bit
+    # for bit; its layers are then checked against the oracle
+    parity, cpu = None, None
+    if rank == 0 and not args.no_cpu_baseline:
+        rec = Record(L, T, H, k, dev)
+        x_chk = torch.empty(T, H, dtype=torch.float32, device=dev)
+        act_chk = [torch.empty(E + 1, dtype=torch.int32, device=dev) for _ in range(L)]
+        grc = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(grc, stream=s):
+            stack.step(xs[0], x_chk, act_chk, None, rec)
+        xs[0].copy_(hx[0])
+        graphs[0].replay()
+        ref_out = x_out[0].clone()
+        grc.replay()
+        torch.cuda.synchronize()
+        same = bool(torch.equal(x_chk, ref_out))
+        del grc
+        parity, cpu = parity_and_oracle_time(stack, rec, args)
+        parity["graph_output_bitexact"] = same
+        parity["pass"] = parity["pass"] and same
     result = None
     if rank == 0:
-        cpu = None
-        if ws_ == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(stack, xs[0], args)
+        fmt_name = "Q2_32" if cfg.fmt == 1 else "Q4CB_32"
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": ws_,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "data": "synthetic (seeded; random-init weights of the stated shape)",
-            "config": {"workload": f"C{args.config}: {L} stacked MoE layers, H={H}, E={E}, "
-                                   f"I={stack.I}, top-{k}, "
-                                   f"{'Q2_32' if cfg.fmt == 1 else 'Q4CB_32'} experts "
-                                   f"({L * E * stack.ebytes / 1e9:.2f} GB), T={T} tokens per step",
+            "config": {"workload": f"C{config}: {L} stacked MoE layer(s), H={H}, E={E}, "
+                                   f"I={stack.I}, top-{k}, {fmt_name} experts "
+                                   f"({L * E * stack.ebytes / 1e9:.2f} GB), T={T} tokens per step"
+                                   + (", prefill" if prefill else ", decode"),
                        "layers": L, "T": T, "tokens_per_step_per_gpu": T,
                        "parallelism": f"replicas x{ws_}",
-                       "accumulate": "f32", "weights": "2.5 bits/weight" if cfg.fmt == 1 else "4.5 bits/weight",
-                       "l2": "no flush: per-step weight stream (~%.1f GB) >> 126 MB L2"
-                             % (sum(bytes_[:L]) / 1e9) if not prefill else
+                       "accumulate": "f32",
+                       "weights": "2.5 bits/weight" if cfg.fmt == 1 else "4.5 bits/weight",
+                       "l2": ("no flush: per-step weight stream (~%.1f GB) >> 126 MB L2"
+                              % (sum(bytes_[:L]) / 1e9)) if not prefill else
                              "no flush: per-step working set (weights + activations) > 1 GB",
                        "graphs": G},
             "e2e": {"value": round(e2e, 2), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * H * 4, "d2h_bytes_per_step": T * H * 4},
             "gpu_launches": kernels_per_layer(T, k, cfg.shared_fmt is not None) * L * args.steps,
-            "roofline": ({"kernel": "moe_experts decode stage (fused gate/up + down kernel)",
+            "roofline": ({"kernel": "moe_experts decode stage (counter reset + fused gate/up + "
+                                    "down kernel)",
                           "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
                           "unit": "GB/s", "frac": round(achieved / hbm, 4),
-                          "peak_source": f"{src} (MEASURED_PEAKS.json hbm_gbs, burst)"
-                          if src == "measured" else "fallback 6.65 TB/s",
+                          "peak_source": (f"measured (MEASURED_PEAKS.json hbm_gbs, burst)"
+                                          if src == "measured" else "fallback 6.65 TB/s"),
                           "avg_launch_us": round(avg_dur * 1e6, 3),
                           "timed": "external CUDA events around moe_experts of every layer in "
                                    "one of the G replayed step graphs",
@@ -395,8 +560,9 @@ def run_ours(args):
                           "peak": bf16_sus, "unit": "TFLOP/s",
                           "frac": round(achieved_tf / bf16_sus, 4),
                           "frac_of_burst": round(achieved_tf / bf16, 4),
-                          "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained (fp16 "
-                                         "kind::f16 runs at the bf16 rate)",
+                          "peak_source": ("measured (MEASURED_PEAKS.json bf16_tflops_sustained; "
+                                          "fp16 kind::f16 runs at the bf16 rate)"
+                                          if sus_src == "measured" else "fallback 1.4 PFLOP/s"),
                           "avg_launch_us": round(avg_dur * 1e6, 3),
                           "timed": "external CUDA events around moe_experts of every layer in "
                                    "one of the G replayed step graphs",
@@ -404,123 +570,83 @@ def run_ours(args):
                           "traffic": traffic}),
             "clocks": clk,
         }
+        if parity is not None:
+            result["parity"] = parity
         if cpu is not None:
             result["cpu_baseline"] = cpu
-        print(json.dumps(result), flush=True)
     for gr in graphs:
         del gr
     graphs.clear()
-    if ws_ > 1:
-        torch.distributed.destroy_process_group()
+    del stack
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
     return result
 
 
-# ---------------------------------------------------------------- CPU side
-def oracle_sample(config, T, layers, device_stack=None, target_s=15.0, x0=None):
-    """Time the oracle on the workload until about target_s seconds of CPU
-    work: decode (T <= 16) runs whole layers of the stack in order; prefill
-    runs 16-token slices of the first layer.  Returns (tokens/s of the whole
-    workload, description, threads)."""
-    import numpy as np
-
-    import oracle
-    c = mi.CONFIGS[config]
-    x = (x0.cpu() if x0 is not None else mi.gen_x(T, c.H, mi.seed_for(config, 0, "xstep"))).numpy()
-    spent, n = 0.0, 0
-
-    def layer_inputs(l):
-        if device_stack is not None:
-            wr = device_stack.wr[l].cpu().view(torch.int16).numpy().view(np.uint16)
-            bias = None if device_stack.bias[l] is None else device_stack.bias[l].cpu().numpy()
-            blobs = device_stack.experts[l].cpu().numpy()
-            sh = None if device_stack.shared[l] is None else device_stack.shared[l][0].cpu().numpy()
-        else:
-            inp = mi.make_layer(config, 1, layer=l, device="cpu")
-            wr = inp.w_router.view(torch.int16).numpy().view(np.uint16)
-            bias = None if inp.bias is None else inp.bias.numpy()
-            blobs = inp.experts.numpy()
-            sh = None if inp.shared is None else inp.shared[0].numpy()
-        return wr, bias, blobs, sh
-
-    if T <= 16:
-        for l in range(layers):
-            wr, bias, blobs, sh = layer_inputs(l)
-            t0 = time.perf_counter()
-            hid = oracle.rmsnorm(x, c.eps)
-            r = oracle.moe_layer(hid, wr, bias, c.E, c.k, c.fmt, c.I, blobs,
-                                 shared_fmt=c.shared_fmt or 0, shared_blob=sh, residual=x)
-            spent += time.perf_counter() - t0
-            n += 1
-            x = r["residual_out"]
-            if spent >= target_s:
-                break
-        per_layer = spent / n
-        return (T / (per_layer * layers),
-                f"{n} of {layers} layers, T={T}, scaled to a {layers}-layer step "
-                f"({per_layer:.3f} s per layer)", min(oracle.num_threads(), T))
-    wr, bias, blobs, sh = layer_inputs(0)
-    tok = 0
-    while spent < target_s and tok < T:
-        sl = x[tok:tok + 16]
-        t0 = time.perf_counter()
-        hid = oracle.rmsnorm(sl, c.eps)
-        oracle.moe_layer(hid, wr, bias, c.E, c.k, c.fmt, c.I, blobs,
-                         shared_fmt=c.shared_fmt or 0, shared_blob=sh, residual=sl)
-        spent += time.perf_counter() - t0
-        tok += sl.shape[0]
-    return (tok / (spent * layers), f"{tok} of {T} tokens of layer 0 in 16-token slices, "
-            f"scaled to {layers} layer(s)", min(oracle.num_threads(), 16))
+def run_ours(args):
+    ws_, rank, local = dist_env()
+    if ws_ > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    lines = line_specs(args)
+    results = []
+    for i, (config, T) in enumerate(lines):
+        cfg = mi.CONFIGS[config]
+        L = args.layers or cfg.layers
+        r = run_line(args, config, T, L, ws_, rank, dev)
+        if r is not None:
+            if i == len(lines) - 1 and len(results) > 0:
+                r["other_lines"] = [{"workload": o["config"]["workload"], "value": o["value"],
+                                     "unit": o["unit"], "roofline_frac": o["roofline"]["frac"],
+                                     "roofline_unit": o["roofline"]["unit"]} for o in results]
+            print(json.dumps(r), flush=True)
+            results.append(r)
+    if ws_ > 1:
+        torch.distributed.destroy_process_group()
+    return results[-1] if results else None
 
 
-def cpu_baseline(stack, x0, args):
-    tok_s, desc, cores = oracle_sample(args.config, stack.T, stack.L, stack, args.cpu_seconds, x0)
-    return {"value": round(tok_s, 4), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": desc}
+def line_specs(args):
+    if args.config is not None:
+        cfg = mi.CONFIGS[args.config]
+        return [(args.config, args.tokens or cfg.Ts[0])]
+    return parse_lines(args.lines)
 
 
+# ---------------------------------------------------------------- reference arm
 def run_reference(args):
-    """The oracle as the reference arm.  One step times a bounded unit of the
-    workload: one token's router logits + softmax/top-k and ONE of its k
-    expert FFNs (cycling over tokens, experts and two cached layers), plus
-    that token's combine; the step time of the full workload is then
-    L x (router + k x expert + combine) per token."""
-    import numpy as np
-
+    """The oracle as the reference arm, on the headline workload (the last
+    line).  Decode: each step is one whole layer of the stack on all T tokens
+    (cycling over two host-generated layers), the oracle's own routing;
+    the step time of the workload is the mean layer time x L.  Prefill: each
+    step is one 16-token slice of the layer."""
     import oracle
     ws_, rank, _ = dist_env()
     if rank != 0:
         return None
-    cfg = mi.CONFIGS[args.config]
-    T = args.tokens or cfg.Ts[0]
+    config, T = line_specs(args)[-1]
+    cfg = mi.CONFIGS[config]
     L = args.layers or cfg.layers
+    decode = T <= 16
+    Tu = T if decode else 16
     cached = []
     for l in range(min(L, 2)):
-        inp = mi.make_layer(args.config, T, layer=l, device="cpu")
-        hid = oracle.rmsnorm(inp.x.numpy(), cfg.eps)
-        wr = inp.w_router.view(torch.int16).numpy().view(np.uint16)
-        bias = None if inp.bias is None else inp.bias.numpy()
-        cached.append((hid, wr, bias, inp.experts.numpy(),
+        inp = mi.make_layer(config, Tu, layer=l, device="cpu")
+        cached.append((inp.x.numpy(), u16(inp.w_router),
+                       None if inp.bias is None else inp.bias.numpy(), inp.experts.numpy(),
                        None if inp.shared is None else inp.shared[0].numpy()))
-    t_router, t_expert, t_comb = [], [], []
+    times = []
 
     def unit(i, record):
-        hid, wr, bias, blobs, sh = cached[i % len(cached)]
-        t = (i // len(cached)) % T
-        j = (i // (len(cached) * T)) % cfg.k
+        x, wr, bias, blobs, sh = cached[i % len(cached)]
         a = time.perf_counter()
-        lg = oracle.router_logits(hid[t:t + 1], wr, bias)
-        ids, w = oracle.topk(lg, cfg.k)
-        b = time.perf_counter()
-        y = oracle.expert_ffn(cfg.fmt, blobs[ids[0, j]], cfg.H, cfg.I, hid[t])
-        if sh is not None and j == 0:
-            y = y + oracle.expert_ffn(cfg.shared_fmt, sh, cfg.H, cfg.I, hid[t])
-        c = time.perf_counter()
-        oracle.combine(np.repeat(y[None, :], cfg.k, 0), w)
-        d = time.perf_counter()
+        hid = oracle.rmsnorm(x, cfg.eps)
+        oracle.moe_layer(hid, wr, bias, cfg.E, cfg.k, cfg.fmt, cfg.I, blobs,
+                         shared_fmt=cfg.shared_fmt or 0, shared_blob=sh, residual=x)
         if record:
-            t_router.append(b - a)
-            t_expert.append(c - b)
-            t_comb.append(d - c)
+            times.append(time.perf_counter() - a)
 
     for i in range(args.warmup):
         unit(i, False)
@@ -528,24 +654,26 @@ def run_reference(args):
     for i in range(args.steps):
         unit(i, True)
     wall = time.perf_counter() - wall0
-    per_tok_layer = (statistics.mean(t_router) + cfg.k * statistics.mean(t_expert)
-                     + statistics.mean(t_comb))
-    step_s = per_tok_layer * L * T
+    per_unit = statistics.mean(times)
+    step_s = per_unit * L * (T / Tu)
     value = T / step_s
+    cores = min(oracle.num_threads(), Tu)
     res = {"metric": METRIC, "value": round(value, 4), "unit": "tokens/s", "n_gpus": ws_,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
            "data": "synthetic (seeded; random-init weights of the stated shape)",
-           "config": {"workload": f"C{args.config}: {L} stacked MoE layers, H={cfg.H}, E={cfg.E}, "
+           "config": {"workload": f"C{config}: {L} stacked MoE layer(s), H={cfg.H}, E={cfg.E}, "
                                   f"I={cfg.I}, top-{cfg.k}, T={T} tokens per step",
                       "layers": L, "T": T},
            "impl": "reference",
-           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1,
+           "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": cores,
                             "kind": "oracle",
-                            "sample": f"{args.steps} units of one token's router+top-k and one "
-                                      f"of its {cfg.k} expert FFNs (+combine), cycling over "
-                                      f"{len(cached)} cached layers; scaled to {L} layers x "
-                                      f"{cfg.k} experts x {T} tokens ({wall:.1f} s wall)"},
+                            "sample": (f"{args.steps} steps of one whole layer (T={T}, the "
+                                       f"oracle's own routing), cycling over {len(cached)} "
+                                       f"layers; scaled to {L} layers ({wall:.1f} s wall)")
+                            if decode else
+                            (f"{args.steps} steps of one 16-token slice of the layer, scaled "
+                             f"to T={T} x {L} layer(s) ({wall:.1f} s wall)")},
            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(res), flush=True)
@@ -555,15 +683,19 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--config", type=int, default=1)
+    ap.add_argument("--lines", default=DEFAULT_LINES,
+                    help="config:T list, run in order; the last line is the headline")
+    ap.add_argument("--config", type=int, default=None, help="run this one config only")
     ap.add_argument("--tokens", type=int, default=0)
     ap.add_argument("--layers", type=int, default=0)
     ap.add_argument("--graphs", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-sample", type=int, default=64)
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle parity check and CPU baseline")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

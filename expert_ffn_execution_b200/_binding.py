@@ -121,8 +121,8 @@ def _qw(w):
 
 
 # ---------------------------------------------------------------- helpers
-def strata_selftest_wait(budget_cycles, complete, dev_status, dev_out, stream=None, check=True):
-    rc = load().strata_selftest_wait(int(budget_cycles), 1 if complete else 0, _ptr(dev_status),
+def strata_selftest_wait(budget_cycles, mode, dev_status, dev_out, stream=None, check=True):
+    rc = load().strata_selftest_wait(int(budget_cycles), int(mode), _ptr(dev_status),
                                      _ptr(dev_out), _stream(stream))
     return _check("strata_selftest_wait", rc) if check else rc
 

@@ -1,9 +1,9 @@
 // abi.cu -- extern "C" entry points of libstrata_moe.so: argument checks,
 // workspace carving and kernel launches.  See include/strata_moe.h.
 #include <algorithm>
-#include <mutex>
 
 #include "decode.cuh"
+#include "scratch_cache.h"
 
 using namespace strata;
 
@@ -84,12 +84,13 @@ int32_t run_experts(const uint16_t* hidden, const strata_qweights* w, const int3
     a.y = reinterpret_cast<float*>(y);
     a.status = status;
     a.num_sms = num_sms_of_current_device();
-    (void)ws_bytes;
+    // both callers have checked ws_bytes against experts_ws(); check again
+    // here so that no path launches on a short workspace
+    if (ws_bytes < experts_ws(w, T, k, shared)) return STRATA_EINVAL;
     const int Umax = shared ? 1 : std::min(E, P);
-    if (decode_tc_supported(T, w->hidden, w->inter, Umax, w->fmt, a.num_sms))
-      return from_cuda(launch_experts_decode_tc(a, st));
-    if (decode_smem_bytes(T, w->hidden) > 200u * 1024u) return STRATA_EUNSUPPORTED;
-    return from_cuda(launch_experts_decode(a, st));
+    if (!decode_tc_supported(T, w->hidden, w->inter, Umax, w->fmt, a.num_sms))
+      return STRATA_EUNSUPPORTED;
+    return from_cuda(launch_experts_decode_tc(a, st));
   }
   PrefillArgs a;
   a.hidden = hidden;
@@ -153,12 +154,13 @@ int32_t strata_read_status(const int32_t* dev_status, void* stream) {
   return STRATA_OK;
 }
 
-int32_t strata_selftest_wait(uint64_t budget_cycles, int32_t complete, int32_t* dev_status,
+int32_t strata_selftest_wait(uint64_t budget_cycles, int32_t mode, int32_t* dev_status,
                              int32_t* dev_out, void* stream) {
-  if (budget_cycles > 4000000000ull || !dev_status || !dev_out || !aligned(dev_out, 4))
+  if (budget_cycles > 4000000000ull || mode < 0 || mode > 2 || !dev_status || !dev_out ||
+      !aligned(dev_out, 4))
     return STRATA_EINVAL;
-  return from_cuda(launch_wait_selftest((long long)budget_cycles, complete ? 1 : 0, dev_status,
-                                        dev_out, reinterpret_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_wait_selftest((long long)budget_cycles, mode, dev_status, dev_out,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int32_t moe_rmsnorm(const float* x, int32_t T, int32_t H, float eps, uint16_t* hidden,
@@ -453,22 +455,37 @@ constexpr uint64_t kStaticScratchBytes = kStaticHBytes + 4096;  // + T*k <= 512 
 static __device__ __align__(256) uint8_t g_experts_static_scratch[kStaticScratchBytes];
 
 namespace {
-std::mutex g_static_scratch_mu;
-void* g_static_scratch_ptr[kMaxDevices] = {};
+ScratchAddressCache<kMaxDevices> g_static_scratch_addr;
 
-// Device address of the array on the current device, looked up once per
-// device (with that device current) and cached; nullptr if the lookup fails.
+// Handle of the calling thread's current context, through the driver entry
+// point (the library does not link libcuda); nullptr if unavailable.
+void* current_context() {
+  typedef int (*CtxGetCurrentFn)(void**);
+  static CtxGetCurrentFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  void* ctx = nullptr;
+  if (!fn || fn(&ctx) != 0) return nullptr;
+  return ctx;
+}
+
+// Device address of the array in the current device's current context:
+// looked up (cudaGetSymbolAddress, with that device current) on the first
+// call in a context and cached per device and context; nullptr if the
+// lookup fails.
 void* static_scratch_on_current_device() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-  if (!g_static_scratch_ptr[dev]) {
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  return g_static_scratch_addr.get(dev, current_context, [] {
     void* ptr = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress((void**)&ptr, g_experts_static_scratch);
-    if (e != cudaSuccess || !ptr) return nullptr;
-    g_static_scratch_ptr[dev] = ptr;
-  }
-  return g_static_scratch_ptr[dev];
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_experts_static_scratch);
+    return e == cudaSuccess ? ptr : nullptr;
+  });
 }
 }  // namespace
 

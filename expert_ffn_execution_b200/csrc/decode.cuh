@@ -22,8 +22,6 @@ struct DecodeArgs {
   int32_t* sync;   // scratch: one counter per active expert (Umax ints), or nullptr
   int num_sms;
 };
-cudaError_t launch_experts_decode(const DecodeArgs& a, cudaStream_t st);
-size_t decode_smem_bytes(int T, int H);
 // Umax: most active experts of a call (1 for the shared expert, else min(E, T*k)).
 bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid);
 cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st);
@@ -65,7 +63,7 @@ bool route_decode_supported(int T, int H, int E, int k);
 uint64_t route_decode_workspace_bytes(int T, int H, int E);
 cudaError_t launch_route_decode(const RouteArgs& a, cudaStream_t st);
 
-cudaError_t launch_wait_selftest(long long budget, int complete, int32_t* status, int32_t* out,
+cudaError_t launch_wait_selftest(long long budget, int mode, int32_t* status, int32_t* out,
                                  cudaStream_t st);
 cudaError_t launch_rmsnorm(const float* x, int T, int H, float eps, uint16_t* out, cudaStream_t st);
 uint64_t router_workspace_bytes(int T, int H, int E, int k);

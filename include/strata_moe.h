@@ -125,19 +125,26 @@ STRATA_API uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t int
 STRATA_API int32_t strata_read_status(const int32_t* dev_status, void* stream);
 
 /* Failure-detection self-test of the bounded device waits (the pages have
- * no counterpart: it checks this library's own error path).  One CTA waits
- * on an mbarrier with the same bounded waits every kernel uses, first the
- * pipeline's (abort-flag guarded) wait, then the epilogue's backoff wait.
- * complete != 0: the barrier's phase is completed first, both waits succeed,
- * dev_out = {1, 1} and dev_status is untouched.  complete == 0: nothing ever
- * arrives; the first wait gives up after budget_cycles SM cycles (kernels
- * use about 4e9, 2 s), ORs STRATA_DEV_TIMEOUT into *dev_status and raises
- * the CTA's abort flag, the second wait then returns at once, dev_out =
- * {0, 0}; strata_read_status reports STRATA_ETIMEOUT and the context stays
- * usable.  Nothing faults, traps or hangs.
+ * no counterpart: it checks this library's own error path).  One CTA runs
+ * two of the bounded waits every kernel uses and writes their results
+ * (1 = the wait succeeded, 0 = it gave up) to dev_out[0], dev_out[1]:
+ *   mode 1: an mbarrier's phase is completed first; the pipeline's
+ *           (abort-flag guarded) wait and the epilogue's wait both succeed,
+ *           dev_out = {1, 1}, dev_status untouched.
+ *   mode 0: nothing arrives on the mbarrier; the first wait gives up after
+ *           budget_cycles SM cycles (kernels use about 4e9, 2 s), ORs
+ *           STRATA_DEV_TIMEOUT into *dev_status and raises the CTA's abort
+ *           flag; the second returns at once; dev_out = {0, 0}.
+ *   mode 2: the first wait is the cross-CTA counter wait of the fused decode
+ *           kernel, on dev_out[0] (zeroed by the kernel, raised by nobody);
+ *           it gives up the same way, the second returns at once;
+ *           dev_out = {0, 0}.
+ * After a timeout strata_read_status reports STRATA_ETIMEOUT and the context
+ * stays usable.  Nothing faults, traps or hangs.
  *   dev_status int32 device word; dev_out int32[2] device.
- *   budget_cycles <= 4e9, else STRATA_EINVAL.  Asynchronous on `stream`. */
-STRATA_API int32_t strata_selftest_wait(uint64_t budget_cycles, int32_t complete,
+ *   budget_cycles <= 4e9 and mode in 0..2, else STRATA_EINVAL.
+ *   Asynchronous on `stream`. */
+STRATA_API int32_t strata_selftest_wait(uint64_t budget_cycles, int32_t mode,
                              int32_t* dev_status, int32_t* dev_out, void* stream);
 
 /* ---------------------------------------------------------------- calls */
@@ -186,10 +193,12 @@ STRATA_API int32_t moe_bucket(const int32_t* topk_ids, int32_t T, int32_t k, int
 
 /* The routing step in one call: moe_rmsnorm(x) -> moe_router_topk ->
  * moe_bucket, with the same outputs as those three calls (bit for bit).
- * For T <= STRATA_DECODE_MAX_T (and E <= 512) it runs as ONE kernel: a
- * 16-CTA thread-block cluster that streams W_r through shared memory,
- * reduces the partial logits over distributed shared memory and sorts the
- * pairs in the leader CTA.
+ * For T <= STRATA_DECODE_MAX_T (E a multiple of 16, up to 1024) it runs as
+ * two kernels over the whole GPU: route_logits (one CTA per 16 experts and
+ * slice of H: RMSNorm of the rows, then partial logits from its slice of
+ * W_r) and route_select (one CTA: the partial logits summed in a fixed
+ * order, + bias, top-k per token, the stable bucket), chained by
+ * programmatic dependent launch; other sizes run the three calls.
  *   x      fp32 [T,H];  hidden bf16 [T,H] out (the normalised tokens)
  *   the other arguments as in moe_router_topk and moe_bucket. */
 STRATA_API uint64_t moe_route_workspace_size(int32_t T, int32_t H, int32_t E, int32_t k);
@@ -214,7 +223,15 @@ STRATA_API int32_t moe_route(const float* x, int32_t T, int32_t H, float eps,
  *      T > STRATA_DECODE_MAX_T: fp16 (prefill
  *      path, tcgen05 grouped GEMM over dequantised fp16 tiles).
  *   offsets/perm/active: as written by moe_bucket for the same (T, k, E).
- * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket. */
+ * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket;
+ * decode: H a multiple of 256, else STRATA_EUNSUPPORTED.
+ * Concurrency (decode path): the fused kernel runs one CTA per SM and its
+ * down tiles wait for gate/up tiles of other CTAs, so all its CTAs must be
+ * resident together.  Do not run decode moe_experts calls concurrently with
+ * other kernels on the device (other streams, other host threads, MPS
+ * clients with a share of the SMs): a CTA that cannot become resident
+ * leaves the waits of the others to run out, and the call ends with
+ * STRATA_DEV_TIMEOUT (after about 2 s) and undefined y. */
 STRATA_API uint64_t moe_experts_workspace_size(const strata_qweights* w, int32_t T, int32_t k);
 STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
                     const int32_t* offsets, const int32_t* perm,
@@ -234,9 +251,10 @@ STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
  *   Limit: T <= STRATA_DECODE_MAX_T and T*k*I <= 1,048,576 (2 MiB of fp16);
  *   beyond it the call returns STRATA_EUNSUPPORTED and launches nothing.
  *   Set-up: the first call on each device, with that device current, looks
- *   up the array's device address (cudaGetSymbolAddress) and caches it; make
- *   that first call before any stream capture.  A failed lookup returns
- *   STRATA_ECUDA.
+ *   up the array's device address (cudaGetSymbolAddress) and caches it for
+ *   that device and its current CUDA context (a new context, e.g. after
+ *   cudaDeviceReset, looks it up again); make that first call before any
+ *   stream capture.  A failed lookup returns STRATA_ECUDA.
  *   Sharing: all calls on a device use the same array, which keeps the last
  *   call's contents; no part of it has to start at zero (each call zeroes its
  *   counters before use and reads only the h rows it wrote).  Calls that

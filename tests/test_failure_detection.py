@@ -18,11 +18,42 @@ from expert_ffn_execution_b200._binding import EINVAL, ETIMEOUT, OK
 
 def test_selftest_argument_checks():
     # rejected on the host before any launch: budget above the kernels' own,
-    # or missing buffers
+    # an unknown mode, or missing buffers
     assert sm.strata_selftest_wait(5_000_000_000, 0, 1 << 20, 1 << 20, stream=0,
                                    check=False) == EINVAL
+    assert sm.strata_selftest_wait(1000, 3, 1 << 20, 1 << 20, stream=0, check=False) == EINVAL
+    assert sm.strata_selftest_wait(1000, -1, 1 << 20, 1 << 20, stream=0, check=False) == EINVAL
     assert sm.strata_selftest_wait(1000, 0, None, 1 << 20, stream=0, check=False) == EINVAL
     assert sm.strata_selftest_wait(1000, 0, 1 << 20, None, stream=0, check=False) == EINVAL
+
+
+def _usable_after_timeout(torch):
+    """An ordinary call with a fresh status word runs cleanly: the routing of
+    one token through moe_route, whose kernels take dev_status."""
+    import moe_inputs as mi
+    c = mi.CONFIGS[0]
+    T, E, k, H = 1, 16, 4, c.H
+    inp = mi.make_layer(0, T, layer=0, device="cuda", E=E)
+    dev = "cuda"
+    status2 = torch.zeros(1, dtype=torch.int32, device=dev)
+    hid = torch.empty(T, H, dtype=torch.bfloat16, device=dev)
+    ids = torch.full((T, k), -1, dtype=torch.int32, device=dev)
+    w = torch.empty(T, k, dtype=torch.float32, device=dev)
+    counts = torch.empty(E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(T * k, dtype=torch.int32, device=dev)
+    inv = torch.empty(T * k, dtype=torch.int32, device=dev)
+    active = torch.empty(E + 1, dtype=torch.int32, device=dev)
+    n = max(sm.moe_route_workspace_size(T, H, E, k), 256)
+    wsb = torch.empty(n, dtype=torch.uint8, device=dev)
+    sm.moe_route(inp.x, T, H, c.eps, inp.w_router, inp.bias, E, k, hid, ids, w, counts, offsets,
+                 perm, inv, active, wsb, n, status2)
+    torch.cuda.synchronize()
+    assert sm.strata_read_status(status2) == OK
+    assert torch.isfinite(hid.float()).all()
+    got = ids[0].tolist()
+    assert len(set(got)) == k and all(0 <= e < E for e in got)
+    assert int(offsets[E]) == T * k
 
 
 @pytest.mark.gpu
@@ -46,13 +77,24 @@ def test_bounded_wait_times_out_and_context_stays_usable():
     assert out.tolist() == [0, 0]
     assert sm.strata_read_status(status) == ETIMEOUT
     assert elapsed < 1.0, elapsed
-    # the context is usable: a fresh status word and an ordinary layer call
-    import moe_inputs as mi
-    c = mi.CONFIGS[0]
-    inp = mi.make_layer(0, 1, layer=0, device="cuda", E=16)
-    hid = torch.empty(1, c.H, dtype=torch.bfloat16, device="cuda")
-    status2 = torch.zeros(1, dtype=torch.int32, device="cuda")
-    sm.moe_rmsnorm(inp.x, 1, c.H, c.eps, hid)
+    _usable_after_timeout(torch)
+
+
+@pytest.mark.gpu
+def test_counter_wait_times_out_and_context_stays_usable():
+    """The cross-CTA counter wait (the fused decode kernel's wait for another
+    CTA's h rows) on a counter nobody raises: it gives up within its budget,
+    reports STRATA_DEV_TIMEOUT, and the next call runs cleanly."""
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    t0 = time.perf_counter()
+    sm.strata_selftest_wait(2_000_000, 2, status, out)
     torch.cuda.synchronize()
-    assert torch.isfinite(hid.float()).all()
-    assert sm.strata_read_status(status2) == OK
+    elapsed = time.perf_counter() - t0
+    assert out.tolist() == [0, 0]
+    assert sm.strata_read_status(status) == ETIMEOUT
+    assert elapsed < 1.0, elapsed
+    _usable_after_timeout(torch)

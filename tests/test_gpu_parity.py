@@ -21,7 +21,8 @@ if not torch.cuda.is_available():
 import expert_ffn_execution_b200 as sm  # noqa: E402
 import moe_inputs as mi  # noqa: E402
 import oracle  # noqa: E402
-from tests.harness import OUT_REL_L2, TOPK_W_ATOL, check_routing, rel_l2_rows  # noqa: E402
+from tests.harness import (OUT_REL_L2, TOPK_W_ATOL, check_routing, parallel_rows,  # noqa: E402
+                           rel_l2_rows, stratified_tokens)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -99,9 +100,10 @@ class Run:
 
 
 def check_layer(r: Run, sample=None):
-    """Full check of one run; `sample` = token indices for the router,
-    expert and output checks (all tokens if None).  Bucket and RMSNorm are
-    always checked on every token."""
+    """Full check of one run.  RMSNorm, router logits, top-k ids and weights
+    and the bucket are checked on every token; `sample` = token indices for
+    the combine, expert-output and layer-output checks (all tokens if None).
+    Returns the per-token relative L2 of the layer output on the sample."""
     T, H, E, k = r.T, r.H, r.E, r.k
     hid = u16(r.hidden)
     # RMSNorm within one bf16 ulp
@@ -110,21 +112,22 @@ def check_layer(r: Run, sample=None):
     b = oracle.bf16_bits_to_f32(ref_h).astype(np.float64)
     ulp = 2.0 ** (np.floor(np.log2(np.maximum(np.abs(b), 1e-30))) - 7)
     assert np.all(np.abs(a - b) <= ulp), "rmsnorm beyond one bf16 ulp"
-    # router on the GPU's hidden
+    # router on the GPU's hidden, every token (the oracle in token chunks on
+    # the host's cores)
     wr = u16(r.inp.w_router)
     bias = None if r.inp.bias is None else r.inp.bias.cpu().numpy()
-    toks = np.arange(T) if sample is None else np.asarray(sample)
-    ref_lg = oracle.router_logits(hid[toks], wr, bias)
-    gl = r.logits.cpu().numpy()[toks]
-    assert np.all(np.abs(gl - ref_lg) <= 1e-4 + 1e-4 * np.abs(ref_lg))
+    ref_lg = np.concatenate(parallel_rows(
+        lambda lo, hi: oracle.router_logits(hid[lo:hi], wr, bias), T, 256))
+    gl = r.logits.cpu().numpy()
+    assert np.all(np.abs(gl - ref_lg) <= 1e-4 + 1e-4 * np.abs(ref_lg)), "router logits"
     gids = r.ids.cpu().numpy()
-    ok, near, bad = check_routing(ref_lg, gids[toks], k)
+    ok, near, bad = check_routing(ref_lg, gids, k)
     assert ok, f"routing mismatch on tokens {bad[:10]}"
     if near:
-        print(f"near-tie tokens: {list(toks[near])}")
+        print(f"near-tie tokens: {near}")
     ref_ids_gpu_logits, ref_w = oracle.topk(gl, k)
-    np.testing.assert_array_equal(ref_ids_gpu_logits, gids[toks])
-    assert np.abs(r.w.cpu().numpy()[toks] - ref_w).max() <= TOPK_W_ATOL
+    np.testing.assert_array_equal(ref_ids_gpu_logits, gids)
+    assert np.abs(r.w.cpu().numpy() - ref_w).max() <= TOPK_W_ATOL
     # bucket bit-exact on the GPU's ids (all tokens)
     counts, offsets, perm, inv = oracle.bucket(gids, E)
     np.testing.assert_array_equal(r.counts.cpu().numpy(), counts)
@@ -135,6 +138,7 @@ def check_layer(r: Run, sample=None):
     nz = np.nonzero(counts)[0]
     assert act[0] == len(nz)
     np.testing.assert_array_equal(act[1:1 + len(nz)], nz)
+    toks = np.arange(T) if sample is None else np.asarray(sample)
     # combine bit-exact given the GPU's y (sampled tokens)
     rows = inv.reshape(T, k)[toks]
     yg = r.y[torch.as_tensor(rows.reshape(-1), device=DEV).long()].float().cpu().numpy()
@@ -144,16 +148,27 @@ def check_layer(r: Run, sample=None):
     np.testing.assert_array_equal(r.acc.cpu().numpy()[toks], of)
     # expert outputs and the layer output vs the oracle (teacher-forced ids)
     blobs = r.blobs_for(gids[toks])
-    for i, t in enumerate(toks):
-        for j in range(k):
+    pairs = [(i, int(t), j) for i, t in enumerate(toks) for j in range(k)]
+
+    def expert_errs(lo, hi):
+        out = []
+        for i, t, j in pairs[lo:hi]:
             e = int(gids[t, j])
             ref_y = oracle.expert_ffn(r.c.fmt, blobs[e], H, r.I, hid[t])
-            assert rel_l2_rows(yg[i * k + j], ref_y) <= OUT_REL_L2, (int(t), j, e)
+            out.append((rel_l2_rows(yg[i * k + j], ref_y), t, j, e))
+        return out
+    for errs in parallel_rows(expert_errs, len(pairs), 16):
+        for err, t, j, e in errs:
+            assert err <= OUT_REL_L2, (t, j, e, float(err))
     sb = None if r.inp.shared is None else r.inp.shared[0].cpu().numpy()
     if sb is not None:
-        for i, t in enumerate(toks):
-            ref_s = oracle.expert_ffn(r.c.shared_fmt, sb, H, r.I, hid[t])
-            assert rel_l2_rows(sh[i], ref_s) <= OUT_REL_L2, ("shared", int(t))
+        def shared_errs(lo, hi):
+            return [(rel_l2_rows(sh[i], oracle.expert_ffn(r.c.shared_fmt, sb, H, r.I,
+                                                          hid[toks[i]])), int(toks[i]))
+                    for i in range(lo, hi)]
+        for errs in parallel_rows(shared_errs, len(toks), 8):
+            for err, t in errs:
+                assert err <= OUT_REL_L2, ("shared", t, float(err))
     ref = oracle.moe_layer(hid[toks], wr, bias, E, k, r.c.fmt, r.I, blobs,
                            shared_fmt=r.c.shared_fmt or 0, shared_blob=sb,
                            forced_ids=gids[toks])
@@ -164,8 +179,11 @@ def check_layer(r: Run, sample=None):
 
 
 @pytest.mark.parametrize("config,T", [(0, 1), (1, 4), (3, 1), (3, 4), (4, 1), (4, 4), (4, 8),
-                                      (4, 16)])
+                                      (4, 16), (5, 1), (5, 4)])
 def test_decode_layer_parity(config, T):
+    """Configs 0, 1, 3 and 4 at their decode token counts, and config 5
+    ("C3b": the all-4-bit-codebook reading of config 3 at E = 512), each
+    checked on every token with the parity bars."""
     r = Run(config, T).run()
     err = check_layer(r)
     print(f"C{config} T={T}: max rel L2 {err.max():.2e}")
@@ -307,10 +325,14 @@ def test_prefill_one_expert_takes_everything():
 @pytest.mark.parametrize("config", [2, 3, 4])
 def test_prefill_full_size(config):
     """The T = 8192 prefill chunks (2-bit routed; + 4-bit shared expert; 4-bit
-    large experts) at full size, checked on 24 sampled tokens."""
+    large experts) at full size: RMSNorm, router logits, top-k ids and weights
+    and the bucket on all 8192 tokens; combine, expert outputs and layer
+    output on a stratified sample of 256 tokens (the least-loaded expert's
+    tokens, the most-loaded expert's full tiles and last partial tile, the
+    tail token of other experts, then uniform random tokens)."""
     r = Run(config, 8192).run()
-    rng = np.random.default_rng(config)
-    sample = np.sort(rng.choice(8192, 24, replace=False))
+    sample = stratified_tokens(r.counts.cpu().numpy(), r.offsets.cpu().numpy(),
+                               r.perm.cpu().numpy(), r.k, r.T, n=256, seed=config)
     err = check_layer(r, sample=sample)
     print(f"C{config} T=8192: max rel L2 {err.max():.2e} over {len(sample)} tokens")
 
