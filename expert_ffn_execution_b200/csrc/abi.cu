@@ -48,10 +48,23 @@ bool decode_supported(const strata_qweights* w) {
   return w->hidden % 256 == 0 && w->inter % 128 == 0 && w->hidden % 64 == 0;
 }
 
+// Decode scratch: h fp16 [P, I], its Z fp32 [P, I/32], then one progress
+// counter per active expert (at most P).
+struct DecodeScratch {
+  uint64_t h, z, sync, total;
+};
+DecodeScratch decode_scratch(int P, int I) {
+  DecodeScratch d;
+  d.h = 0;
+  d.z = up256((uint64_t)P * I * 2);
+  d.sync = d.z + up256((uint64_t)P * (I / 32) * 4);
+  d.total = d.sync + up256((uint64_t)P * 4);
+  return d;
+}
+
 uint64_t experts_ws(const strata_qweights* w, int T, int k, int shared) {
   const int P = shared ? T : T * k;
-  // decode: h fp16 [P, I], then one progress counter per active expert
-  if (T <= kDecodeMaxTokens) return up256((uint64_t)P * w->inter * 2) + up256((uint64_t)P * 4);
+  if (T <= kDecodeMaxTokens) return decode_scratch(P, w->inter).total;
   return prefill_workspace_bytes(T, w->hidden, w->inter, shared ? 1 : w->num_experts, shared ? 1 : k,
                                  shared);
 }
@@ -77,10 +90,12 @@ int32_t run_experts(const uint16_t* hidden, const strata_qweights* w, const int3
     a.perm = perm;
     a.active = active;
     a.shared_mode = shared;
-    a.hbuf = reinterpret_cast<uint16_t*>(ws);
     const int P = shared ? T : T * k;
-    a.sync = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) +
-                                        up256((uint64_t)P * w->inter * 2));
+    const DecodeScratch ds = decode_scratch(P, w->inter);
+    uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+    a.hbuf = reinterpret_cast<uint16_t*>(wsb + ds.h);
+    a.zdn = reinterpret_cast<float*>(wsb + ds.z);
+    a.sync = reinterpret_cast<int32_t*>(wsb + ds.sync);
     a.y = reinterpret_cast<float*>(y);
     a.status = status;
     a.num_sms = num_sms_of_current_device();
@@ -439,17 +454,19 @@ int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router, c
 // all free HBM up front (weights plus a cache pool), where a cudaMalloc in the
 // middle of a step would fail and a cudaFree would synchronise the device.
 // The call allocates nothing: no cudaMalloc, cudaFree or allocating library
-// routine.  Its scratch is the fp16 SwiGLU activation h [T*k, I] and the
-// per-expert progress counters of the fused decode kernel.
+// routine.  Its scratch is the fp16 SwiGLU activation h [T*k, I], the
+// offset sums Z of the h rows [T*k, I/32] and the per-expert progress
+// counters of the fused decode kernel.
 //
 // Every call on a device shares the one array, which keeps the last call's
 // contents.  Nothing in it must start at zero: the down tiles read only the
-// h rows that the gate/up tiles of the same call wrote, and each call zeroes
+// h and Z rows that the gate/up tiles of the same call wrote, and each call zeroes
 // its counters before the kernel that uses them.  Calls whose kernels overlap
 // on the GPU (other streams, other host threads) race on the array.
 namespace {
-constexpr uint64_t kStaticHBytes = 2ull << 20;  // T*k*I <= 1,048,576 fp16
-constexpr uint64_t kStaticScratchBytes = kStaticHBytes + 4096;  // + T*k <= 512 counters
+constexpr uint64_t kStaticMaxPI = 1ull << 20;  // T*k*I <= 1,048,576
+// h fp16 (2 MiB) + its Z (128 KiB) + T*k <= 512 counters, each part padded
+constexpr uint64_t kStaticScratchBytes = kStaticMaxPI * 2 + kStaticMaxPI / 8 + 256 + 4096;
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_experts_static_scratch[kStaticScratchBytes];
@@ -496,7 +513,7 @@ extern "C" int32_t moe_experts_static_scratch(const uint16_t* hidden, const stra
   if (!valid_weights(w) || T < 0 || k < 1 || k > w->num_experts || k > 32) return STRATA_EINVAL;
   if (w->num_experts > 1024) return STRATA_EINVAL;
   // sizes beyond the array (or beyond the decode path) are rejected up front
-  if (T > kDecodeMaxTokens || (uint64_t)T * k * w->inter * 2 > kStaticHBytes)
+  if (T > kDecodeMaxTokens || (uint64_t)T * k * w->inter > kStaticMaxPI)
     return STRATA_EUNSUPPORTED;
   if (T == 0) return STRATA_OK;
   if (!hidden || !offsets || !perm || !active || !y) return STRATA_EINVAL;

@@ -2,57 +2,69 @@
 // (T <= STRATA_DECODE_MAX_T) on the 5th-generation tensor cores.
 //
 // With at most 16 tokens per call the expert FFN is bound by streaming the
-// quantised weights out of HBM and decoding them, not by multiply-adds.  So
-// every weight row is decoded by exactly one thread, straight into that row's
-// lane of tensor memory (tcgen05.st), and the MMA reads its A operand
-// (128 weight rows x 16 K, fp16) from tensor memory; B is the token block
-// (N = 16 columns, fp16, in shared memory).  Decoded weights never pass
-// through shared memory, whose bandwidth would otherwise cap the path.  Codes
-// and scales arrive by TMA into a ring of shared-memory stages.
+// quantised weights out of HBM and turning them into tensor-core operands,
+// not by multiply-adds, so the work per weight is kept to a few integer
+// instructions:
+//   - Every weight row is decoded by one thread straight into that row's lane
+//     of tensor memory (tcgen05.st); the MMA reads its A operand (128 rows x
+//     16 K, fp16) from there and B (the tokens, N = 16) from shared memory.
+//   - The decode does not apply the block scale.  A 2-bit code c becomes the
+//     fp16 value M + c (one lop3 puts c into the mantissa of a power of two
+//     M), a 4-bit code the fp16 value 1024 + (KV[c] + 128) (byte lookups).
+//     Each 32-element block is multiplied into its own accumulator in tensor
+//     memory, D_b = sum_k A_k x_k, and the epilogue applies the block's scale
+//     and removes the offset:  y += d_b * (D_b - Z_b),  where
+//     Z_b = sum_k (M_k + 1.5) x_k (2-bit) or 1152 * sum_k x_k (4-bit) depends
+//     on the tokens only and is computed once per call (gate/up: from the
+//     tokens; down: by the gate/up epilogue, next to each h row).  The
+//     offsets are exact in fp16 and the scale is applied in fp32, so the
+//     result is the exact block dot product up to fp32 rounding.
 //
 // Two kinds of tile:
-//   gate/up  64 rows of I: lanes 0-63 decode the gate rows, lanes 64-127 the
-//            same up rows.  B = every token of the call, so a tile computes
-//            all T columns and the epilogue keeps the tokens routed to the
-//            tile's expert: h = SwiGLU(gate, up) -> fp16 [P, I] in sorted pair
-//            order, K permuted within 16-groups the way the down tiles'
-//            decode orders K.
-//   down     128 rows of H of one expert.  B = that expert's h rows (TMA from
-//            h); y fp32 [P, H] in sorted order.
+//   gate/up  64 rows of I: lanes 0-63 the gate rows, lanes 64-127 the same up
+//            rows.  B = every token of the call; the epilogue keeps the
+//            columns of the tokens routed to the tile's expert, exchanges gate
+//            and up through shared memory, and writes h = SwiGLU fp16 [P, I]
+//            in sorted pair order (K permuted within 16-groups the way the
+//            down tiles' decode orders K) and the down tiles' Z per h row.
+//   down     128 rows of H of one expert.  B = that expert's h rows (TMA);
+//            y fp32 [P, H] in sorted order.
 // and three kernel forms (MODE):
 //   2  fused: one launch runs both kinds.  Each CTA takes its gate/up tiles
 //      round robin, then a share of the down tiles chosen so that every CTA
-//      has about the same weighted work (a gate/up tile costs H, a down tile
-//      I plus a fixed overhead, in 64-column units).  Down tiles are dealt in
-//      rounds counted back from each CTA's last tile, from the end of the
-//      expert order: the experts whose gate/up tiles finish last become the
-//      last tile of many CTAs rather than all tiles of a few, and the extra
-//      down tiles of CTAs with fewer gate/up tiles come from the experts that
-//      are ready first.  A down
-//      tile's h block is loaded once its expert's gate/up tiles are all done:
-//      each gate/up epilogue publishes its h rows and then counts itself in a
-//      per-expert counter (release); the producer polls it (acquire, bounded)
-//      before the TMA.  The counters are zeroed by a one-thread-block kernel
+//      has about the same weighted work (deal.h).  A down tile's h block is
+//      loaded once its expert's gate/up tiles are all done: each gate/up
+//      epilogue publishes its h rows and then counts itself in a per-expert
+//      counter (release); the producer polls it (acquire, bounded) before
+//      the TMA.  The counters are zeroed by a one-thread-block kernel
 //      launched just before, so the workspace needs no initial contents.
 //   0, 1  gate/up alone, then down alone (chained by programmatic dependent
 //      launch): used when the fused form's shared memory leaves too few
 //      stages.
 // Every CTA of a fused grid is resident at once (one per SM, grid <= SMs),
 // and a CTA's gate/up tiles depend on nothing outside it, so the waits on the
-// counters always end; they are bounded all the same.
+// counters end while the kernel has the GPU to itself; they are bounded all
+// the same.
 //
 // One persistent CTA per SM with a static tile list.  Warps:
-//   0-3   epilogue: tcgen05.ld of their TMEM lane quarter (and the tile table)
-//   4..   decoders: kTcGroups groups of four warps taking K chunks in turn;
-//         a thread owns one tile row (= TMEM lane), reads its codes from
-//         the swizzled stage (conflict-free), decodes to fp16 and stores them
-//         into the A stage in tensor memory
-//   then  the TMA producer warp (codes, scales; down: the tile's scales and
-//         h blocks) and the warp that allocates tensor memory and issues
-//         the MMAs (one thread)
-// Barriers: full/empty (smem stages), tfull/tempty (TMEM A stages),
-// afull/aempty (two accumulators), sfull/sempty and bfull/bempty (down:
-// per-tile scales, per-expert h block).  Every wait is bounded.
+//   0-3   epilogue: per 128-K half chunk, tcgen05.ld of the block
+//         accumulators of the routed columns, then y += d_b (D_b - Z_b) in
+//         registers; at the end of a tile, the SwiGLU / h / y stores.  They
+//         also build the tile table.
+//   4-11  decoders: two groups of four warps taking 256-K chunks in turn; a
+//         thread owns one tile row (= TMEM lane), reads its codes from the
+//         swizzled stage (conflict-free) and stores the decoded halves into
+//         its group's two tensor-memory stages
+//   12    the TMA producer (codes, scales; down: the tile's scales, the h
+//         block and its Z rows)
+//   13    tensor-memory allocation and the MMA issue (one thread)
+// Tensor memory: four stages of 128 columns, two per decoder group (one per
+// half chunk): A in columns 0-63 (128 K of fp16), then four 16-column block
+// accumulators.
+// Barriers: full/empty (smem stages), tfull/afree (A written / A read by the
+// MMAs), accfull/accfree (accumulators written / read), sfull/sempty and
+// bfull/bempty (down: per-tile scales, per-expert h block).  Every wait is
+// bounded.
 #include <algorithm>
 
 #include "deal.h"
@@ -62,23 +74,23 @@
 
 namespace strata {
 
-constexpr int kTcGroups = 3;                      // decoder groups (4 warps each)
-constexpr int kTcProdWarp = 4 + 4 * kTcGroups;     // TMA producer warp
-constexpr int kTcMmaWarp = kTcProdWarp + 1;        // TMEM allocation + MMA warp
+constexpr int kTcGroups = 2;                          // decoder groups (4 warps each)
+constexpr int kTcDecWarp0 = 4;
+constexpr int kTcProdWarp = kTcDecWarp0 + 4 * kTcGroups;  // TMA producer warp
+constexpr int kTcMmaWarp = kTcProdWarp + 1;               // TMEM allocation + MMA warp
 constexpr int kTcWarps = kTcMmaWarp + 1;
 constexpr int kTcThreads = kTcWarps * 32;
-constexpr int kTcKC = 256;        // K per chunk (one smem stage / one TMEM A stage)
-constexpr int kTcTS = 3;          // TMEM A stages
-constexpr int kTcACol0 = 64;      // A stage t at columns 64 + 128 t (accumulators at 0, 32)
+constexpr int kTcKC = 256;      // K per chunk (one shared-memory stage)
+constexpr int kTcKH = 128;      // K per half chunk (one tensor-memory stage)
+constexpr int kTcTS = 2 * kTcGroups;  // tensor-memory stages: two per group
+constexpr int kTcStageCols = 128;     // A: 64 columns, then 4 block accumulators of 16
+constexpr int kTcAccCol = 64;
 constexpr int kTcTmemCols = 512;
 constexpr int kTcMaxStages = 16;
 constexpr int kTcSmemBudget = 227 * 1024;
-constexpr int kTcFusedMinStages = 9;  // fewer: run the two-kernel form
+constexpr int kTcFusedMinStages = 8;  // fewer: run the two-kernel form
 constexpr int kTcMaxGrid = 1024;      // the fused tile dealing keeps one int per CTA
-// Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
-// only after the MMAs of its previous one retired, so with at least as many
-// stages as groups no waiter runs two phases ahead of a stage's barrier.
-static_assert(kTcTS >= kTcGroups, "TMEM A stages must cover the decoder groups");
+static_assert(kTcTS * kTcStageCols <= kTcTmemCols, "tensor memory stages fit");
 
 struct TcParams {
   const uint16_t* hidden;
@@ -90,11 +102,11 @@ struct TcParams {
   const int32_t* active;
   int shared_mode;
   uint16_t* hbuf;  // gate/up output, down input: fp16 [P, I]
+  float* zdn;      // gate/up output, down input: Z of each h row and 32-block, fp32 [P, I/32]
   float* y;        // down output: fp32 [P, H]
   int32_t* status;
   int32_t* sync;   // fused form: finished gate/up tiles per active expert (zeroed)
   int S;           // shared-memory stages (a multiple of kTcGroups)
-  int NB;          // B rows: 8 (T <= 8; rows 8-15 of the MMA repeat them) or 16
   int maxT;        // capacity of the tile table: tiles per CTA at most
 };
 
@@ -109,16 +121,18 @@ __host__ __device__ constexpr int tc_cbr() {  // code bytes per row per chunk
 }
 
 struct TcLayout {
-  uint32_t codes_bytes, stage_bytes, b, b_bytes, hb, hb_bytes, sbuf, s_bytes, xch, tbl, bars,
-      total;
+  uint32_t codes_bytes, stage_bytes, b, b_bytes, zg, zg_bytes, hb, hb_bytes, zd, zd_bytes, sbuf,
+      s_bytes, xch, tbl, bars, total;
 };
 
 __host__ __device__ inline uint32_t up1k(uint32_t x) { return (x + 1023u) & ~1023u; }
+__host__ __device__ inline uint32_t up128(uint32_t x) { return (x + 127u) & ~127u; }
 
 // Shared memory, from a 1024-byte aligned base: S stages | gate/up: the token
-// block | down: two h blocks | down: two per-tile scale blocks | gate/up: the
-// SwiGLU exchange buffer (also the fused form's dealing scratch) | the tile
-// table | barriers.  Every TMA destination is 1024-byte aligned.
+// block and its Z | down: two h blocks, their Z rows and two per-tile scale
+// blocks | gate/up: the SwiGLU exchange buffer (also the fused form's dealing
+// scratch) | the tile table | barriers.  Every TMA destination is 1024-byte
+// aligned, every bulk-copy destination 128-byte aligned.
 __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, int I, int S,
                                               int maxT) {
   TcLayout L;
@@ -130,49 +144,69 @@ __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, 
   L.b = off;
   L.b_bytes = gu ? (uint32_t)NB * (uint32_t)H * 2u : 0u;
   off += L.b_bytes;
+  L.zg = off;
+  L.zg_bytes = gu ? up128((uint32_t)(H / 32) * (uint32_t)NB * 4u) : 0u;
+  off = up1k(off + L.zg_bytes);
   L.hb = off;
   L.hb_bytes = dn ? (uint32_t)NB * (uint32_t)I * 2u : 0u;
   off += 2u * L.hb_bytes;
+  L.zd = off;
+  L.zd_bytes = dn ? up128((uint32_t)NB * (uint32_t)(I / 32) * 4u) : 0u;
+  off += 2u * L.zd_bytes;
   L.sbuf = off;
-  L.s_bytes = dn ? up1k(8u * (uint32_t)I) : 0u;
+  L.s_bytes = dn ? up128(8u * (uint32_t)I) : 0u;
   off += 2u * L.s_bytes;
   L.xch = off;
-  off += gu ? up1k(2u * 64u * 17u * 4u) : 0u;
+  off += gu ? up128(std::max(64u * 17u * 4u, 4u * (uint32_t)kTcMaxGrid)) : 0u;
   L.tbl = off;
-  off += up1k((uint32_t)sizeof(TcTile) * (uint32_t)maxT);
+  off += up128((uint32_t)sizeof(TcTile) * (uint32_t)maxT);
   L.bars = off;
   off += 1024u;
   L.total = off;
   return L;
 }
-static_assert(2 * 64 * 17 * 4 >= 4 * kTcMaxGrid, "dealing scratch fits the exchange buffer");
 
 // ---------------------------------------------------------------- decode
-// One Q2 word (16 codes, element j at bits 2j) -> R[i] = fp16x2 (element i,
-// element i + 8) * d.  A code placed at mantissa bit p of an fp16 whose
-// exponent gives that bit unit weight is M_p + c exactly (M_p = 2^(10-p));
-// subtracting M_p + 1.5 leaves c - 1.5 exactly; the multiply by the block
-// scale rounds once.
-STRATA_DEVFN void dq_q2_word(uint32_t w, uint32_t d2, uint32_t* R) {
+// Offsets of the unscaled 2-bit decode.  In a 16-element group element e and
+// element e + 8 share one fp16x2 register R[e % 8]; the code sits at mantissa
+// bit p of an fp16 whose exponent gives that bit unit weight, so the value is
+// M + c exactly with M = 2^(10-p): M = 256, 256, 64, 16, 4, 256, 64, 16 for
+// e % 8 = 0..7.  The weight is d (c - 1.5) = d (value - (M + 1.5)).
+__host__ __device__ inline float q2_offset(int e) {
+  const int m = e & 7;
+  const float M = (m == 0 || m == 1 || m == 5) ? 256.f : (m == 2 || m == 6) ? 64.f
+                  : (m == 3 || m == 7) ? 16.f : 4.f;
+  return M + 1.5f;
+}
+// The unscaled 4-bit decode gives 1024 + (KV[c] + 128) = KV[c] + 1152.
+constexpr float kQ4Offset = 1152.f;
+
+// One Q2 word (16 codes, element j at bits 2j) -> R[i] = fp16x2 (M_i + c_i,
+// M_i + c_{i+8}): one lop3 per register.
+STRATA_DEVFN void dq_q2_word_raw(uint32_t w, uint32_t* R) {
   const uint32_t wl = w << 2, wr = w >> 8;
   const uint32_t src[8] = {wl, w, w, w, w, wr, wr, wr};
   const uint32_t msk[8] = {0x000C000Cu, 0x000C000Cu, 0x00300030u, 0x00C000C0u,
                            0x03000300u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
   const uint32_t mag[8] = {0x5C005C00u, 0x5C005C00u, 0x54005400u, 0x4C004C00u,
                            0x44004400u, 0x5C005C00u, 0x54005400u, 0x4C004C00u};
-  const uint32_t sub[8] = {0x5C065C06u, 0x5C065C06u, 0x54185418u, 0x4C604C60u,
-                           0x45804580u, 0x5C065C06u, 0x54185418u, 0x4C604C60u};
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    uint32_t v, t;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(src[i]), "r"(msk[i]), "r"(mag[i]));
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(v), "r"(sub[i]));
-    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(R[i]) : "r"(t), "r"(d2));
-  }
+  for (int i = 0; i < 8; ++i)
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(R[i]) : "r"(src[i]), "r"(msk[i]), "r"(mag[i]));
 }
 
-STRATA_DEVFN uint32_t dup_lo(uint32_t x) { return __byte_perm(x, 0, 0x1010); }
-STRATA_DEVFN uint32_t dup_hi(uint32_t x) { return __byte_perm(x, 0, 0x3232); }
+// Two Q4CB words (elements 0..7, 8..15 of a 16-group) -> R[i] = fp16x2
+// (element 2i, element 2i+1), each KV[c] + 1152 exactly: byte lookups give
+// u = KV[c] + 128, placed under the fp16 exponent byte 0x64 (1024 + u).
+STRATA_DEVFN void dq_q4_group_raw(uint32_t w0, uint32_t w1, const Q4Table& T, uint32_t* R) {
+  const uint32_t u[4] = {q4_lookup4(w0, T), q4_lookup4(w0 >> 16, T), q4_lookup4(w1, T),
+                         q4_lookup4(w1 >> 16, T)};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    R[2 * i] = __byte_perm(u[i], 0x64646464u, 0x4140u);
+    R[2 * i + 1] = __byte_perm(u[i], 0x64646464u, 0x4342u);
+  }
+}
 
 STRATA_DEVFN uint4 lds128(const void* p) {
   uint4 v;
@@ -187,56 +221,74 @@ STRATA_DEVFN uint2 lds64(const void* p) {
   return v;
 }
 
-// Gate/up B operand: token rows n < T of hidden (bf16 -> fp16, exact in the
-// normal range), rows T..NB-1 zero, K permuted within each 16-group like the
-// decoded codes, in the 128-byte-swizzled K-major layout (atoms of 64 K x NB
-// rows, 128 bytes per row, 16-byte piece c of row n at c ^ (n & 7)).  Thread
-// `tid` of `nthr` fills items tid, tid + nthr, ...; each batch issues all of
-// its loads before any conversion, so the fill costs a few L2 round trips.
+STRATA_DEVFN float half_lo(uint32_t x) { return __half2float(__ushort_as_half((uint16_t)x)); }
+STRATA_DEVFN float half_hi(uint32_t x) {
+  return __half2float(__ushort_as_half((uint16_t)(x >> 16)));
+}
+
+// Gate/up B operand and its Z.  B: token rows n < T of hidden (bf16 -> fp16,
+// exact in the normal range), rows T..NB-1 zero, K permuted within each
+// 16-group like the decoded codes, in the 128-byte-swizzled K-major layout
+// (atoms of 64 K x NB rows, 128 bytes per row, 16-byte piece c of row n at
+// c ^ (n & 7)).  Z: zg[b * NB + n] = sum over the 32-block b of offset(k) *
+// fp16(x_k), in k order.  Thread `tid` of `nthr` fills the (row, block) items
+// tid, tid + nthr, ...; each batch issues all of its loads before any
+// conversion, so the fill costs a few L2 round trips.
 template <int FMT>
-STRATA_DEVFN void fill_tokens(uint8_t* bsm, const uint16_t* __restrict__ hidden, int T, int H,
-                              int NB, int tid, int nthr) {
-  constexpr int kBatch = 4;
-  const int ng = H / 16, total = NB * ng;
+STRATA_DEVFN void fill_tokens(uint8_t* bsm, float* zg, const uint16_t* __restrict__ hidden,
+                              int T, int H, int NB, int tid, int nthr) {
+  constexpr int kBatch = 2;
+  const int nb = H / 32, total = NB * nb;
   for (int i0 = tid; i0 < total; i0 += kBatch * nthr) {
-    uint4 a[kBatch], b[kBatch];
+    uint4 a[kBatch][4];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int idx = i0 + u * nthr;
-      const int n = idx / ng, g = idx - n * ng;
-      a[u] = b[u] = make_uint4(0, 0, 0, 0);
-      if (idx < total && n < T) {
-        a[u] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 16 * g);
-        b[u] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 16 * g + 8);
+      const int n = idx / nb, b = idx - n * nb;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        a[u][v] = make_uint4(0, 0, 0, 0);
+        if (idx < total && n < T)
+          a[u][v] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 32 * b + 8 * v);
       }
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int idx = i0 + u * nthr;
       if (idx >= total) break;
-      const int n = idx / ng, g = idx - n * ng;
-      const uint32_t w[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
-      uint16_t e[16];
+      const int n = idx / nb, b = idx - n * nb;
+      float z = 0.f;
 #pragma unroll
-      for (int kk = 0; kk < 16; ++kk) {
-        const uint16_t bf = (uint16_t)((kk & 1) ? (w[kk >> 1] >> 16) : (w[kk >> 1] & 0xffffu));
-        e[group_slot<FMT>(kk)] = bf16_to_f16_bits(bf);
+      for (int gg = 0; gg < 2; ++gg) {  // the block's two 16-groups
+        const uint32_t w[8] = {a[u][2 * gg].x, a[u][2 * gg].y, a[u][2 * gg].z, a[u][2 * gg].w,
+                               a[u][2 * gg + 1].x, a[u][2 * gg + 1].y, a[u][2 * gg + 1].z,
+                               a[u][2 * gg + 1].w};
+        uint16_t e[16];
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk) {
+          const uint16_t bf = (uint16_t)((kk & 1) ? (w[kk >> 1] >> 16) : (w[kk >> 1] & 0xffffu));
+          const uint16_t h = bf16_to_f16_bits(bf);
+          e[group_slot<FMT>(kk)] = h;
+          const float off = FMT == STRATA_FMT_Q2_32 ? q2_offset(kk) : kQ4Offset;
+          z = fmaf(off, __half2float(__ushort_as_half(h)), z);
+        }
+        uint32_t o[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) o[j] = (uint32_t)e[2 * j] | ((uint32_t)e[2 * j + 1] << 16);
+        const int g = 2 * b + gg;  // 16-group index along K
+        const int pc = (g & 3) * 2;
+        uint8_t* row = bsm + (size_t)(g >> 2) * (NB * 128) + n * 128;
+        *reinterpret_cast<uint4*>(row + ((pc ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4*>(row + (((pc + 1) ^ (n & 7)) << 4)) =
+            make_uint4(o[4], o[5], o[6], o[7]);
       }
-      uint32_t o[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) o[j] = (uint32_t)e[2 * j] | ((uint32_t)e[2 * j + 1] << 16);
-      const int pc = (g & 3) * 2;
-      uint8_t* row = bsm + (size_t)(g >> 2) * (NB * 128) + n * 128;
-      *reinterpret_cast<uint4*>(row + ((pc ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4*>(row + (((pc + 1) ^ (n & 7)) << 4)) =
-          make_uint4(o[4], o[5], o[6], o[7]);
+      zg[b * NB + n] = z;
     }
   }
 }
 
-
 // ---------------------------------------------------------------- kernel
-template <int MODE, int FMT>
+template <int MODE, int FMT, int NB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
                  const __grid_constant__ CUtensorMap mu,   // up codes
@@ -249,18 +301,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   constexpr int CBR = tc_cbr<FMT>();
   constexpr int PIECE_K = (FMT == STRATA_FMT_Q2_32) ? 64 : 32;  // K per 16-byte code piece
   constexpr int NPC = CBR / 16;                                  // pieces per full chunk
+  constexpr int NPH = NPC / 2;                                   // pieces per half chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const TcLayout L = tc_layout(MODE, FMT, p.NB, p.H, p.I, p.S, p.maxT);
+  const TcLayout L = tc_layout(MODE, FMT, NB, p.H, p.I, p.S, p.maxT);
   const int S = p.S;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + kTcMaxStages;
   uint64_t* tfull = empty + kTcMaxStages;
-  uint64_t* tempty = tfull + kTcTS;
-  uint64_t* afull = tempty + kTcTS;
-  uint64_t* aempty = afull + 2;
-  uint64_t* sfull = aempty + 2;
+  uint64_t* afree = tfull + kTcTS;
+  uint64_t* accfull = afree + kTcTS;
+  uint64_t* accfree = accfull + kTcTS;
+  uint64_t* sfull = accfree + kTcTS;
   uint64_t* sempty = sfull + 2;
   uint64_t* bfull = sempty + 2;
   uint64_t* bempty = bfull + 2;
@@ -269,31 +322,33 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   TcTile* tbl = reinterpret_cast<TcTile*>(smem + L.tbl);
+  float* zg = reinterpret_cast<float*>(smem + L.zg);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.H, I = p.I, T = p.T;
   const int nchA = H / kTcKC;                // H % 256 == 0
-  const int nchB = (I + kTcKC - 1) / kTcKC;  // I % 128 == 0: the last chunk may be 128 wide
+  const int nchB = (I + kTcKC - 1) / kTcKC;  // I % 128 == 0: the last chunk may be one half
   const int tpeA = I / 64, tpeB = H / 128;   // tiles per expert
   const Planes PL = plane_offsets(FMT, H, I);
   const int G = gridDim.x, cta = blockIdx.x;
+  const int nbI = I / 32;                    // 32-blocks along the down tiles' K
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 128);
+      mbar_init(&empty[s], 256);  // the owning decoder group + the epilogue
     }
     for (int t = 0; t < kTcTS; ++t) {
       mbar_init(&tfull[t], 128);
-      mbar_init(&tempty[t], 1);
+      mbar_init(&afree[t], 1);
+      mbar_init(&accfull[t], 1);
+      mbar_init(&accfree[t], 128);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&afull[a], 1);
-      mbar_init(&aempty[a], 128);
       mbar_init(&sfull[a], 1);
-      mbar_init(&sempty[a], 128 * kTcGroups);
+      mbar_init(&sempty[a], 128);
       mbar_init(&bfull[a], 1);
-      mbar_init(&bempty[a], 1);
+      mbar_init(&bempty[a], 1 + 128);  // the MMAs' commit + the epilogue's Z reads
     }
     mbar_init(tbl_ready, 128);
     mbar_init(done, 1);
@@ -373,6 +428,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     u = j / tpeB;
     rb = j - u * tpeB;
   };
+  auto is_a = [&](int i) { return kGU && (MODE == 0 || i < nA); };
 
   if (warp == kTcProdWarp) {
     // ------------------------------------------------ TMA producer
@@ -385,19 +441,21 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         ++gc;
         return s;
       };
-      // the expert's h rows [s0, s0 + NB) into the next B buffer
-      auto load_h = [&](int e) {
+      // the expert's h rows [s0, s0 + NB) and its n rows of Z into the next
+      // B buffer
+      auto load_h = [&](int s0, int n) {
         ++bseq;
         const int b = bseq & 1;
-        const int s0 = p.shared_mode ? 0 : p.offsets[e];
         mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
-        const uint32_t ab = (uint32_t)p.NB * 128u;
-        mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
+        const uint32_t ab = (uint32_t)NB * 128u;
+        const uint32_t zb = (uint32_t)n * (uint32_t)nbI * 4u;
+        mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64) + zb);
         for (int a = 0; a < I / 64; ++a)
           tma_load_2d(smem + L.hb + b * L.hb_bytes + a * ab, &mh, 64 * a, s0, &bfull[b]);
+        bulk_g2s(smem + L.zd + b * L.zd_bytes, p.zdn + (size_t)s0 * nbI, zb, &bfull[b]);
       };
       for (int i = 0; i < tcount; ++i) {
-        if (kGU && (MODE == 0 || i < nA)) {
+        if (is_a(i)) {
           int u, rb;
           tile_a(i, u, rb);
           const int e = expert_of(u);
@@ -413,15 +471,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         }
         if constexpr (kDN) {
           const int ib = i - nA;  // down-tile sequence number
-          int u, rb;
-          if constexpr (MODE == 1) {
-            tile_b1(i, u, rb);
-          } else {
-            if (ib == 0) mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
-            u = tbl[i].u;
-            rb = tbl[i].rb;
-          }
-          const int e = expert_of(u);
+          if (ib == 0) mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
+          const int u = tbl[i].u, rb = tbl[i].rb, e = tbl[i].e;
           // the tile's scales: rows rb*128.. of the down plane, all of K
           const int sb = ib & 1;
           mbar_wait_guarded(&sempty[sb], ((ib >> 1) & 1) ^ 1, p.status, abort_flag);
@@ -440,8 +491,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
             const int pre = (ib == 0) ? min(nchB, S) : 0;
             for (int c = 0; c < pre; ++c) issue_b(c);
             if (new_h) {
-              if (bseq < 0) pdl_wait_prior();  // h is written by the preceding grid
-              load_h(e);
+              if (bseq < 0) pdl_wait_prior();  // h and Z are written by the preceding grid
+              load_h(tbl[i].s0, tbl[i].n);
             }
             for (int c = pre; c < nchB; ++c) issue_b(c);
           } else {
@@ -451,21 +502,31 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
               // has counted itself; then read it through the async proxy
               gmem_wait_geq(p.sync + u, tpeA, p.status, abort_flag);
               fence_proxy_async_global();
-              load_h(e);
+              load_h(tbl[i].s0, tbl[i].n);
             }
           }
           prev_e = e;
         }
       }
+      // Before the CTA can exit, every copy it issued has landed (normally
+      // the consumers have seen them all; after a timed-out wait this waits,
+      // bounded, for the copies still in flight).
+      constexpr long long kDrain = 20000000;  // about 10 ms per copy
+      for (int x = max(0, gc - S); x < gc; ++x)
+        mbar_wait_bounded(&full[x % S], (x / S) & 1, p.status, kDrain);
+      for (int x = max(0, nB - 2); x < nB; ++x)
+        mbar_wait_bounded(&sfull[x & 1], (x >> 1) & 1, p.status, kDrain);
+      for (int x = max(0, bseq - 1); x <= bseq; ++x)
+        mbar_wait_bounded(&bfull[x & 1], (x >> 1) & 1, p.status, kDrain);
     }
     __syncwarp();
   } else {
-    // ---- everyone else: the gate/up B operand, then (epilogue warps) the
-    // tile table
+    // ---- everyone else: the gate/up B operand and Z, then (epilogue warps)
+    // the tile table
     if constexpr (kGU) {
       // the producer warp is not among the fillers: renumber the warps after it
       const int ftid = warp < kTcProdWarp ? (int)threadIdx.x : (int)threadIdx.x - 32;
-      fill_tokens<FMT>(smem + L.b, p.hidden, T, H, p.NB, ftid, (kTcWarps - 1) * 32);
+      fill_tokens<FMT>(smem + L.b, zg, p.hidden, T, H, NB, ftid, (kTcWarps - 1) * 32);
       fence_proxy_async_smem();
       named_bar_sync(2, (kTcWarps - 1) * 32);
     }
@@ -480,7 +541,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
       for (int i = r; i < tcount; i += 128) {
         TcTile& t = tbl[i];
         int u, rb;
-        if (kGU && (MODE == 0 || i < nA)) {
+        if (is_a(i)) {
           tile_a(i, u, rb);
         } else if (MODE == 1) {
           tile_b1(i, u, rb);
@@ -503,10 +564,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
             dev_flag(p.status, STRATA_DEV_BOUNDS);
             t.n = 0;
           }
+          if (t.s0 < 0 || t.s0 + t.n > Pn) {
+            dev_flag(p.status, STRATA_DEV_BOUNDS);
+            t.s0 = 0;
+            t.n = 0;
+          }
         }
-        if (t.n < 0 || t.n > p.NB) {
+        if (t.n < 0 || t.n > NB) {
           dev_flag(p.status, STRATA_DEV_BOUNDS);
-          t.n = t.n < 0 ? 0 : p.NB;
+          t.n = t.n < 0 ? 0 : NB;
         }
       }
       named_bar_sync(1, 128);
@@ -532,35 +598,139 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     // ------------------------------------------------ epilogue
     mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
     const int r = threadIdx.x;  // tile row = TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     float* xch = reinterpret_cast<float*>(smem + L.xch);
+    int gc = 0, bseq = -1, prev_e = -1;
+    uint32_t par = 0;  // bit st: parity of the next use of tensor-memory stage st
     for (int i = 0; i < tcount; ++i) {
       const TcTile& ti = tbl[i];
-      const int a = i & 1;
-      mbar_wait_backoff(&afull[a], (i >> 1) & 1, p.status, abort_flag);
-      tc_fence_after();
-      uint32_t v[16];
-      tmem_ld16(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)(a * 32), v);
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&aempty[a]);
-      if (kGU && (MODE == 0 || i < nA)) {
-        float* xr = xch + r * 17;  // rows 0-63 gate, 64-127 up
+      const bool isA = is_a(i);
+      const int ib = i - nA;
+      const int n = ti.n;
+      const int nch = isA ? nchA : nchB;
+      const int K = isA ? H : I;
+      int col[NB];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) xr[j] = __uint_as_float(v[j]);
-        named_bar_sync(1, 128);
-        for (int idx = r; idx < ti.n * 64; idx += 128) {
-          const int j = idx >> 6, l = idx & 63;
-          const int t = ti.tok[j];
-          const float gv = xch[l * 17 + t], uv = xch[(64 + l) * 17 + t];
-          const float h = silu_f32(gv) * uv;
-          const int ii = ti.rb * 64 + l;
-          const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
-          p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(__float2half_rn(h));
+      for (int j = 0; j < NB; ++j) col[j] = isA ? ((j < n) ? ti.tok[j] : 0) : j;
+      const float* zsrc = zg;
+      if (!isA) {
+        mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
+        if (ib == 0 || ti.e != prev_e) ++bseq;
+        prev_e = ti.e;
+        // Z rows of this expert's h (they arrive with the h block)
+        mbar_wait_guarded(&bfull[bseq & 1], (bseq >> 1) & 1, p.status, abort_flag);
+        zsrc = reinterpret_cast<const float*>(smem + L.zd + (bseq & 1) * L.zd_bytes);
+      }
+      const uint8_t* srow =
+          isA ? nullptr : smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
+      float acc[NB];
+#pragma unroll
+      for (int j = 0; j < NB; ++j) acc[j] = 0.f;
+      for (int c = 0; c < nch; ++c, ++gc) {
+        const int g = gc % kTcGroups;
+        const int s = gc % S;
+        // this row's 8 block scales of the chunk (gate/up: in the stage)
+        uint4 scv;
+        if (isA) {
+          mbar_wait_guarded(&full[s], (gc / S) & 1, p.status, abort_flag);
+          scv = lds128(smem + s * L.stage_bytes + L.codes_bytes + r * 16);
+        } else {
+          const int nb4 = min(8, (K - c * kTcKC) / 32);
+          const uint2 lo = lds64(srow + c * 16);
+          scv = make_uint4(lo.x, lo.y, 0u, 0u);
+          if (nb4 > 4) {
+            const uint2 hi = lds64(srow + c * 16 + 8);
+            scv.z = hi.x;
+            scv.w = hi.y;
+          }
         }
-        if constexpr (MODE == 2) {
-          // publish this thread's h stores (to the TMA reads of other CTAs)
-          fence_proxy_async_global();
-          __threadfence();
+        const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
+        const int nh = (K - c * kTcKC) >= kTcKC ? 2 : 1;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h >= nh) break;
+          const int st = 2 * g + h;
+          mbar_wait_backoff(&accfull[st], (par >> st) & 1u, p.status, abort_flag);
+          par ^= 1u << st;
+          tc_fence_after();
+          const uint32_t acc_t = tmem_base + lane_off + (uint32_t)(st * kTcStageCols + kTcAccCol);
+          // the four block accumulators, QB blocks per pass (registers)
+          constexpr int QB = NB == 16 ? 2 : 4;
+#pragma unroll
+          for (int q0 = 0; q0 < 4; q0 += QB) {
+            uint32_t D[QB][NB];
+#pragma unroll
+            for (int q = 0; q < QB; ++q)
+#pragma unroll
+              for (int j = 0; j < NB; ++j)
+                if (j < n) D[q][j] = tmem_ld1(acc_t + (uint32_t)(16 * (q0 + q) + col[j]));
+            tmem_wait_ld();
+#pragma unroll
+            for (int q = 0; q < QB; ++q)
+#pragma unroll
+              for (int j = 0; j < NB; ++j)
+                if (j < n) reg_after_wait(D[q][j]);
+            if (q0 + QB == 4) {
+              tc_fence_before();
+              mbar_arrive(&accfree[st]);
+            }
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+              const int qq = 4 * h + q0 + q;  // block within the chunk
+              const float d = (qq & 1) ? half_hi(scw[qq >> 1]) : half_lo(scw[qq >> 1]);
+              const int b = c * 8 + qq;  // block along K
+#pragma unroll
+              for (int j = 0; j < NB; ++j) {
+                if (j < n) {
+                  const float z = isA ? zsrc[b * NB + col[j]] : zsrc[j * nbI + b];
+                  acc[j] = fmaf(d, __uint_as_float(D[q][j]) - z, acc[j]);
+                }
+              }
+            }
+          }
+        }
+        // the stage's (gate/up: scale) reads are done: order them before the
+        // producer's next TMA write, then release
+        fence_proxy_async_smem();
+        mbar_arrive(&empty[s]);
+      }
+      if (!isA) {
+        fence_proxy_async_smem();
+        mbar_arrive(&sempty[ib & 1]);
+        // the last tile on this h block: its Z rows are read
+        if (i + 1 == tcount || tbl[i + 1].e != ti.e) mbar_arrive(&bempty[bseq & 1]);
+      }
+      if (isA) {
+        // SwiGLU: rows 0-63 gate, 64-127 the same up rows
+        if (r >= 64) {
+#pragma unroll
+          for (int j = 0; j < NB; ++j)
+            if (j < n) xch[(r - 64) * 17 + j] = acc[j];
+        }
+        named_bar_sync(1, 128);
+        if (r < 64) {
+          const int ii = ti.rb * 64 + r;  // row of I
+          const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
+          const float off = FMT == STRATA_FMT_Q2_32 ? q2_offset(ii & 15) : kQ4Offset;
+#pragma unroll
+          for (int j = 0; j < NB; ++j) {
+            if (j < n) {
+              const float hv = silu_f32(acc[j]) * xch[r * 17 + j];
+              const __half h16 = __float2half_rn(hv);
+              p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(h16);
+              // this h row's Z over the 32-block of rows (one warp), in lane order
+              float zc = off * __half2float(h16);
+#pragma unroll
+              for (int o = 1; o < 32; o <<= 1) zc += __shfl_xor_sync(0xffffffffu, zc, o);
+              if (lane == 0) p.zdn[(size_t)(ti.s0 + j) * nbI + (ii >> 5)] = zc;
+            }
+          }
+          if constexpr (MODE == 2) {
+            // publish this thread's h and Z stores (to the TMA reads of
+            // other CTAs)
+            fence_proxy_async_global();
+            __threadfence();
+          }
         }
         named_bar_sync(1, 128);
         if constexpr (MODE == 2) {
@@ -569,29 +739,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
       } else if constexpr (kDN) {
         const int row = ti.rb * 128 + r;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j < ti.n) p.y[(size_t)(ti.s0 + j) * H + row] = __uint_as_float(v[j]);
+        for (int j = 0; j < NB; ++j)
+          if (j < n) p.y[(size_t)(ti.s0 + j) * H + row] = acc[j];
       }
     }
   } else if (warp < kTcProdWarp) {
     // ------------------------------------------------ decoders
-    const int g = (warp - 4) >> 2;
+    const int g = (warp - kTcDecWarp0) >> 2;
     const int qd = warp & 3;
     const int r = 32 * qd + lane;  // tile row = TMEM lane
     const uint32_t swz = ((uint32_t)(r * CBR) >> 7) & (uint32_t)(NPC - 1);
-    const uint32_t tl = tmem_base + ((uint32_t)(32 * qd) << 16) + kTcACol0;
+    const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
     const Q4Table T4 = q4_table();
     int gc = 0;
+    uint32_t par = 0;  // bit h: parity of the next use of this group's stage 2g + h
     for (int i = 0; i < tcount; ++i) {
-      const bool isA = kGU && (MODE == 0 || i < nA);
-      const int ib = i - nA;
+      const bool isA = is_a(i);
       const int K = isA ? H : I;
       const int nch = isA ? nchA : nchB;
-      const uint8_t* srow = nullptr;
-      if (!isA) {
-        mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
-        srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
-      }
       for (int c = 0; c < nch; ++c, ++gc) {
         if (gc % kTcGroups != g) continue;
         const int s = gc % S;
@@ -603,72 +768,44 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
 #pragma unroll
         for (int pc = 0; pc < NPC; ++pc)
           cw[pc] = (pc < np) ? lds128(st + r * CBR + ((pc ^ swz) << 4)) : make_uint4(0, 0, 0, 0);
-        uint32_t sc[4];
-        if (isA) {
-          const uint4 v = lds128(st + L.codes_bytes + r * 16);
-          sc[0] = v.x;
-          sc[1] = v.y;
-          sc[2] = v.z;
-          sc[3] = v.w;
-        } else {
-          const uint2 lo = lds64(srow + c * 16);
-          sc[0] = lo.x;
-          sc[1] = lo.y;
-          sc[2] = 0;
-          sc[3] = 0;
-          if (kv > 128) {
-            const uint2 hi = lds64(srow + c * 16 + 8);
-            sc[2] = hi.x;
-            sc[3] = hi.y;
-          }
-        }
         // The stage is released before its loads are consumed: order those
         // generic-proxy reads before the producer's next TMA (async-proxy)
         // write into the stage, which the barrier alone does not.
         fence_proxy_async_smem();
         mbar_arrive(&empty[s]);
-        const int t = gc % kTcTS;
-        mbar_wait_guarded(&tempty[t], ((gc / kTcTS) & 1) ^ 1, p.status, abort_flag);
-        tc_fence_after();
-        const uint32_t ta = tl + (uint32_t)t * 128u;
-        if constexpr (FMT == STRATA_FMT_Q2_32) {
+        const int nh = kv / kTcKH;
 #pragma unroll
-          for (int pc = 0; pc < NPC; ++pc) {
-            if (pc < np) {
-              uint32_t R[32];
-              const uint32_t d0 = dup_lo(sc[pc]), d1 = dup_hi(sc[pc]);
-              dq_q2_word(cw[pc].x, d0, R);
-              dq_q2_word(cw[pc].y, d0, R + 8);
-              dq_q2_word(cw[pc].z, d1, R + 16);
-              dq_q2_word(cw[pc].w, d1, R + 24);
-              tmem_st32(ta + pc * 32, R);
+        for (int h = 0; h < 2; ++h) {
+          if (h >= nh) break;
+          uint32_t R[64];
+          if constexpr (FMT == STRATA_FMT_Q2_32) {
+#pragma unroll
+            for (int pp = 0; pp < NPH; ++pp) {
+              const uint4 v = cw[h * NPH + pp];
+              dq_q2_word_raw(v.x, R + 32 * pp);
+              dq_q2_word_raw(v.y, R + 32 * pp + 8);
+              dq_q2_word_raw(v.z, R + 32 * pp + 16);
+              dq_q2_word_raw(v.w, R + 32 * pp + 24);
+            }
+          } else {
+#pragma unroll
+            for (int pp = 0; pp < NPH; ++pp) {
+              const uint4 v = cw[h * NPH + pp];
+              dq_q4_group_raw(v.x, v.y, T4, R + 16 * pp);
+              dq_q4_group_raw(v.z, v.w, T4, R + 16 * pp + 8);
             }
           }
-        } else {
-#pragma unroll
-          for (int pc = 0; pc < NPC; ++pc) {
-            if (pc < np) {
-              uint32_t R[16], R0[8], R1[8];
-              const __half2 d2 =
-                  u32_as_h2((pc & 1) ? dup_hi(sc[pc >> 1]) : dup_lo(sc[pc >> 1]));
-              dq_q4_group(cw[pc].x, cw[pc].y, d2, T4, R0);
-              dq_q4_group(cw[pc].z, cw[pc].w, d2, T4, R1);
-#pragma unroll
-              for (int j = 0; j < 8; ++j) {
-                R[j] = R0[j];
-                R[8 + j] = R1[j];
-              }
-              tmem_st16(ta + pc * 16, R);
-            }
-          }
+          const int stg = 2 * g + h;
+          mbar_wait_guarded(&afree[stg], ((par >> h) & 1u) ^ 1u, p.status, abort_flag);
+          par ^= 1u << h;
+          tc_fence_after();
+          const uint32_t ta = tmem_base + lane_off + (uint32_t)(stg * kTcStageCols);
+          tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(R));
+          tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(R + 32));
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&tfull[stg]);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&tfull[t]);
-      }
-      if (!isA) {
-        fence_proxy_async_smem();  // same for the scale block and its next bulk copy
-        mbar_arrive(&sempty[ib & 1]);
       }
     }
   } else if (warp == kTcMmaWarp) {
@@ -676,13 +813,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     if constexpr (MODE == 1) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
     if (elect_one()) {
       const uint32_t idesc = idesc_f16_f32(16);
-      const uint32_t sbo = p.NB == 16 ? 1024u : 0u;
-      const uint32_t ab = (uint32_t)p.NB * 128u;
+      const uint32_t sbo = NB == 16 ? 1024u : 0u;
+      const uint32_t ab = (uint32_t)NB * 128u;
       // descriptor start-address steps (16-byte units): one 64-K atom, one K16 step
       const uint64_t d_atom = ab >> 4, d_k16 = 32 >> 4;
       int gc = 0, bseq = -1, prev_e = -1;
+      uint32_t par = 0;  // bit st: parity of the next use of tensor-memory stage st
       for (int i = 0; i < tcount; ++i) {
-        const bool isA = kGU && (MODE == 0 || i < nA);
+        const bool isA = is_a(i);
         uint32_t bbase = smem_addr(smem + L.b);
         int b = 0;
         if (!isA) {
@@ -699,28 +837,34 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         }
         const int K = isA ? H : I;
         const int nch = isA ? nchA : nchB;
-        const int a = i & 1;
-        mbar_wait_guarded(&aempty[a], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
-        tc_fence_after();
-        const uint32_t d = tmem_base + (uint32_t)(a * 32);
         // B descriptor of the chunk's first K16 step; the steps inside a
-        // chunk are constant offsets from it (the loop is unrolled)
+        // chunk are constant offsets from it
         uint64_t bd = smem_desc_k128_sbo(bbase, sbo);
         for (int c = 0; c < nch; ++c, ++gc, bd += 4 * d_atom) {
-          const int t = gc % kTcTS;
-          mbar_wait_guarded(&tfull[t], (gc / kTcTS) & 1, p.status, abort_flag);
-          tc_fence_after();
-          const bool half = K - c * kTcKC < kTcKC;  // ragged last chunk: 128 K
-          const uint32_t at = tmem_base + kTcACol0 + (uint32_t)t * 128u;
+          const int g = gc % kTcGroups;
+          const int nh = (K - c * kTcKC) >= kTcKC ? 2 : 1;
 #pragma unroll
-          for (int kk = 0; kk < kTcKC / 16; ++kk) {
-            if (kk < kTcKC / 32 || !half)
-              mma_f16_ts(d, at + (uint32_t)kk * 8u, bd + (kk >> 2) * d_atom + (kk & 3) * d_k16,
-                         idesc, (c > 0 || kk > 0) ? 1u : 0u);
+          for (int h = 0; h < 2; ++h) {
+            if (h >= nh) break;
+            const int st = 2 * g + h;
+            const uint32_t ph = (par >> st) & 1u;
+            par ^= 1u << st;
+            mbar_wait_guarded(&tfull[st], ph, p.status, abort_flag);
+            mbar_wait_guarded(&accfree[st], ph ^ 1u, p.status, abort_flag);
+            tc_fence_after();
+            const uint32_t at = tmem_base + (uint32_t)(st * kTcStageCols);
+            const uint32_t dt = at + kTcAccCol;
+#pragma unroll
+            for (int kk = 0; kk < 8; ++kk) {
+              const int k16 = 8 * h + kk;  // K16 step within the chunk
+              mma_f16_ts(dt + 16u * (uint32_t)(kk >> 1), at + 8u * (uint32_t)kk,
+                         bd + (uint64_t)(k16 >> 2) * d_atom + (uint64_t)(k16 & 3) * d_k16, idesc,
+                         (uint32_t)(kk & 1));
+            }
+            mma_commit(&afree[st]);
+            mma_commit(&accfull[st]);
           }
-          mma_commit(&tempty[t]);
         }
-        mma_commit(&afull[a]);
         if (!isA) {
           if (i + 1 == tcount || tbl[i + 1].e != tbl[i].e) mma_commit(&bempty[b]);
         }
@@ -785,10 +929,10 @@ void pdl_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, in
   cfg.numAttrs = 1;
 }
 
-template <int MODE, int FMT>
+template <int MODE, int FMT, int NB>
 cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, cudaStream_t st) {
-  auto kern = decode_tc_kernel<MODE, FMT>;
-  const size_t smem = 1024 + tc_layout(MODE, FMT, prm.NB, prm.H, prm.I, prm.S, prm.maxT).total;
+  auto kern = decode_tc_kernel<MODE, FMT, NB>;
+  const size_t smem = 1024 + tc_layout(MODE, FMT, NB, prm.H, prm.I, prm.S, prm.maxT).total;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -796,6 +940,20 @@ cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, 
   cudaLaunchAttribute attr[1];
   pdl_config(cfg, attr, grid, kTcThreads, smem, st);
   return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], prm);
+}
+
+template <int MODE, int NB>
+cudaError_t launch_tc_fmt(int fmt, const CUtensorMap (&m)[6], const TcParams& prm, int grid,
+                          cudaStream_t st) {
+  if (fmt == STRATA_FMT_Q2_32) return launch_tc<MODE, STRATA_FMT_Q2_32, NB>(m, prm, grid, st);
+  return launch_tc<MODE, STRATA_FMT_Q4CB_32, NB>(m, prm, grid, st);
+}
+
+template <int MODE>
+cudaError_t launch_tc_nb(int NB, int fmt, const CUtensorMap (&m)[6], const TcParams& prm,
+                         int grid, cudaStream_t st) {
+  if (NB == 8) return launch_tc_fmt<MODE, 8>(fmt, m, prm, grid, st);
+  return launch_tc_fmt<MODE, 16>(fmt, m, prm, grid, st);
 }
 
 cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
@@ -881,29 +1039,23 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.active = a.active;
   prm.shared_mode = a.shared_mode;
   prm.hbuf = a.hbuf;
+  prm.zdn = a.zdn;
   prm.y = a.y;
   prm.status = a.status;
   prm.sync = a.sync;
-  prm.NB = NB;
   cudaError_t e;
   if (a.sync && tc_fused_fits(NB, a.H, a.I, Umax, a.fmt, a.num_sms)) {
     prm.maxT = tc_max_tiles(2, Umax, a.H, a.I, a.num_sms);
     prm.S = tc_stages(2, a.fmt, NB, a.H, a.I, prm.maxT);
     if ((e = launch_sync_reset(a.sync, Umax, st)) != cudaSuccess) return e;
-    if (q2) return launch_tc<2, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
-    return launch_tc<2, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+    return launch_tc_nb<2>(NB, a.fmt, m, prm, a.num_sms, st);
   }
   prm.maxT = tc_max_tiles(0, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);
-  if (q2)
-    e = launch_tc<0, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
-  else
-    e = launch_tc<0, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
-  if (e != cudaSuccess) return e;
+  if ((e = launch_tc_nb<0>(NB, a.fmt, m, prm, a.num_sms, st)) != cudaSuccess) return e;
   prm.maxT = tc_max_tiles(1, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(1, a.fmt, NB, a.H, a.I, prm.maxT);
-  if (q2) return launch_tc<1, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
-  return launch_tc<1, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+  return launch_tc_nb<1>(NB, a.fmt, m, prm, a.num_sms, st);
 }
 
 }  // namespace strata

@@ -155,6 +155,18 @@ STRATA_DEVFN void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 STRATA_DEVFN void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
+// Ties a register to the point after a tcgen05.wait::ld: the compiler keeps
+// volatile asm in order, and every use of x depends on this one.
+STRATA_DEVFN void reg_after_wait(uint32_t& x) { asm volatile("" : "+r"(x)); }
+
+// 32 lanes x 32 bits, one column per thread (thread i of the warp reads lane
+// base + i).  The column may differ between calls (a runtime address).
+STRATA_DEVFN uint32_t tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
+
 // Register -> tensor memory: 32 lanes x 32 bits, N consecutive columns per
 // thread (thread i of the warp writes lane base + i).
 STRATA_DEVFN void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
