@@ -57,9 +57,8 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_SUSTAINED = 1400.0
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 peak"
 NCU_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-DEFAULT_LINES = "2:8192,1:4"   # config:T, run in this order; the last is the headline
+DEFAULT_LINES = "2:8192,2:32768,1:4"   # config:T, in this order; the last is the headline
 OUT_REL_L2 = 5e-3
-NEAR_TIE_REL = 1e-5
 
 
 def peaks():
@@ -304,15 +303,18 @@ def rel_l2_rows(a, b):
 
 def _routing_compare(ref_logits, gpu_ids, k):
     """(exact tokens, near-tie tokens accepted, mismatched tokens) of the GPU
-    ids against the oracle's logits; the tie band is NEAR_TIE_REL."""
+    ids against the oracle's logits (the tie band of tests.harness: twice the
+    router-logit tolerance)."""
     from tests.harness import check_routing
     ok, near, bad = check_routing(ref_logits, gpu_ids, k)
     return near, bad
 
 
-def _near_ties(ref_logits, k, t_offset=0, max_list=16):
+def _near_ties(ref_logits, k, tokens, max_list=16):
+    """Near-tie listing of the oracle's logits of `tokens` (their rows in
+    ref_logits, in order)."""
     from tests.harness import near_tie_report
-    return [{"token": t + t_offset, "rank": r, "rel_gap": g}
+    return [{"token": int(tokens[t]), "rank": r, "gap": g}
             for t, r, g in near_tie_report(ref_logits, None, k, max_list)]
 
 
@@ -341,19 +343,22 @@ def parity_and_oracle_time(stack, rec, args):
         ulp_ok &= bool(np.all(np.abs(a - b) <= ulp))
         wr = u16(stack.wr[l])
         bias = None if stack.bias[l] is None else stack.bias[l].cpu().numpy()
+        # routing on every token up to 8192 tokens, else on every 4th token
+        rt = np.arange(T) if T <= 8192 else np.arange(0, T, 4)
         ref_lg = np.concatenate(parallel_rows(
-            lambda lo, hi: oracle.router_logits(hid[lo:hi], wr, bias), T, 256))
-        n_l, bad_l = _routing_compare(ref_lg, gids, k)
-        mismatched += [(l, t) for t in bad_l]
-        near += [(l, t) for t in n_l]
-        near_ties += [dict(layer=l, **d) for d in _near_ties(ref_lg, k)]
+            lambda lo, hi: oracle.router_logits(hid[rt[lo:hi]], wr, bias), len(rt), 256))
+        n_l, bad_l = _routing_compare(ref_lg, gids[rt], k)
+        mismatched += [(l, int(rt[t])) for t in bad_l]
+        near += [(l, int(rt[t])) for t in n_l]
+        near_ties += [dict(layer=l, **d) for d in _near_ties(ref_lg, k, rt)]
+        routed_checked = len(rt)
         if stack.decode:
             toks = np.arange(T)
         else:
             toks = stratified_tokens(stack.counts.cpu().numpy(), stack.offsets.cpu().numpy(),
                                      stack.perm.cpu().numpy(), k, T, n=args.prefill_sample,
                                      seed=l)
-        oracle_ids, _ = oracle.topk(ref_lg[toks], k)
+        oracle_ids, _ = oracle.topk(oracle.router_logits(hid[toks], wr, bias), k)
         _, _, blobs, sh = oracle_layer_inputs(stack, l, np.concatenate([oracle_ids.ravel(),
                                                                         gids[toks].ravel()]))
         # the timed oracle call: the whole layer on these tokens, routed by
@@ -375,7 +380,7 @@ def parity_and_oracle_time(stack, rec, args):
             break
     parity = {"layers_checked": checked, "layers": L,
               "tokens_checked_per_layer": int(len(toks)),
-              "routing_tokens_per_layer": T,
+              "routing_tokens_per_layer": routed_checked,
               "rmsnorm_within_1ulp": ulp_ok,
               "ids_exact": not mismatched and not near,
               "near_tie_tokens_accepted": [{"layer": a, "token": b} for a, b in near][:32],

@@ -17,6 +17,7 @@ FMT_Q2_32 = 1
 FMT_Q4CB_32 = 2
 DTYPE_F32 = 0
 DTYPE_F16 = 1
+DTYPE_BF16 = 2
 DECODE_MAX_T = 16
 DEV_TIMEOUT = 0x1
 DEV_BOUNDS = 0x2
@@ -60,6 +61,7 @@ _SIGS = {
     "moe_shared_expert_workspace_size": (_U64, [_QW, _I]),
     "moe_shared_expert": (_I, [_P, _QW, _I, _P, _P, _U64, _P, _P]),
     "moe_combine": (_I, [_P, _I, _P, _P, _P, _I, _P, _I, _I, _I, _P, _P, _P, _P]),
+    "moe_gather_rows": (_I, [_P, _I, _I, _I, _P, _I, _I, _P, _I, _P, _P]),
     "moe_layer_workspace_size": (_U64, [_I, _I, _I, _QW, _QW]),
     "moe_layer_forward": (_I, [_P, _I, _P, _P, _I, _I, _QW, _QW, _F, _P, _P, _P, _P, _P, _U64,
                                _P, _P]),
@@ -222,6 +224,13 @@ def moe_combine(y, y_dtype, inv, topk_w, shared_y, shared_dtype, residual, T, k,
                             shared_dtype, _ptr(residual), T, k, H, _ptr(out), _ptr(residual_out),
                             _ptr(dev_status), _stream(stream))
     return _check("moe_combine", rc) if check else rc
+
+
+def moe_gather_rows(src, src_dtype, n_src, H, idx, div, n, dst, dst_dtype, dev_status,
+                    stream=None, check=True):
+    rc = load().moe_gather_rows(_ptr(src), src_dtype, n_src, H, _ptr(idx), div, n, _ptr(dst),
+                                dst_dtype, _ptr(dev_status), _stream(stream))
+    return _check("moe_gather_rows", rc) if check else rc
 
 
 def moe_layer_workspace_size(T, E, k, w: QWeights, shared: QWeights | None) -> int:

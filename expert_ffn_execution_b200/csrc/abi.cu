@@ -347,6 +347,26 @@ int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* inv, const fl
                                   reinterpret_cast<cudaStream_t>(stream)));
 }
 
+namespace {
+int dtype_bytes(int32_t dt) {
+  return dt == STRATA_DTYPE_F32 ? 4 : (dt == STRATA_DTYPE_F16 || dt == STRATA_DTYPE_BF16) ? 2 : 0;
+}
+}  // namespace
+
+extern "C" int32_t moe_gather_rows(const void* src, int32_t src_dtype, int32_t n_src, int32_t H,
+                                   const int32_t* idx, int32_t div, int32_t n, void* dst,
+                                   int32_t dst_dtype, int32_t* dev_status, void* stream) {
+  const int sb = dtype_bytes(src_dtype), db = dtype_bytes(dst_dtype);
+  if (!sb || !db || n < 0 || n_src < 0 || div < 1 || H < 8 || H % 8) return STRATA_EINVAL;
+  const bool widen = src_dtype == STRATA_DTYPE_F16 && dst_dtype == STRATA_DTYPE_F32;
+  if (!widen && src_dtype != dst_dtype) return STRATA_EINVAL;
+  if (n == 0) return STRATA_OK;
+  if (!src || !idx || !dst || !aligned(src, 16) || !aligned(dst, 16)) return STRATA_EINVAL;
+  return from_cuda(launch_gather_rows(src, (uint64_t)H * sb, idx, div, n_src, n, dst,
+                                      widen ? 1 : 0, dev_status, num_sms_of_current_device(),
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
 // ---------------------------------------------------------------- composite
 namespace {
 struct LayerWs {

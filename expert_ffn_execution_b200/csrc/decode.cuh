@@ -76,6 +76,9 @@ uint64_t bucket_workspace_bytes(int T, int k, int E);
 cudaError_t launch_bucket(const int32_t* ids, int T, int k, int E, int32_t* counts,
                           int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* active,
                           void* ws, int32_t* status, cudaStream_t st);
+cudaError_t launch_gather_rows(const void* src, uint64_t src_row_bytes, const int32_t* idx,
+                               int div, int n_src, int n, void* dst, int widen,
+                               int32_t* status, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const void* y, int y_dtype, const int32_t* inv, const float* w,
                            const void* shared_y, int shared_dtype, const float* residual,
                            int T, int k, int H, uint16_t* out, float* residual_out,

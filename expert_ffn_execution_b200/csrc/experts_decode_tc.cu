@@ -108,6 +108,7 @@ struct TcParams {
   int32_t* sync;   // fused form: finished gate/up tiles per active expert (zeroed)
   int S;           // shared-memory stages (a multiple of kTcGroups)
   int maxT;        // capacity of the tile table: tiles per CTA at most
+  int hbn;         // h block buffers (2, or 1 where two leave too few stages)
 };
 
 struct TcTile {
@@ -122,7 +123,7 @@ __host__ __device__ constexpr int tc_cbr() {  // code bytes per row per chunk
 
 struct TcLayout {
   uint32_t codes_bytes, stage_bytes, b, b_bytes, zg, zg_bytes, hb, hb_bytes, zd, zd_bytes, sbuf,
-      s_bytes, xch, tbl, bars, total;
+      s_bytes, pt, xch, tbl, bars, total;
 };
 
 __host__ __device__ inline uint32_t up1k(uint32_t x) { return (x + 1023u) & ~1023u; }
@@ -130,11 +131,12 @@ __host__ __device__ inline uint32_t up128(uint32_t x) { return (x + 127u) & ~127
 
 // Shared memory, from a 1024-byte aligned base: S stages | gate/up: the token
 // block and its Z | down: two h blocks, their Z rows and two per-tile scale
-// blocks | gate/up: the SwiGLU exchange buffer (also the fused form's dealing
-// scratch) | the tile table | barriers.  Every TMA destination is 1024-byte
-// aligned, every bulk-copy destination 128-byte aligned.
-__host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, int I, int S,
-                                              int maxT) {
+// blocks | the decoder groups' partial sums of two tiles | gate/up: the SwiGLU
+// exchange buffer (also the fused form's dealing scratch) | the tile table |
+// barriers.  Every TMA destination is 1024-byte aligned, every bulk-copy
+// destination 128-byte aligned.
+__host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int TP, int H, int I,
+                                              int S, int maxT, int hbn) {
   TcLayout L;
   const bool gu = mode != 1, dn = mode != 0;
   const uint32_t cbr = fmt == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
@@ -149,13 +151,15 @@ __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, 
   off = up1k(off + L.zg_bytes);
   L.hb = off;
   L.hb_bytes = dn ? (uint32_t)NB * (uint32_t)I * 2u : 0u;
-  off += 2u * L.hb_bytes;
+  off += (uint32_t)hbn * L.hb_bytes;
   L.zd = off;
   L.zd_bytes = dn ? up128((uint32_t)NB * (uint32_t)(I / 32) * 4u) : 0u;
-  off += 2u * L.zd_bytes;
+  off += (uint32_t)hbn * L.zd_bytes;
   L.sbuf = off;
   L.s_bytes = dn ? up128(8u * (uint32_t)I) : 0u;
   off += 2u * L.s_bytes;
+  L.pt = off;
+  off += 2u * (uint32_t)kTcGroups * (uint32_t)TP * 128u * 4u;
   L.xch = off;
   off += gu ? up128(std::max(64u * 17u * 4u, 4u * (uint32_t)kTcMaxGrid)) : 0u;
   L.tbl = off;
@@ -288,7 +292,7 @@ STRATA_DEVFN void fill_tokens(uint8_t* bsm, float* zg, const uint16_t* __restric
 }
 
 // ---------------------------------------------------------------- kernel
-template <int MODE, int FMT, int NB>
+template <int MODE, int FMT, int NB, int TP>
 __global__ void __launch_bounds__(kTcThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
                  const __grid_constant__ CUtensorMap mu,   // up codes
@@ -302,27 +306,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   constexpr int PIECE_K = (FMT == STRATA_FMT_Q2_32) ? 64 : 32;  // K per 16-byte code piece
   constexpr int NPC = CBR / 16;                                  // pieces per full chunk
   constexpr int NPH = NPC / 2;                                   // pieces per half chunk
+  static_assert(TP <= NB, "token columns fit the B rows");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const TcLayout L = tc_layout(MODE, FMT, NB, p.H, p.I, p.S, p.maxT);
+  const TcLayout L = tc_layout(MODE, FMT, NB, TP, p.H, p.I, p.S, p.maxT, p.hbn);
   const int S = p.S;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + kTcMaxStages;
-  uint64_t* tfull = empty + kTcMaxStages;
-  uint64_t* afree = tfull + kTcTS;
-  uint64_t* accfull = afree + kTcTS;
-  uint64_t* accfree = accfull + kTcTS;
-  uint64_t* sfull = accfree + kTcTS;
+  uint64_t* accfull = empty + kTcMaxStages;
+  uint64_t* sfull = accfull + kTcTS;
   uint64_t* sempty = sfull + 2;
   uint64_t* bfull = sempty + 2;
   uint64_t* bempty = bfull + 2;
-  uint64_t* tbl_ready = bempty + 2;
+  uint64_t* pfull = bempty + 2;
+  uint64_t* pfree = pfull + 2;
+  uint64_t* tbl_ready = pfree + 2;
   uint64_t* done = tbl_ready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   TcTile* tbl = reinterpret_cast<TcTile*>(smem + L.tbl);
   float* zg = reinterpret_cast<float*>(smem + L.zg);
+  float* part = reinterpret_cast<float*>(smem + L.pt);  // [2 bufs][groups][TP][128 rows]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.H, I = p.I, T = p.T;
@@ -336,22 +341,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 256);  // the owning decoder group + the epilogue
+      mbar_init(&empty[s], 128);  // the decoder group that owns the chunk
     }
-    for (int t = 0; t < kTcTS; ++t) {
-      mbar_init(&tfull[t], 128);
-      mbar_init(&afree[t], 1);
-      mbar_init(&accfull[t], 1);
-      mbar_init(&accfree[t], 128);
-    }
+    for (int t = 0; t < kTcTS; ++t) mbar_init(&accfull[t], 1);
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sfull[a], 1);
-      mbar_init(&sempty[a], 128);
+      mbar_init(&sempty[a], 128 * kTcGroups);
       mbar_init(&bfull[a], 1);
-      mbar_init(&bempty[a], 1 + 128);  // the MMAs' commit + the epilogue's Z reads
+      mbar_init(&bempty[a], 128 * kTcGroups);  // after the decoders' last MMA and Z reads
+      mbar_init(&pfull[a], 128 * kTcGroups);
+      mbar_init(&pfree[a], 128);
     }
     mbar_init(tbl_ready, 128);
-    mbar_init(done, 1);
+    mbar_init(done, kTcGroups);  // each group's last MMAs
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -429,6 +431,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     rb = j - u * tpeB;
   };
   auto is_a = [&](int i) { return kGU && (MODE == 0 || i < nA); };
+  // buffer and phase parity of the q-th h block (one or two buffers)
+  auto hb_idx = [&](int q) { return p.hbn == 2 ? (q & 1) : 0; };
+  auto hb_par = [&](int q) { return (uint32_t)(p.hbn == 2 ? ((q >> 1) & 1) : (q & 1)); };
+  // the last down tile on an expert's h block (the buffer is then released)
+  auto last_on_h = [&](int i) { return i + 1 == tcount || tbl[i + 1].e != tbl[i].e; };
 
   if (warp == kTcProdWarp) {
     // ------------------------------------------------ TMA producer
@@ -445,14 +452,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
       // B buffer
       auto load_h = [&](int s0, int n) {
         ++bseq;
-        const int b = bseq & 1;
-        mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
+        const int b = hb_idx(bseq);
+        mbar_wait_guarded(&bempty[b], hb_par(bseq) ^ 1u, p.status, abort_flag);
         const uint32_t ab = (uint32_t)NB * 128u;
         const uint32_t zb = (uint32_t)n * (uint32_t)nbI * 4u;
         mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64) + zb);
         for (int a = 0; a < I / 64; ++a)
           tma_load_2d(smem + L.hb + b * L.hb_bytes + a * ab, &mh, 64 * a, s0, &bfull[b]);
-        bulk_g2s(smem + L.zd + b * L.zd_bytes, p.zdn + (size_t)s0 * nbI, zb, &bfull[b]);
+        if (zb) bulk_g2s(smem + L.zd + b * L.zd_bytes, p.zdn + (size_t)s0 * nbI, zb, &bfull[b]);
       };
       for (int i = 0; i < tcount; ++i) {
         if (is_a(i)) {
@@ -516,8 +523,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         mbar_wait_bounded(&full[x % S], (x / S) & 1, p.status, kDrain);
       for (int x = max(0, nB - 2); x < nB; ++x)
         mbar_wait_bounded(&sfull[x & 1], (x >> 1) & 1, p.status, kDrain);
-      for (int x = max(0, bseq - 1); x <= bseq; ++x)
-        mbar_wait_bounded(&bfull[x & 1], (x >> 1) & 1, p.status, kDrain);
+      for (int x = max(0, bseq - p.hbn + 1); x <= bseq; ++x)
+        mbar_wait_bounded(&bfull[hb_idx(x)], hb_par(x), p.status, kDrain);
     }
     __syncwarp();
   } else {
@@ -570,9 +577,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
             t.n = 0;
           }
         }
-        if (t.n < 0 || t.n > NB) {
+        if (t.n < 0 || t.n > TP) {
           dev_flag(p.status, STRATA_DEV_BOUNDS);
-          t.n = t.n < 0 ? 0 : NB;
+          t.n = t.n < 0 ? 0 : TP;
         }
       }
       named_bar_sync(1, 128);
@@ -595,135 +602,44 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   }
 
   if (warp < 4) {
-    // ------------------------------------------------ epilogue
+    // ------------------------------------------------ tile ends: the two
+    // decoder groups' partial sums, then SwiGLU / h / y
     mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
-    const int r = threadIdx.x;  // tile row = TMEM lane
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const int r = threadIdx.x;  // tile row
     float* xch = reinterpret_cast<float*>(smem + L.xch);
-    int gc = 0, bseq = -1, prev_e = -1;
-    uint32_t par = 0;  // bit st: parity of the next use of tensor-memory stage st
     for (int i = 0; i < tcount; ++i) {
       const TcTile& ti = tbl[i];
-      const bool isA = is_a(i);
-      const int ib = i - nA;
       const int n = ti.n;
-      const int nch = isA ? nchA : nchB;
-      const int K = isA ? H : I;
-      int col[NB];
+      const int pb = i & 1;
+      mbar_wait_backoff(&pfull[pb], (i >> 1) & 1, p.status, abort_flag);
+      const float* p0 = part + (size_t)pb * kTcGroups * TP * 128;
+      // column of pair j: its token (gate/up: B holds every token) or j (down)
+      auto val = [&](int j) {
+        const int col = is_a(i) ? ti.tok[j] : j;
+        float v = 0.f;
 #pragma unroll
-      for (int j = 0; j < NB; ++j) col[j] = isA ? ((j < n) ? ti.tok[j] : 0) : j;
-      const float* zsrc = zg;
-      if (!isA) {
-        mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
-        if (ib == 0 || ti.e != prev_e) ++bseq;
-        prev_e = ti.e;
-        // Z rows of this expert's h (they arrive with the h block)
-        mbar_wait_guarded(&bfull[bseq & 1], (bseq >> 1) & 1, p.status, abort_flag);
-        zsrc = reinterpret_cast<const float*>(smem + L.zd + (bseq & 1) * L.zd_bytes);
-      }
-      const uint8_t* srow =
-          isA ? nullptr : smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
-      float acc[NB];
-#pragma unroll
-      for (int j = 0; j < NB; ++j) acc[j] = 0.f;
-      for (int c = 0; c < nch; ++c, ++gc) {
-        const int g = gc % kTcGroups;
-        const int s = gc % S;
-        // this row's 8 block scales of the chunk (gate/up: in the stage)
-        uint4 scv;
-        if (isA) {
-          mbar_wait_guarded(&full[s], (gc / S) & 1, p.status, abort_flag);
-          scv = lds128(smem + s * L.stage_bytes + L.codes_bytes + r * 16);
-        } else {
-          const int nb4 = min(8, (K - c * kTcKC) / 32);
-          const uint2 lo = lds64(srow + c * 16);
-          scv = make_uint4(lo.x, lo.y, 0u, 0u);
-          if (nb4 > 4) {
-            const uint2 hi = lds64(srow + c * 16 + 8);
-            scv.z = hi.x;
-            scv.w = hi.y;
-          }
-        }
-        const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
-        const int nh = (K - c * kTcKC) >= kTcKC ? 2 : 1;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (h >= nh) break;
-          const int st = 2 * g + h;
-          mbar_wait_backoff(&accfull[st], (par >> st) & 1u, p.status, abort_flag);
-          par ^= 1u << st;
-          tc_fence_after();
-          const uint32_t acc_t = tmem_base + lane_off + (uint32_t)(st * kTcStageCols + kTcAccCol);
-          // the four block accumulators, QB blocks per pass (registers)
-          constexpr int QB = NB == 16 ? 2 : 4;
-#pragma unroll
-          for (int q0 = 0; q0 < 4; q0 += QB) {
-            uint32_t D[QB][NB];
-#pragma unroll
-            for (int q = 0; q < QB; ++q)
-#pragma unroll
-              for (int j = 0; j < NB; ++j)
-                if (j < n) D[q][j] = tmem_ld1(acc_t + (uint32_t)(16 * (q0 + q) + col[j]));
-            tmem_wait_ld();
-#pragma unroll
-            for (int q = 0; q < QB; ++q)
-#pragma unroll
-              for (int j = 0; j < NB; ++j)
-                if (j < n) reg_after_wait(D[q][j]);
-            if (q0 + QB == 4) {
-              tc_fence_before();
-              mbar_arrive(&accfree[st]);
-            }
-#pragma unroll
-            for (int q = 0; q < QB; ++q) {
-              const int qq = 4 * h + q0 + q;  // block within the chunk
-              const float d = (qq & 1) ? half_hi(scw[qq >> 1]) : half_lo(scw[qq >> 1]);
-              const int b = c * 8 + qq;  // block along K
-#pragma unroll
-              for (int j = 0; j < NB; ++j) {
-                if (j < n) {
-                  const float z = isA ? zsrc[b * NB + col[j]] : zsrc[j * nbI + b];
-                  acc[j] = fmaf(d, __uint_as_float(D[q][j]) - z, acc[j]);
-                }
-              }
-            }
-          }
-        }
-        // the stage's (gate/up: scale) reads are done: order them before the
-        // producer's next TMA write, then release
-        fence_proxy_async_smem();
-        mbar_arrive(&empty[s]);
-      }
-      if (!isA) {
-        fence_proxy_async_smem();
-        mbar_arrive(&sempty[ib & 1]);
-        // the last tile on this h block: its Z rows are read
-        if (i + 1 == tcount || tbl[i + 1].e != ti.e) mbar_arrive(&bempty[bseq & 1]);
-      }
-      if (isA) {
+        for (int g = 0; g < kTcGroups; ++g) v += p0[(g * TP + col) * 128 + r];
+        return v;
+      };
+      if (is_a(i)) {
         // SwiGLU: rows 0-63 gate, 64-127 the same up rows
         if (r >= 64) {
-#pragma unroll
-          for (int j = 0; j < NB; ++j)
-            if (j < n) xch[(r - 64) * 17 + j] = acc[j];
+          for (int j = 0; j < n; ++j) xch[(r - 64) * 17 + j] = val(j);
         }
         named_bar_sync(1, 128);
         if (r < 64) {
           const int ii = ti.rb * 64 + r;  // row of I
           const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
           const float off = FMT == STRATA_FMT_Q2_32 ? q2_offset(ii & 15) : kQ4Offset;
+          for (int j = 0; j < n; ++j) {
+            const float hv = silu_f32(val(j)) * xch[r * 17 + j];
+            const __half h16 = __float2half_rn(hv);
+            p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(h16);
+            // this h row's Z over the 32-block of rows (one warp), in lane order
+            float zc = off * __half2float(h16);
 #pragma unroll
-          for (int j = 0; j < NB; ++j) {
-            if (j < n) {
-              const float hv = silu_f32(acc[j]) * xch[r * 17 + j];
-              const __half h16 = __float2half_rn(hv);
-              p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(h16);
-              // this h row's Z over the 32-block of rows (one warp), in lane order
-              float zc = off * __half2float(h16);
-#pragma unroll
-              for (int o = 1; o < 32; o <<= 1) zc += __shfl_xor_sync(0xffffffffu, zc, o);
-              if (lane == 0) p.zdn[(size_t)(ti.s0 + j) * nbI + (ii >> 5)] = zc;
-            }
+            for (int o = 1; o < 32; o <<= 1) zc += __shfl_xor_sync(0xffffffffu, zc, o);
+            if (lane == 0) p.zdn[(size_t)(ti.s0 + j) * nbI + (ii >> 5)] = zc;
           }
           if constexpr (MODE == 2) {
             // publish this thread's h and Z stores (to the TMA reads of
@@ -738,25 +654,51 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         }
       } else if constexpr (kDN) {
         const int row = ti.rb * 128 + r;
-#pragma unroll
-        for (int j = 0; j < NB; ++j)
-          if (j < n) p.y[(size_t)(ti.s0 + j) * H + row] = acc[j];
+        for (int j = 0; j < n; ++j) p.y[(size_t)(ti.s0 + j) * H + row] = val(j);
       }
+      mbar_arrive(&pfree[pb]);
     }
   } else if (warp < kTcProdWarp) {
-    // ------------------------------------------------ decoders
+    // ------------------------------------------------ decoders (and the
+    // per-block scale/offset epilogue of their own half chunks)
     const int g = (warp - kTcDecWarp0) >> 2;
     const int qd = warp & 3;
     const int r = 32 * qd + lane;  // tile row = TMEM lane
     const uint32_t swz = ((uint32_t)(r * CBR) >> 7) & (uint32_t)(NPC - 1);
     const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
     const Q4Table T4 = q4_table();
-    int gc = 0;
-    uint32_t par = 0;  // bit h: parity of the next use of this group's stage 2g + h
+    const bool leader = r == 0;  // issues the group's MMAs
+    const uint32_t idesc = idesc_f16_f32(16);
+    const uint32_t sbo = NB == 16 ? 1024u : 0u;
+    // descriptor start-address steps (16-byte units): one 64-K atom, one K16 step
+    const uint32_t d_atom = ((uint32_t)NB * 128u) >> 4, d_k16 = 32u >> 4;
+    const uint32_t bhi = smem_desc_k128_hi(sbo);
+    int gc = 0, bseq = -1, prev_e = -1;
+    uint32_t par = 0;  // bit h: parity of the next accumulator wait of stage 2g + h
     for (int i = 0; i < tcount; ++i) {
       const bool isA = is_a(i);
       const int K = isA ? H : I;
       const int nch = isA ? nchA : nchB;
+      const int ib = i - nA;
+      const float* zsrc = zg;  // gate/up: [block][NB tokens]; down: [pair][nbI blocks]
+      const uint8_t* srow = nullptr;
+      if (!isA) {
+        if (ib == 0) mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
+        const int e = tbl[i].e;
+        if (ib == 0 || e != prev_e) ++bseq;
+        prev_e = e;
+        mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
+        mbar_wait_guarded(&bfull[hb_idx(bseq)], hb_par(bseq), p.status, abort_flag);
+        zsrc = reinterpret_cast<const float*>(smem + L.zd + hb_idx(bseq) * L.zd_bytes);
+        srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
+      }
+      // B: every token (gate/up) or the expert's h block (down)
+      const uint32_t bbase = isA ? smem_addr(smem + L.b)
+                                 : smem_addr(smem + L.hb) + (uint32_t)hb_idx(bseq) * L.hb_bytes;
+      const uint32_t blo0 = smem_desc_k128_lo(bbase);
+      float acc[TP];
+#pragma unroll
+      for (int t = 0; t < TP; ++t) acc[t] = 0.f;
       for (int c = 0; c < nch; ++c, ++gc) {
         if (gc % kTcGroups != g) continue;
         const int s = gc % S;
@@ -768,12 +710,27 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
 #pragma unroll
         for (int pc = 0; pc < NPC; ++pc)
           cw[pc] = (pc < np) ? lds128(st + r * CBR + ((pc ^ swz) << 4)) : make_uint4(0, 0, 0, 0);
+        // this row's 8 block scales of the chunk
+        uint4 scv;
+        if (isA) {
+          scv = lds128(st + L.codes_bytes + r * 16);
+        } else {
+          const uint2 lo = lds64(srow + c * 16);
+          scv = make_uint4(lo.x, lo.y, 0u, 0u);
+          if (kv > kTcKH) {
+            const uint2 hi = lds64(srow + c * 16 + 8);
+            scv.z = hi.x;
+            scv.w = hi.y;
+          }
+        }
         // The stage is released before its loads are consumed: order those
         // generic-proxy reads before the producer's next TMA (async-proxy)
         // write into the stage, which the barrier alone does not.
         fence_proxy_async_smem();
         mbar_arrive(&empty[s]);
         const int nh = kv / kTcKH;
+        // decode both halves into the group's two tensor-memory stages (the
+        // previous use of a stage was read back by this thread already)
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           if (h >= nh) break;
@@ -796,83 +753,86 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
             }
           }
           const int stg = 2 * g + h;
-          mbar_wait_guarded(&afree[stg], ((par >> h) & 1u) ^ 1u, p.status, abort_flag);
-          par ^= 1u << h;
-          tc_fence_after();
           const uint32_t ta = tmem_base + lane_off + (uint32_t)(stg * kTcStageCols);
           tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(R));
           tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(R + 32));
           tmem_wait_st();
           tc_fence_before();
-          mbar_arrive(&tfull[stg]);
-        }
-      }
-    }
-  } else if (warp == kTcMmaWarp) {
-    // ------------------------------------------------ MMA issue (one thread)
-    if constexpr (MODE == 1) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
-    if (elect_one()) {
-      const uint32_t idesc = idesc_f16_f32(16);
-      const uint32_t sbo = NB == 16 ? 1024u : 0u;
-      const uint32_t ab = (uint32_t)NB * 128u;
-      // descriptor start-address steps (16-byte units): one 64-K atom, one K16 step
-      const uint64_t d_atom = ab >> 4, d_k16 = 32 >> 4;
-      int gc = 0, bseq = -1, prev_e = -1;
-      uint32_t par = 0;  // bit st: parity of the next use of tensor-memory stage st
-      for (int i = 0; i < tcount; ++i) {
-        const bool isA = is_a(i);
-        uint32_t bbase = smem_addr(smem + L.b);
-        int b = 0;
-        if (!isA) {
-          if (MODE == 2 && i == nA) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
-          const int e = tbl[i].e;
-          if (i == nA || e != prev_e) {
-            ++bseq;
-            mbar_wait_guarded(&bfull[bseq & 1], (bseq >> 1) & 1, p.status, abort_flag);
+          // every row of the half is in tensor memory: one thread multiplies
+          // its four blocks into their accumulators (K16 steps in pairs)
+          named_bar_sync(3 + g, 128);
+          if (leader) {
             tc_fence_after();
-          }
-          prev_e = e;
-          b = bseq & 1;
-          bbase = smem_addr(smem + L.hb) + (uint32_t)b * L.hb_bytes;
-        }
-        const int K = isA ? H : I;
-        const int nch = isA ? nchA : nchB;
-        // B descriptor of the chunk's first K16 step; the steps inside a
-        // chunk are constant offsets from it
-        uint64_t bd = smem_desc_k128_sbo(bbase, sbo);
-        for (int c = 0; c < nch; ++c, ++gc, bd += 4 * d_atom) {
-          const int g = gc % kTcGroups;
-          const int nh = (K - c * kTcKC) >= kTcKC ? 2 : 1;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            if (h >= nh) break;
-            const int st = 2 * g + h;
-            const uint32_t ph = (par >> st) & 1u;
-            par ^= 1u << st;
-            mbar_wait_guarded(&tfull[st], ph, p.status, abort_flag);
-            mbar_wait_guarded(&accfree[st], ph ^ 1u, p.status, abort_flag);
-            tc_fence_after();
-            const uint32_t at = tmem_base + (uint32_t)(st * kTcStageCols);
+            const uint32_t at = tmem_base + (uint32_t)(stg * kTcStageCols);
             const uint32_t dt = at + kTcAccCol;
+            const uint32_t blo = blo0 + (uint32_t)c * 4u * d_atom;
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const int k16 = 8 * h + kk;  // K16 step within the chunk
               mma_f16_ts(dt + 16u * (uint32_t)(kk >> 1), at + 8u * (uint32_t)kk,
-                         bd + (uint64_t)(k16 >> 2) * d_atom + (uint64_t)(k16 & 3) * d_k16, idesc,
-                         (uint32_t)(kk & 1));
+                         blo + (uint32_t)(k16 >> 2) * d_atom + (uint32_t)(k16 & 3) * d_k16, bhi,
+                         idesc, (uint32_t)(kk & 1));
             }
-            mma_commit(&afree[st]);
-            mma_commit(&accfull[st]);
+            mma_commit(&accfull[stg]);
           }
         }
-        if (!isA) {
-          if (i + 1 == tcount || tbl[i + 1].e != tbl[i].e) mma_commit(&bempty[b]);
+        // the two halves' block accumulators: y += d_b (D_b - Z_b)
+        const uint32_t scw[4] = {scv.x, scv.y, scv.z, scv.w};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h >= nh) break;
+          const int stg = 2 * g + h;
+          mbar_wait_guarded(&accfull[stg], (par >> h) & 1u, p.status, abort_flag);
+          par ^= 1u << h;
+          tc_fence_after();
+          const uint32_t acc_t =
+              tmem_base + lane_off + (uint32_t)(stg * kTcStageCols + kTcAccCol);
+          // QB of the four block accumulators per pass (registers)
+          constexpr int QB = TP == 16 ? 2 : 4;
+#pragma unroll
+          for (int q0 = 0; q0 < 4; q0 += QB) {
+            uint32_t D[QB][TP];  // the loads and their wait are one asm statement
+            if constexpr (TP == 4)
+              tmem_ld4x4_wait(acc_t, acc_t + 16u, acc_t + 32u, acc_t + 48u,
+                              *reinterpret_cast<uint32_t(*)[16]>(&D[0][0]));
+            else if constexpr (TP == 8)
+              tmem_ld8x4_wait(acc_t, acc_t + 16u, acc_t + 32u, acc_t + 48u,
+                              *reinterpret_cast<uint32_t(*)[32]>(&D[0][0]));
+            else
+              tmem_ld16x2_wait(acc_t + 16u * (uint32_t)q0, acc_t + 16u * (uint32_t)(q0 + 1),
+                               *reinterpret_cast<uint32_t(*)[32]>(&D[0][0]));
+#pragma unroll
+            for (int q = 0; q < QB; ++q) {
+              const int qq = 4 * h + q0 + q;  // block within the chunk
+              const float d = (qq & 1) ? half_hi(scw[qq >> 1]) : half_lo(scw[qq >> 1]);
+              const int b = c * 8 + qq;  // block along K
+#pragma unroll
+              for (int t = 0; t < TP; ++t) {
+                const float z = isA ? zsrc[b * NB + t] : zsrc[t * nbI + b];
+                acc[t] = fmaf(d, __uint_as_float(D[q][t]) - z, acc[t]);
+              }
+            }
+          }
         }
       }
-      mma_commit(done);
-      // every MMA retired before the tensor memory is released (bounded)
-      mbar_wait_bounded(done, 0, p.status);
+      // this group's partial sums of the tile, for the tile-end warps
+      const int pb = i & 1;
+      mbar_wait_guarded(&pfree[pb], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
+      float* pp = part + ((size_t)pb * kTcGroups + g) * TP * 128;
+#pragma unroll
+      for (int t = 0; t < TP; ++t) pp[t * 128 + r] = acc[t];
+      mbar_arrive(&pfull[pb]);
+      if (!isA) {
+        fence_proxy_async_smem();  // scale and Z reads before the next bulk copies
+        mbar_arrive(&sempty[ib & 1]);
+        if (last_on_h(i)) mbar_arrive(&bempty[hb_idx(bseq)]);
+      }
     }
+    if (leader) mma_commit(done);  // arrives once the group's MMAs are done
+  } else if (warp == kTcMmaWarp) {
+    // ------------------------------------------------ tensor memory owner:
+    // every MMA of both groups retired before it is released (bounded)
+    if (lane == 0) mbar_wait_bounded(done, 0, p.status);
     __syncwarp();
   }
   tc_fence_before();
@@ -908,8 +868,8 @@ int tc_max_tiles(int mode, int Umax, int H, int I, int grid) {
 // group count: chunk c uses stage c % S and group c % kTcGroups, so every
 // use of a stage belongs to one group and its barrier phases are awaited in
 // order (a waiter two phases ahead would see its parity as complete).
-int tc_stages(int mode, int fmt, int NB, int H, int I, int maxT) {
-  const TcLayout L0 = tc_layout(mode, fmt, NB, H, I, 0, maxT);
+int tc_stages(int mode, int fmt, int NB, int TP, int H, int I, int maxT, int hbn) {
+  const TcLayout L0 = tc_layout(mode, fmt, NB, TP, H, I, 0, maxT, hbn);
   const long long room = (long long)kTcSmemBudget - 1024 - (long long)L0.total;
   if (room <= 0) return 0;
   const int s = (int)std::min<long long>(kTcMaxStages, room / L0.stage_bytes);
@@ -929,10 +889,11 @@ void pdl_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, in
   cfg.numAttrs = 1;
 }
 
-template <int MODE, int FMT, int NB>
+template <int MODE, int FMT, int NB, int TP>
 cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, cudaStream_t st) {
-  auto kern = decode_tc_kernel<MODE, FMT, NB>;
-  const size_t smem = 1024 + tc_layout(MODE, FMT, NB, prm.H, prm.I, prm.S, prm.maxT).total;
+  auto kern = decode_tc_kernel<MODE, FMT, NB, TP>;
+  const size_t smem =
+      1024 + tc_layout(MODE, FMT, NB, TP, prm.H, prm.I, prm.S, prm.maxT, prm.hbn).total;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -942,18 +903,24 @@ cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, 
   return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], prm);
 }
 
-template <int MODE, int NB>
+template <int MODE, int NB, int TP>
 cudaError_t launch_tc_fmt(int fmt, const CUtensorMap (&m)[6], const TcParams& prm, int grid,
                           cudaStream_t st) {
-  if (fmt == STRATA_FMT_Q2_32) return launch_tc<MODE, STRATA_FMT_Q2_32, NB>(m, prm, grid, st);
-  return launch_tc<MODE, STRATA_FMT_Q4CB_32, NB>(m, prm, grid, st);
+  if (fmt == STRATA_FMT_Q2_32) return launch_tc<MODE, STRATA_FMT_Q2_32, NB, TP>(m, prm, grid, st);
+  return launch_tc<MODE, STRATA_FMT_Q4CB_32, NB, TP>(m, prm, grid, st);
 }
 
+// B rows NB (8: rows 8-15 of the N = 16 MMA repeat rows 0-7) and the token
+// columns TP the epilogue reads, from the call's token count.
+inline int tc_nb(int T) { return T <= 8 ? 8 : 16; }
+inline int tc_tp(int T) { return T <= 4 ? 4 : T <= 8 ? 8 : 16; }
+
 template <int MODE>
-cudaError_t launch_tc_nb(int NB, int fmt, const CUtensorMap (&m)[6], const TcParams& prm,
+cudaError_t launch_tc_nb(int T, int fmt, const CUtensorMap (&m)[6], const TcParams& prm,
                          int grid, cudaStream_t st) {
-  if (NB == 8) return launch_tc_fmt<MODE, 8>(fmt, m, prm, grid, st);
-  return launch_tc_fmt<MODE, 16>(fmt, m, prm, grid, st);
+  if (T <= 4) return launch_tc_fmt<MODE, 8, 4>(fmt, m, prm, grid, st);
+  if (T <= 8) return launch_tc_fmt<MODE, 8, 8>(fmt, m, prm, grid, st);
+  return launch_tc_fmt<MODE, 16, 16>(fmt, m, prm, grid, st);
 }
 
 cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
@@ -963,18 +930,33 @@ cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, tc_sync_reset_kernel, sync, n);
 }
 
-bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
-  return grid <= kTcMaxGrid &&
-         tc_stages(2, fmt, NB, H, I, tc_max_tiles(2, Umax, H, I, grid)) >= kTcFusedMinStages;
+// Stages and h buffers of one kernel form: two h buffers unless that leaves
+// fewer than `want` stages.
+constexpr int kTcWantStages = 6;
+void tc_plan(int mode, int fmt, int T, int H, int I, int maxT, int want, int& S, int& hbn) {
+  hbn = 2;
+  S = tc_stages(mode, fmt, tc_nb(T), tc_tp(T), H, I, maxT, 2);
+  if (mode != 0 && S < want) {
+    hbn = 1;
+    S = tc_stages(mode, fmt, tc_nb(T), tc_tp(T), H, I, maxT, 1);
+  }
+}
+
+bool tc_fused_fits(int T, int H, int I, int Umax, int fmt, int grid) {
+  if (grid > kTcMaxGrid) return false;
+  int S, hbn;
+  tc_plan(2, fmt, T, H, I, tc_max_tiles(2, Umax, H, I, grid), kTcFusedMinStages, S, hbn);
+  return S >= kTcFusedMinStages;
 }
 
 }  // namespace
 
 bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid) {
   if (T < 1 || T > kDecodeMaxTokens || H % 256 || I % 128 || grid < 1 || Umax < 1) return false;
-  const int NB = T <= 8 ? 8 : 16;
-  return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, Umax, H, I, grid)) >= kTcGroups &&
-         tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, Umax, H, I, grid)) >= kTcGroups;
+  int S0, S1, hbn;
+  tc_plan(0, fmt, T, H, I, tc_max_tiles(0, Umax, H, I, grid), kTcWantStages, S0, hbn);
+  tc_plan(1, fmt, T, H, I, tc_max_tiles(1, Umax, H, I, grid), kTcWantStages, S1, hbn);
+  return S0 >= kTcGroups && S1 >= kTcGroups;
 }
 
 cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
@@ -982,7 +964,7 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   const long long P = a.shared_mode ? a.T : (long long)a.T * a.k;
   const int Umax = a.shared_mode ? 1 : (int)std::min<long long>(a.E, P);
   if (!decode_tc_supported(a.T, a.H, a.I, Umax, a.fmt, a.num_sms)) return cudaErrorNotSupported;
-  const int NB = a.T <= 8 ? 8 : 16;
+  const int NB = tc_nb(a.T);
   const Planes PL = plane_offsets(a.fmt, a.H, a.I);
   const bool q2 = a.fmt == STRATA_FMT_Q2_32;
   const cuuint32_t cbr = q2 ? kTcKC / 4 : kTcKC / 2;
@@ -1044,18 +1026,18 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.status = a.status;
   prm.sync = a.sync;
   cudaError_t e;
-  if (a.sync && tc_fused_fits(NB, a.H, a.I, Umax, a.fmt, a.num_sms)) {
+  if (a.sync && tc_fused_fits(a.T, a.H, a.I, Umax, a.fmt, a.num_sms)) {
     prm.maxT = tc_max_tiles(2, Umax, a.H, a.I, a.num_sms);
-    prm.S = tc_stages(2, a.fmt, NB, a.H, a.I, prm.maxT);
+    tc_plan(2, a.fmt, a.T, a.H, a.I, prm.maxT, kTcFusedMinStages, prm.S, prm.hbn);
     if ((e = launch_sync_reset(a.sync, Umax, st)) != cudaSuccess) return e;
-    return launch_tc_nb<2>(NB, a.fmt, m, prm, a.num_sms, st);
+    return launch_tc_nb<2>(a.T, a.fmt, m, prm, a.num_sms, st);
   }
   prm.maxT = tc_max_tiles(0, Umax, a.H, a.I, a.num_sms);
-  prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);
-  if ((e = launch_tc_nb<0>(NB, a.fmt, m, prm, a.num_sms, st)) != cudaSuccess) return e;
+  tc_plan(0, a.fmt, a.T, a.H, a.I, prm.maxT, kTcWantStages, prm.S, prm.hbn);
+  if ((e = launch_tc_nb<0>(a.T, a.fmt, m, prm, a.num_sms, st)) != cudaSuccess) return e;
   prm.maxT = tc_max_tiles(1, Umax, a.H, a.I, a.num_sms);
-  prm.S = tc_stages(1, a.fmt, NB, a.H, a.I, prm.maxT);
-  return launch_tc_nb<1>(NB, a.fmt, m, prm, a.num_sms, st);
+  tc_plan(1, a.fmt, a.T, a.H, a.I, prm.maxT, kTcWantStages, prm.S, prm.hbn);
+  return launch_tc_nb<1>(a.T, a.fmt, m, prm, a.num_sms, st);
 }
 
 }  // namespace strata

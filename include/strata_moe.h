@@ -97,9 +97,10 @@ typedef enum strata_status {
 #define STRATA_FMT_Q2_32 1
 #define STRATA_FMT_Q4CB_32 2
 
-/* Element types of expert outputs y. */
+/* Element types of expert outputs y (and of moe_gather_rows rows). */
 #define STRATA_DTYPE_F32 0
 #define STRATA_DTYPE_F16 1
+#define STRATA_DTYPE_BF16 2
 
 /* Largest T served by the weight-streaming decode path of moe_experts;
  * larger T takes the tensor-core grouped-GEMM path. */
@@ -299,6 +300,22 @@ STRATA_API int32_t moe_combine(const void* y, int32_t y_dtype, const int32_t* in
                     int32_t shared_dtype, const float* residual, int32_t T,
                     int32_t k, int32_t H, uint16_t* out, float* residual_out,
                     int32_t* dev_status, void* stream);
+
+/* Row gather, the data movement of expert parallelism (the pages mention
+ * experts on several GPUs, lcz.me/topic/2153 "path D" list; they give no
+ * kernel for it):  dst[i] = src[idx[i] / div] for i < n.
+ *   src   [n_src, H] rows of src_dtype; dst [n, H] rows of dst_dtype
+ *   idx   int32 [n]; an index outside [0, n_src*div) sets STRATA_DEV_BOUNDS
+ *         and that row of dst is written as zeros
+ *   div   >= 1 (k: the hidden rows of (token, slot) pairs in sorted order,
+ *         idx = perm; 1: rows put back in another order, idx = inv)
+ *   dtypes STRATA_DTYPE_F32 / _F16 / _BF16; dst_dtype == src_dtype, or
+ *         src F16 -> dst F32 (exact widening)
+ * H a multiple of 8; src and dst 16-byte aligned.  n == 0 is a no-op. */
+STRATA_API int32_t moe_gather_rows(const void* src, int32_t src_dtype, int32_t n_src,
+                                   int32_t H, const int32_t* idx, int32_t div, int32_t n,
+                                   void* dst, int32_t dst_dtype, int32_t* dev_status,
+                                   void* stream);
 
 /* The whole layer in one call: moe_rmsnorm(x) -> moe_router_topk ->
  * moe_bucket -> moe_experts -> moe_shared_expert (if `shared` != NULL) ->

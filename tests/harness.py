@@ -5,7 +5,13 @@ from __future__ import annotations
 
 import numpy as np
 
-NEAR_TIE_REL = 1e-5       # near-tie band on oracle logits (relative)
+# Router logits: the kernels sum H bf16 x bf16 products in fp32 (about H/16
+# sequential fp32 additions of K16 partial sums); the oracle sums in fp64 and
+# rounds once.  With |x w| summing to about 40 at the workloads' magnitudes
+# (H <= 4096, W_r ~ N(0, 0.02), RMS-normalised x), four standard deviations of
+# that rounding walk, sqrt(H/16) * 2^-24 * 40 * 4, come to about 1e-4.
+ROUTER_LOGIT_ATOL = 1e-4
+ROUTER_LOGIT_RTOL = 1e-4
 TOPK_W_ATOL = 1e-5        # |GPU w - oracle w|
 OUT_REL_L2 = 5e-3         # per-token relative L2 of the layer output
 
@@ -28,44 +34,64 @@ def oracle_topk_order(logits, k):
     return order[:, :min(E, k + 1)]
 
 
-def check_routing(oracle_logits, gpu_ids, k):
+def logit_tol(ref):
+    """Tolerance on a GPU router logit against the oracle's value `ref`."""
+    return ROUTER_LOGIT_ATOL + ROUTER_LOGIT_RTOL * np.abs(ref)
+
+
+def tie_band(a, b):
+    """Two oracle logits closer than this may be ranked either way by a kernel
+    whose logits each lie within logit_tol of the oracle's."""
+    return 2.0 * (ROUTER_LOGIT_ATOL + ROUTER_LOGIT_RTOL * max(abs(a), abs(b)))
+
+
+def check_routing(oracle_logits, gpu_ids, k, gpu_logits=None):
     """Compare GPU top-k ids with the oracle's logits.
 
-    A token is exact if the GPU ids equal the oracle's sorted top-k (logit
-    descending, index ascending).  It is a near-tie if two adjacent logits
-    among the oracle's top k+1 differ by less than NEAR_TIE_REL relative; a
-    near-tie token is accepted when, position by position, the GPU's expert
-    has an oracle logit within the tie band of the oracle's logit at that
-    rank.  Returns (ok, near_tie_tokens, mismatched_tokens)."""
+    The top-k is a decision taken on floating-point logits, so it is checked
+    in the precision the kernel takes it in: when the GPU's own logits are
+    given, its ids must be their top-k (logit descending, index ascending)
+    exactly, for every token.  Against the oracle, a token is exact if the
+    GPU ids equal the oracle's sorted top-k; otherwise it is accepted as a
+    near tie when the GPU's ids are k distinct experts and, rank by rank, the
+    GPU's expert has an oracle logit within tie_band of the oracle's logit at
+    that rank.  Returns (ok, near_tie_tokens, mismatched_tokens); a token
+    whose ids are not the top-k of the GPU's logits counts as mismatched."""
     L = np.asarray(oracle_logits, np.float64)
     T, E = L.shape
     ids = np.asarray(gpu_ids)
+    bad = set()
+    if gpu_logits is not None:
+        own = oracle_topk_order(np.asarray(gpu_logits, np.float64), k)[:, :k]
+        bad.update(int(t) for t in np.nonzero(~(own == ids).all(axis=1))[0])
     order = oracle_topk_order(L, k)
     exact = (order[:, :k] == ids).all(axis=1)
-    near, bad = [], []
+    near = []
     for t in np.nonzero(~exact)[0]:
         top = [L[t, e] for e in order[t]]
-        tie = any(abs(top[i] - top[i + 1]) < NEAR_TIE_REL * max(abs(top[i]), abs(top[i + 1]))
-                  for i in range(len(top) - 1))
-        ok = tie and len(set(ids[t])) == k and all(
-            0 <= ids[t, j] < E and abs(L[t, ids[t, j]] - top[j]) <=
-            NEAR_TIE_REL * max(abs(top[j]), 1e-30) for j in range(k))
-        (near if ok else bad).append(int(t))
+        ok = len(set(ids[t].tolist())) == k and all(
+            0 <= ids[t, j] < E and abs(L[t, ids[t, j]] - top[j]) <= tie_band(L[t, ids[t, j]], top[j])
+            for j in range(k))
+        if ok and int(t) not in bad:
+            near.append(int(t))
+        else:
+            bad.add(int(t))
+    bad = sorted(bad)
     return len(bad) == 0, near, bad
 
 
 def near_tie_report(oracle_logits, gpu_ids, k, max_list=32):
-    """Tokens whose oracle logits of ranks k and k+1 (or any two adjacent
-    ranks among the first k+1) lie within the near-tie band, whether or not
-    the GPU's ids differ there: [(token, rank, relative gap)]."""
+    """Tokens with two adjacent logits among the oracle's first k+1 inside
+    the tie band, whether or not the GPU's ids differ there:
+    [(token, rank, gap)], gap the absolute difference of the two logits."""
     L = np.asarray(oracle_logits, np.float64)
     order = oracle_topk_order(L, k)
     top = np.take_along_axis(L, order, axis=1)
     gap = np.abs(top[:, :-1] - top[:, 1:])
     scale = np.maximum(np.abs(top[:, :-1]), np.abs(top[:, 1:]))
-    rel = gap / np.maximum(scale, 1e-30)
-    hits = np.argwhere(rel < NEAR_TIE_REL)
-    return [(int(t), int(r), float(rel[t, r])) for t, r in hits[:max_list]]
+    band = 2.0 * (ROUTER_LOGIT_ATOL + ROUTER_LOGIT_RTOL * scale)
+    hits = np.argwhere(gap < band)
+    return [(int(t), int(r), float(gap[t, r])) for t, r in hits[:max_list]]
 
 
 def parallel_rows(fn, n_rows, chunk, workers=None):

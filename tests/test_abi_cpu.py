@@ -99,11 +99,23 @@ def test_workspace_queries():
 
 
 def test_near_tie_rule():
-    """The routing comparison accepts swaps only inside the tie band."""
-    L = np.array([[3.0, 2.0, 1.0, 0.5], [1.0, 1.0 + 1e-7, 0.2, 0.1]])
-    ok, near, bad = check_routing(L, np.array([[0, 1], [1, 0]]), 2)
+    """The routing comparison accepts swaps only inside the tie band (twice
+    the router-logit tolerance, absolute plus relative), and a token whose
+    ids are not the top-k of the GPU's own logits is a mismatch."""
+    L = np.array([[3.0, 2.0, 1.0, 0.5], [1.0, 1.0 + 1e-7, 0.2, 0.1],
+                  [0.01, 0.01 + 5e-5, -0.3, -0.4], [0.5, 0.5 + 1e-3, 0.1, 0.0]])
+    ok, near, bad = check_routing(L, np.array([[0, 1], [1, 0], [1, 0], [1, 0]]), 2)
     assert ok and near == [] and bad == []
-    ok, near, bad = check_routing(L, np.array([[0, 1], [0, 1]]), 2)
-    assert ok and near == [1]
-    ok, near, bad = check_routing(L, np.array([[1, 0], [1, 0]]), 2)
-    assert not ok and bad == [0]
+    # swaps of logits 1e-7 apart, and of small logits 5e-5 apart (inside the
+    # absolute part of the band), are near ties
+    ok, near, bad = check_routing(L, np.array([[0, 1], [0, 1], [0, 1], [1, 0]]), 2)
+    assert ok and near == [1, 2]
+    # a gap of 1e-3 at 0.5 and a gap of 1 are outside the band
+    ok, near, bad = check_routing(L, np.array([[1, 0], [1, 0], [1, 0], [0, 1]]), 2)
+    assert not ok and bad == [0, 3]
+    # ids that are not the top-k of the GPU's own logits
+    G = L.astype(np.float32)
+    ok, near, bad = check_routing(L, np.array([[0, 1], [0, 1], [1, 0], [1, 0]]), 2, gpu_logits=G)
+    assert not ok and bad == [1]
+    ok, near, bad = check_routing(L, np.array([[0, 1], [1, 0], [1, 0], [1, 0]]), 2, gpu_logits=G)
+    assert ok and bad == []
