@@ -48,16 +48,15 @@ bool decode_supported(const strata_qweights* w) {
   return w->hidden % 256 == 0 && w->inter % 128 == 0 && w->hidden % 64 == 0;
 }
 
-// Decode scratch: h fp16 [P, I], its Z fp32 [P, I/32], then one progress
-// counter per active expert (at most P).
+// Decode scratch: h fp16 [P, I], then one progress counter per active
+// expert (at most P).
 struct DecodeScratch {
-  uint64_t h, z, sync, total;
+  uint64_t h, sync, total;
 };
 DecodeScratch decode_scratch(int P, int I) {
   DecodeScratch d;
   d.h = 0;
-  d.z = up256((uint64_t)P * I * 2);
-  d.sync = d.z + up256((uint64_t)P * (I / 32) * 4);
+  d.sync = up256((uint64_t)P * I * 2);
   d.total = d.sync + up256((uint64_t)P * 4);
   return d;
 }
@@ -94,7 +93,6 @@ int32_t run_experts(const uint16_t* hidden, const strata_qweights* w, const int3
     const DecodeScratch ds = decode_scratch(P, w->inter);
     uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
     a.hbuf = reinterpret_cast<uint16_t*>(wsb + ds.h);
-    a.zdn = reinterpret_cast<float*>(wsb + ds.z);
     a.sync = reinterpret_cast<int32_t*>(wsb + ds.sync);
     a.y = reinterpret_cast<float*>(y);
     a.status = status;
@@ -474,19 +472,18 @@ int32_t moe_layer_forward(const float* x, int32_t T, const uint16_t* w_router, c
 // all free HBM up front (weights plus a cache pool), where a cudaMalloc in the
 // middle of a step would fail and a cudaFree would synchronise the device.
 // The call allocates nothing: no cudaMalloc, cudaFree or allocating library
-// routine.  Its scratch is the fp16 SwiGLU activation h [T*k, I], the
-// offset sums Z of the h rows [T*k, I/32] and the per-expert progress
-// counters of the fused decode kernel.
+// routine.  Its scratch is the fp16 SwiGLU activation h [T*k, I] and the
+// per-expert progress counters of the fused decode kernel.
 //
 // Every call on a device shares the one array, which keeps the last call's
 // contents.  Nothing in it must start at zero: the down tiles read only the
-// h and Z rows that the gate/up tiles of the same call wrote, and each call zeroes
+// h rows that the gate/up tiles of the same call wrote, and each call zeroes
 // its counters before the kernel that uses them.  Calls whose kernels overlap
 // on the GPU (other streams, other host threads) race on the array.
 namespace {
 constexpr uint64_t kStaticMaxPI = 1ull << 20;  // T*k*I <= 1,048,576
-// h fp16 (2 MiB) + its Z (128 KiB) + T*k <= 512 counters, each part padded
-constexpr uint64_t kStaticScratchBytes = kStaticMaxPI * 2 + kStaticMaxPI / 8 + 256 + 4096;
+// h fp16 (2 MiB) + T*k <= 512 counters, each part padded
+constexpr uint64_t kStaticScratchBytes = kStaticMaxPI * 2 + 256 + 4096;
 }  // namespace
 
 static __device__ __align__(256) uint8_t g_experts_static_scratch[kStaticScratchBytes];

@@ -97,11 +97,6 @@ STRATA_DEVFN void fence_barrier_init() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-STRATA_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
 
 STRATA_DEVFN bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -130,14 +125,6 @@ STRATA_DEVFN bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// 1-D bulk copy global -> this CTA's shared memory; completion is counted on
-// `bar` in bytes.  dst, src and bytes must be multiples of 16.
-STRATA_DEVFN void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(smem_addr(dst)), "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
 
 // ldmatrix x4, transposed (four 8x8 b16 tiles).
 STRATA_DEVFN void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {

@@ -75,4 +75,17 @@ STRATA_HD inline int tc_deal_down_tile(const TcDeal& d, const int* bcnt, int cta
   return d.ntB - 1 - jp;
 }
 
+// The same index from per-round counts, without a pass over the grid:
+// gt_all[k] = CTAs with more than k down tiles and gt_below[k] = those of
+// them below `cta`, for k below this CTA's count bc.  Every round before k2
+// contributes its CTAs' tiles (sum over k < k2 of gt_all[k] = sum over CTAs
+// of min(b, k2)), then round k2 the CTAs below this one.
+STRATA_HD inline int tc_deal_down_tile_counted(const TcDeal& d, const int* gt_all,
+                                               const int* gt_below, int bc, int kk) {
+  const int k2 = bc - 1 - kk;
+  int jp = gt_below[k2];
+  for (int k = 0; k < k2; ++k) jp += gt_all[k];
+  return d.ntB - 1 - jp;
+}
+
 }  // namespace strata

@@ -17,7 +17,6 @@ struct DecodeArgs {
   const int32_t* active;
   int shared_mode;
   uint16_t* hbuf;  // scratch fp16 [rows, I]
-  float* zdn;      // scratch fp32 [rows, I/32]: Z of each h row and 32-block
   float* y;        // [rows, H]
   int32_t* status;
   int32_t* sync;   // scratch: one counter per active expert (Umax ints), or nullptr

@@ -108,13 +108,62 @@ STRATA_DEVFN void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
       : "memory");
 }
 
-// 3-D tiled load (c0 innermost), no multicast.
-STRATA_DEVFN void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
-                              uint64_t* bar) {
+// Warp-converged forms of the copy issue: every lane of a converged warp
+// executes the statement and elect.sync picks the one lane that issues, so
+// the warp-uniform operands stay in uniform registers (a lone thread in a
+// divergent branch pays a register move per operand per instruction).  The
+// stage forms arrive on the barrier with the expected bytes and issue the
+// copy in the same statement.
+// One 4-D box at (x, y, w, z).
+STRATA_DEVFN void tma_stage1_4d_warp(uint64_t* bar, uint32_t tx, void* d, const CUtensorMap* m,
+                                     int x, int y, int w, int z) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t"
+      "@e cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%2], [%3, {%4, %5, %6, %7}], [%0];\n\t}" ::"r"(smem_addr(bar)),
+      "r"(tx), "r"(smem_addr(d)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(w),
+      "r"(z)
+      : "memory");
+}
+// One 3-D box at (x, y, z).
+STRATA_DEVFN void tma_stage1_3d_warp(uint64_t* bar, uint32_t tx, void* d, const CUtensorMap* m,
+                                     int x, int y, int z) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t"
+      "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%2], [%3, {%4, %5, %6}], [%0];\n\t}" ::"r"(smem_addr(bar)),
+      "r"(tx), "r"(smem_addr(d)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+STRATA_DEVFN void tma_load_2d_warp(void* dst, const CUtensorMap* map, int c0, int c1,
+                                   uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3}], [%4];\n\t}" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
+      : "memory");
+}
+STRATA_DEVFN void mbar_arrive_expect_tx_warp(uint64_t* bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
+      "r"(bytes)
+      : "memory");
+}
+STRATA_DEVFN void bulk_g2s_warp(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+      "[%3];\n\t}" ::"r"(smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
       : "memory");
 }
 
@@ -155,92 +204,20 @@ STRATA_DEVFN void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 STRATA_DEVFN void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 lanes x 32 bits, 4 / 8 consecutive columns per thread.
-STRATA_DEVFN void tmem_ld4(uint32_t taddr, uint32_t (&r)[4]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(taddr));
-}
-STRATA_DEVFN void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
-                 "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr));
-}
 
-// Loads and their wait in ONE asm statement: the values exist for the
-// compiler only once tcgen05.wait::ld has completed, so no copy or spill of a
-// destination register can read it early.  Four loads of 4 (or 8) columns at
-// a0..a3, or two loads of 16 columns at a0, a1.
-STRATA_DEVFN void tmem_ld4x4_wait(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                  uint32_t (&r)[16]) {
+
+STRATA_DEVFN void tmem_ld16_wait(uint32_t a0, uint32_t (&r)[16]) {
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%16];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%4,%5,%6,%7}, [%17];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%8,%9,%10,%11}, [%18];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x4.b32 {%12,%13,%14,%15}, [%19];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
       "tcgen05.wait::ld.sync.aligned;"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
         "=r"(r[14]), "=r"(r[15])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3)
-      : "memory");
-}
-STRATA_DEVFN void tmem_ld8x4_wait(uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                  uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%32];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8,%9,%10,%11,%12,%13,%14,%15}, [%33];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16,%17,%18,%19,%20,%21,%22,%23}, [%34];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24,%25,%26,%27,%28,%29,%30,%31}, [%35];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3)
-      : "memory");
-}
-STRATA_DEVFN void tmem_ld16x2_wait(uint32_t a0, uint32_t a1, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%32];\n\t"
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%33];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(a0), "r"(a1)
+      : "r"(a0)
       : "memory");
 }
 
-// Ties a register to the point after a tcgen05.wait::ld: the compiler keeps
-// volatile asm in order, and every use of x depends on this one.
-STRATA_DEVFN void reg_after_wait(uint32_t& x) { asm volatile("" : "+r"(x)); }
-
-// 32 lanes x 32 bits, one column per thread (thread i of the warp reads lane
-// base + i).  The column may differ between calls (a runtime address).
-STRATA_DEVFN uint32_t tmem_ld1(uint32_t taddr) {
-  uint32_t r;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-  return r;
-}
-
-// Register -> tensor memory: 32 lanes x 32 bits, N consecutive columns per
-// thread (thread i of the warp writes lane base + i).
-STRATA_DEVFN void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
-}
 STRATA_DEVFN void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -300,29 +277,66 @@ STRATA_DEVFN void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, ui
       : "memory");
 }
 
-// Same with the A operand (128 rows x 16 K, two fp16 per 32-bit column, row
-// m in lane m) read from tensor memory at a_tmem, and the B descriptor given
-// as its two 32-bit words, joined into the 64-bit operand inside the asm
-// statement: the compiler then does no 64-bit arithmetic on a descriptor.
-// (A build that added offsets to a 64-bit descriptor in C++ handed some of
-// these MMAs a descriptor whose high word was lost: B was then read as an
-// unswizzled layout with 16-byte rows.)
-STRATA_DEVFN void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
-                             uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
-      "setp.ne.b32 p, %5, 0;\n\t"
-      "mov.b64 bd, {%2, %3};\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
+
 
 // Arrive on `bar` once all previously issued tcgen05 operations of this
 // thread have completed.
 STRATA_DEVFN void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
+// One 128-K half of a decode tile, issued by a whole converged warp with a
+// single elect.sync: eight K16 MMAs (kind::f16, A from tensor memory) into
+// the 16 columns at d_tmem, where step kk reads A at a_tmem + 8 kk and B at
+// b_lo + (kk / 4) ATOM + (kk % 4) * 2 (16-byte units; ATOM = one 64-K atom
+// of B).  The first step accumulates iff `accumulate` is nonzero, the other
+// seven always.  One asm statement keeps the per-MMA work to three adds in
+// the issuing lane.
+template <int ATOM>
+STRATA_DEVFN void mma_half_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                                   uint32_t idesc, uint32_t accumulate) {
+  static_assert(ATOM == 64 || ATOM == 128, "B atom of 8 or 16 rows");
+#define STRATA_MMA_STEP(AOFF, BOFF, ACC)                                          \
+  "add.u32 a, %1, " #AOFF ";\n\t"                                               \
+  "add.u32 b, %2, " #BOFF ";\n\t"                                               \
+  "mov.b64 bd, {b, %3};\n\t"                                                    \
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], bd, %4, " ACC ";\n\t"
+  if constexpr (ATOM == 128) {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b32 a, b;\n\t.reg .b64 bd;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        STRATA_MMA_STEP(0, 0, "p") STRATA_MMA_STEP(8, 2, "1")
+        STRATA_MMA_STEP(16, 4, "1") STRATA_MMA_STEP(24, 6, "1")
+        STRATA_MMA_STEP(32, 128, "1") STRATA_MMA_STEP(40, 130, "1")
+        STRATA_MMA_STEP(48, 132, "1") STRATA_MMA_STEP(56, 134, "1")
+        "}" ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred e, p;\n\t.reg .b32 a, b;\n\t.reg .b64 bd;\n\t"
+        "setp.ne.b32 p, %5, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        STRATA_MMA_STEP(0, 0, "p") STRATA_MMA_STEP(8, 2, "1")
+        STRATA_MMA_STEP(16, 4, "1") STRATA_MMA_STEP(24, 6, "1")
+        STRATA_MMA_STEP(32, 64, "1") STRATA_MMA_STEP(40, 66, "1")
+        STRATA_MMA_STEP(48, 68, "1") STRATA_MMA_STEP(56, 70, "1")
+        "}" ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
+        : "memory");
+  }
+#undef STRATA_MMA_STEP
+}
+
+// mma_commit executed by a whole converged warp (one elected lane commits;
+// it tracks the MMAs that the same elected lane issued).
+STRATA_DEVFN void mma_commit_warp(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
           smem_addr(bar))
       : "memory");
 }

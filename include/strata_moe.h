@@ -247,9 +247,8 @@ STRATA_API int32_t moe_experts(const uint16_t* hidden, const strata_qweights* w,
  * HBM (weights plus a cache pool), where a cudaMalloc during a step would fail
  * and a cudaFree would synchronise the device.  The call allocates nothing (no
  * cudaMalloc, cudaFree or allocating library routine); its scratch, the fp16
- * activations h [T*k, I] (up to 2 MiB), their fp32 offset sums [T*k, I/32]
- * (up to 128 KiB) and T*k progress counters, lives in one file-scope array of
- * the library.
+ * activations h [T*k, I] (up to 2 MiB) and T*k progress counters, lives in one
+ * file-scope array of the library.
  *   Limit: T <= STRATA_DECODE_MAX_T and T*k*I <= 1,048,576 (2 MiB of fp16);
  *   beyond it the call returns STRATA_EUNSUPPORTED and launches nothing.
  *   Set-up: the first call on each device, with that device current, looks

@@ -4,7 +4,8 @@
 // end at the tile count, every CTA outside the clamped range carries the mean
 // weighted work within one down tile (inside it, none gets a down tile), and
 // no CTA gets more tiles than the
-// table capacity computed for any larger expert count.  Prints "ok <cases>" or the first
+// table capacity computed for any larger expert count, and the per-round-count
+// form of the down-tile index agrees with the direct one.  Prints "ok <cases>" or the first
 // failure, and exits non-zero on a failure.
 #include <cstdio>
 #include <vector>
@@ -30,6 +31,13 @@ static int check(int G, int U, int Umax, int H, int I) {
     }
     bc[c] = bs[c + 1] - bs[c];
   }
+  // per-round counts as the kernel builds them: CTAs with more than k down
+  // tiles, in all and below the current CTA (kept up to date as c grows)
+  int bmax = 0;
+  for (int c = 0; c < G; ++c) bmax = bc[c] > bmax ? bc[c] : bmax;
+  std::vector<int> gt_all(bmax + 1, 0), gt_below(bmax + 1, 0);
+  for (int c = 0; c < G; ++c)
+    for (int k = 0; k < bc[c]; ++k) ++gt_all[k];
   // balance: where F >= 0 at both ends of CTA c's range (no clamp), its
   // weighted work is within one down tile of Tot / G; where F(c+1) < 0 (the
   // CTAs up to c already carry more than their share) it has no down tile
@@ -62,7 +70,13 @@ static int check(int G, int U, int Umax, int H, int I) {
         std::printf("FAIL tile G=%d U=%d c=%d kk=%d j=%d\n", G, U, c, kk, j);
         return 1;
       }
+      const int j2 = tc_deal_down_tile_counted(d, gt_all.data(), gt_below.data(), bc[c], kk);
+      if (j2 != j) {
+        std::printf("FAIL counted G=%d U=%d c=%d kk=%d: %d vs %d\n", G, U, c, kk, j2, j);
+        return 1;
+      }
     }
+    for (int k = 0; k < bc[c]; ++k) ++gt_below[k];
   }
   return 0;
 }
