@@ -344,39 +344,40 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
       }
     }
   } else {
-    // ------------------------------------------------ MMA issue (one thread)
-    if (elect_one()) {
-      int it_k = 0, it = 0;
-      for (int u = blockIdx.x; u < total; u += gridDim.x, ++it) {
-        const NTile tl = tiles[u / MT];
-        const int n16 = (tl.n + 15) & ~15;
-        const uint32_t idesc = idesc_f16_f32(n16);
-        const int a = it & 1;
-        mbar_wait_guarded(&tempty[a], ((it >> 1) & 1) ^ 1, status, abort_flag);
+    // ------------------------------------------------ MMA issue: the whole
+    // warp runs the loop (converged); one elected lane issues each stage's
+    // MMAs in one asm statement, with warp-uniform operands
+    static_assert(kTileBytes / 16 == 1024, "second A tile 1024 descriptor units on");
+    static_assert(kPK == 64, "four K16 steps per stage");
+    const uint32_t tbase = __shfl_sync(0xffffffffu, tmem_base, 0);
+    const uint32_t dhi = smem_desc_k128_hi(1024);
+    const uint32_t smem0 = __shfl_sync(0xffffffffu, smem_addr(smem), 0);
+    int it_k = 0, it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total && ok; u += gridDim.x, ++it) {
+      const NTile tl = tiles[u / MT];
+      const int n16 = (tl.n + 15) & ~15;
+      const uint32_t idesc = idesc_f16_f32(n16);
+      const int a = it & 1;
+      ok = mbar_wait_guarded(&tempty[a], ((it >> 1) & 1) ^ 1, status, abort_flag);
+      const uint32_t d0 = tbase + a * kAccCols;
+      for (int kc = 0; kc < KC && ok; ++kc, ++it_k) {
+        const int s = it_k % C::S;
+        ok = mbar_wait_guarded(&full[s], (it_k / C::S) & 1, status, abort_flag);
+        __syncwarp();
         tc_fence_after();
-        const uint32_t d0 = tmem_base + a * kAccCols;
-        for (int kc = 0; kc < KC; ++kc, ++it_k) {
-          const int s = it_k % C::S;
-          mbar_wait_guarded(&full[s], (it_k / C::S) & 1, status, abort_flag);
-          tc_fence_after();
-          const uint32_t st = smem_addr(smem + s * C::SB);
-          const uint32_t bb = st + C::NA * kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < kPK / 16; ++kk) {
-            const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
-            const uint64_t bdesc = smem_desc_k128(bb + kk * 32);
-            mma_f16_ss(d0, smem_desc_k128(st + kk * 32), bdesc, idesc, acc);
-            if constexpr (MODE == 0)
-              mma_f16_ss(d0 + 128, smem_desc_k128(st + kTileBytes + kk * 32), bdesc, idesc, acc);
-          }
-          mma_commit(&empty[s]);
-        }
-        mma_commit(&tfull[a]);
+        const uint32_t st = smem0 + (uint32_t)(s * C::SB);
+        mma_stage_ss_warp<MODE == 0>(d0, smem_desc_k128_lo(st),
+                                     smem_desc_k128_lo(st + C::NA * kTileBytes), dhi, idesc,
+                                     (uint32_t)(kc > 0));
+        mma_commit_warp(&empty[s]);
       }
-      mma_commit(done);
-      // all MMAs retired before the tensor memory is released (bounded)
-      mbar_wait_bounded(done, 0, status);
+      mma_commit_warp(&tfull[a]);
     }
+    __syncwarp();
+    mma_commit_warp(done);
+    // all MMAs retired before the tensor memory is released (bounded)
+    mbar_wait_bounded(done, 0, status);
     __syncwarp();
   }
   tc_fence_before();
