@@ -2,60 +2,57 @@
 // (T <= STRATA_DECODE_MAX_T) on the 5th-generation tensor cores.
 //
 // With at most 16 tokens per call the expert FFN is bound by streaming the
-// quantised weights out of HBM and turning them into tensor-core operands,
-// not by multiply-adds.  Every weight row is decoded by one thread straight
-// into that row's lane of tensor memory (tcgen05.st): a 2-bit code c becomes
-// d (c - 1.5) and a 4-bit code d KV[c] in fp16 (an exact integer-to-fp16
-// step, then one multiply by the block scale d that rounds once).  The MMA
-// reads A (128 rows x 16 K) from tensor memory and B (the tokens, N = 16)
-// from shared memory, and accumulates a whole tile (all of K) into one
-// 16-column fp32 accumulator, which the tile-end warps read directly.  The
-// decoders therefore never wait for an MMA result: a half chunk is decoded
-// as soon as its tensor-memory stage has been read by the MMA before.
+// quantised weights out of HBM and decoding them, not by multiply-adds.  So
+// every weight row is decoded by exactly one thread, straight into that row's
+// lane of tensor memory (tcgen05.st), and the MMA reads its A operand
+// (128 weight rows x 16 K, fp16) from tensor memory; B is the token block
+// (N = 16 columns, fp16, in shared memory).  Decoded weights never pass
+// through shared memory, whose bandwidth would otherwise cap the path.  Codes
+// and scales arrive by TMA into a ring of shared-memory stages.
 //
 // Two kinds of tile:
-//   gate/up  64 rows of I: lanes 0-63 the gate rows, lanes 64-127 the same up
-//            rows.  B = every token of the call; the tile end keeps the
-//            columns of the tokens routed to the tile's expert, exchanges gate
-//            and up through shared memory, and writes h = SwiGLU fp16 [P, I]
-//            in sorted pair order (K permuted within 16-groups the way the
-//            down tiles' decode orders K).
-//   down     128 rows of H of one expert.  B = that expert's h rows (TMA);
-//            y fp32 [P, H] in sorted order.
+//   gate/up  64 rows of I: lanes 0-63 decode the gate rows, lanes 64-127 the
+//            same up rows.  B = every token of the call, so a tile computes
+//            all T columns and the epilogue keeps the tokens routed to the
+//            tile's expert: h = SwiGLU(gate, up) -> fp16 [P, I] in sorted pair
+//            order, K permuted within 16-groups the way the down tiles'
+//            decode orders K.
+//   down     128 rows of H of one expert.  B = that expert's h rows (TMA from
+//            h); y fp32 [P, H] in sorted order.
 // and three kernel forms (MODE):
 //   2  fused: one launch runs both kinds.  Each CTA takes its gate/up tiles
 //      round robin, then a share of the down tiles chosen so that every CTA
-//      has about the same weighted work (deal.h).  A down tile's h block is
-//      loaded once its expert's gate/up tiles are all done: each gate/up
-//      tile end publishes its h rows and then counts itself in a per-expert
-//      counter (release); the producer polls it (acquire, bounded) before
-//      the TMA.  The counters are zeroed by a one-thread-block kernel
+//      has about the same weighted work (a gate/up tile costs H, a down tile
+//      I plus a fixed overhead, in 64-column units).  Down tiles are dealt in
+//      rounds counted back from each CTA's last tile, from the end of the
+//      expert order: the experts whose gate/up tiles finish last become the
+//      last tile of many CTAs rather than all tiles of a few, and the extra
+//      down tiles of CTAs with fewer gate/up tiles come from the experts that
+//      are ready first.  A down
+//      tile's h block is loaded once its expert's gate/up tiles are all done:
+//      each gate/up epilogue publishes its h rows and then counts itself in a
+//      per-expert counter (release); the producer polls it (acquire, bounded)
+//      before the TMA.  The counters are zeroed by a one-thread-block kernel
 //      launched just before, so the workspace needs no initial contents.
 //   0, 1  gate/up alone, then down alone (chained by programmatic dependent
 //      launch): used when the fused form's shared memory leaves too few
 //      stages.
 // Every CTA of a fused grid is resident at once (one per SM, grid <= SMs),
 // and a CTA's gate/up tiles depend on nothing outside it, so the waits on the
-// counters end while the kernel has the GPU to itself; they are bounded all
-// the same.
+// counters always end; they are bounded all the same.
 //
 // One persistent CTA per SM with a static tile list.  Warps:
-//   0-3   tile ends: tcgen05.ld of the tile's accumulator, then the SwiGLU /
-//         h / y stores.  They also build the tile table.
-//   4-15  decoders: three groups of four warps taking chunks (128 bytes of
-//         codes per row) in turn; a thread owns one tile row (= TMEM lane),
-//         reads its codes from the swizzled stage (conflict-free) and stores
-//         the decoded 128-K pieces into its group's two tensor-memory stages
-//         in turn
-//   16    the TMA producer (codes; the tile's block scales; down: the h block)
-//   17    tensor-memory allocation and the MMA issue: the whole warp runs the
-//         issue loop, one elected lane issues (one asm statement per stage)
-// Tensor memory: six A stages of 64 columns (128 K of fp16 x 128 rows), two
-// per decoder group, then two 16-column accumulators (tiles alternate).
-// Barriers: full/empty (smem stages), afull/afree (A stage stored / read by
-// its MMAs), accfull/accfree (a tile's accumulator complete / read),
-// sfull/sempty and bfull/bempty (down: per-tile scales, per-expert h block).
-// Every wait is bounded.
+//   0-3   epilogue: tcgen05.ld of their TMEM lane quarter (and the tile table)
+//   4..   decoders: kTcGroups groups of four warps taking K chunks in turn;
+//         a thread owns one tile row (= TMEM lane), reads its codes from
+//         the swizzled stage (conflict-free), decodes to fp16 and stores them
+//         into the A stage in tensor memory
+//   then  the TMA producer warp (codes, scales; down: the tile's scales and
+//         h blocks) and the warp that allocates tensor memory and issues
+//         the MMAs (one thread)
+// Barriers: full/empty (smem stages), tfull/tempty (TMEM A stages),
+// afull/aempty (two accumulators), sfull/sempty and bfull/bempty (down:
+// per-tile scales, per-expert h block).  Every wait is bounded.
 #include <algorithm>
 
 #include "deal.h"
@@ -65,27 +62,23 @@
 
 namespace strata {
 
-constexpr int kTcGroups = 3;                          // decoder groups (4 warps each)
-constexpr int kTcDecWarp0 = 4;
-constexpr int kTcProdWarp = kTcDecWarp0 + 4 * kTcGroups;  // TMA producer warp
-constexpr int kTcMmaWarp = kTcProdWarp + 1;               // TMEM allocation + MMA warp
+constexpr int kTcGroups = 3;                      // decoder groups (4 warps each)
+constexpr int kTcProdWarp = 4 + 4 * kTcGroups;     // TMA producer warp
+constexpr int kTcMmaWarp = kTcProdWarp + 1;        // TMEM allocation + MMA warp
 constexpr int kTcWarps = kTcMmaWarp + 1;
 constexpr int kTcThreads = kTcWarps * 32;
-// A shared-memory stage holds 128 bytes of codes per row for 128 rows (the
-// TMA moves whole 128-byte rows: shorter box rows cost the same per row):
-// 512 K of 2-bit or 256 K of 4-bit codes.  A tensor-memory stage holds 128 K.
-constexpr int kTcCBR = 128;     // code bytes per row per chunk
-constexpr int kTcKH = 128;      // K per tensor-memory stage
-constexpr int kTcSPG = 2;       // tensor-memory A stages per decoder group
-constexpr int kTcTS = kTcSPG * kTcGroups;
-constexpr int kTcStageCols = 64;      // A: 128 K of fp16 per lane
-constexpr int kTcAccCol0 = kTcTS * kTcStageCols;  // two 16-column accumulators
+constexpr int kTcKC = 256;        // K per chunk (one smem stage / one TMEM A stage)
+constexpr int kTcTS = 3;          // TMEM A stages
+constexpr int kTcACol0 = 64;      // A stage t at columns 64 + 128 t (accumulators at 0, 32)
 constexpr int kTcTmemCols = 512;
 constexpr int kTcMaxStages = 16;
 constexpr int kTcSmemBudget = 227 * 1024;
-constexpr int kTcFusedMinStages = 6;  // fewer: run the two-kernel form
-constexpr int kTcMaxGrid = 1024;      // grids the fused tile dealing is checked for
-static_assert(kTcAccCol0 + 2 * 16 <= kTcTmemCols, "tensor memory stages fit");
+constexpr int kTcFusedMinStages = 9;  // fewer: run the two-kernel form
+constexpr int kTcMaxGrid = 1024;      // the fused tile dealing keeps one int per CTA
+// Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
+// only after the MMAs of its previous one retired, so with at least as many
+// stages as groups no waiter runs two phases ahead of a stage's barrier.
+static_assert(kTcTS >= kTcGroups, "TMEM A stages must cover the decoder groups");
 
 struct TcParams {
   const uint16_t* hidden;
@@ -101,9 +94,8 @@ struct TcParams {
   int32_t* status;
   int32_t* sync;   // fused form: finished gate/up tiles per active expert (zeroed)
   int S;           // shared-memory stages (a multiple of kTcGroups)
+  int NB;          // B rows: 8 (T <= 8; rows 8-15 of the MMA repeat them) or 16
   int maxT;        // capacity of the tile table: tiles per CTA at most
-  int hbn;         // h block buffers (2, or 1 where two leave too few stages)
-  int sbn;         // per-tile scale buffers (2, or 1 where two leave too few stages)
 };
 
 struct TcTile {
@@ -111,9 +103,9 @@ struct TcTile {
   int tok[16];          // gate/up: token of each of the expert's pairs
 };
 
-// K per shared-memory chunk: 128 bytes of codes per row
-__host__ __device__ constexpr int tc_kc(int fmt) {
-  return fmt == STRATA_FMT_Q2_32 ? kTcCBR * 4 : kTcCBR * 2;
+template <int FMT>
+__host__ __device__ constexpr int tc_cbr() {  // code bytes per row per chunk
+  return FMT == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
 }
 
 struct TcLayout {
@@ -122,42 +114,66 @@ struct TcLayout {
 };
 
 __host__ __device__ inline uint32_t up1k(uint32_t x) { return (x + 1023u) & ~1023u; }
-__host__ __device__ inline uint32_t up128(uint32_t x) { return (x + 127u) & ~127u; }
 
 // Shared memory, from a 1024-byte aligned base: S stages | gate/up: the token
-// block | down: one or two h blocks | one or two per-tile scale blocks | gate/up:
-// the SwiGLU exchange buffer (also the fused form's dealing counts) | the
-// tile table | barriers.  Every TMA destination is 1024-byte aligned, every
-// bulk-copy destination 128-byte aligned.
+// block | down: two h blocks | down: two per-tile scale blocks | gate/up: the
+// SwiGLU exchange buffer (also the fused form's dealing scratch) | the tile
+// table | barriers.  Every TMA destination is 1024-byte aligned.
 __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, int I, int S,
-                                              int maxT, int hbn, int sbn) {
+                                              int maxT) {
   TcLayout L;
   const bool gu = mode != 1, dn = mode != 0;
-  L.codes_bytes = 128u * kTcCBR;
-  L.stage_bytes = L.codes_bytes;
+  const uint32_t cbr = fmt == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
+  L.codes_bytes = 128u * cbr;
+  L.stage_bytes = L.codes_bytes + (gu ? 128u * 16u : 0u);
   uint32_t off = (uint32_t)S * L.stage_bytes;
   L.b = off;
   L.b_bytes = gu ? (uint32_t)NB * (uint32_t)H * 2u : 0u;
-  off = up1k(off + L.b_bytes);
+  off += L.b_bytes;
   L.hb = off;
   L.hb_bytes = dn ? (uint32_t)NB * (uint32_t)I * 2u : 0u;
-  off += (uint32_t)hbn * L.hb_bytes;
+  off += 2u * L.hb_bytes;
   L.sbuf = off;
-  // one tile's block scales (fp16, every K block): gate/up 128 rows x H/32,
-  // down 128 rows x I/32
-  L.s_bytes = up128(std::max(gu ? 8u * (uint32_t)H : 0u, dn ? 8u * (uint32_t)I : 0u));
-  off += (uint32_t)sbn * L.s_bytes;
+  L.s_bytes = dn ? up1k(8u * (uint32_t)I) : 0u;
+  off += 2u * L.s_bytes;
   L.xch = off;
-  off += gu ? up128(std::max(64u * 17u * 4u, 8u * (uint32_t)maxT)) : 0u;
+  off += gu ? up1k(2u * 64u * 17u * 4u) : 0u;
   L.tbl = off;
-  off += up128((uint32_t)sizeof(TcTile) * (uint32_t)maxT);
+  off += up1k((uint32_t)sizeof(TcTile) * (uint32_t)maxT);
   L.bars = off;
   off += 1024u;
   L.total = off;
   return L;
 }
+static_assert(2 * 64 * 17 * 4 >= 4 * kTcMaxGrid, "dealing scratch fits the exchange buffer");
 
 // ---------------------------------------------------------------- decode
+// One Q2 word (16 codes, element j at bits 2j) -> R[i] = fp16x2 (element i,
+// element i + 8) * d.  A code placed at mantissa bit p of an fp16 whose
+// exponent gives that bit unit weight is M_p + c exactly (M_p = 2^(10-p));
+// subtracting M_p + 1.5 leaves c - 1.5 exactly; the multiply by the block
+// scale rounds once.
+STRATA_DEVFN void dq_q2_word(uint32_t w, uint32_t d2, uint32_t* R) {
+  const uint32_t wl = w << 2, wr = w >> 8;
+  const uint32_t src[8] = {wl, w, w, w, w, wr, wr, wr};
+  const uint32_t msk[8] = {0x000C000Cu, 0x000C000Cu, 0x00300030u, 0x00C000C0u,
+                           0x03000300u, 0x000C000Cu, 0x00300030u, 0x00C000C0u};
+  const uint32_t mag[8] = {0x5C005C00u, 0x5C005C00u, 0x54005400u, 0x4C004C00u,
+                           0x44004400u, 0x5C005C00u, 0x54005400u, 0x4C004C00u};
+  const uint32_t sub[8] = {0x5C065C06u, 0x5C065C06u, 0x54185418u, 0x4C604C60u,
+                           0x45804580u, 0x5C065C06u, 0x54185418u, 0x4C604C60u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t v, t;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(v) : "r"(src[i]), "r"(msk[i]), "r"(mag[i]));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(t) : "r"(v), "r"(sub[i]));
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(R[i]) : "r"(t), "r"(d2));
+  }
+}
+
+STRATA_DEVFN uint32_t dup_lo(uint32_t x) { return __byte_perm(x, 0, 0x1010); }
+STRATA_DEVFN uint32_t dup_hi(uint32_t x) { return __byte_perm(x, 0, 0x3232); }
+
 STRATA_DEVFN uint4 lds128(const void* p) {
   uint4 v;
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
@@ -171,91 +187,80 @@ STRATA_DEVFN uint2 lds64(const void* p) {
   return v;
 }
 
-// Block scale (the lo or hi fp16 of a scale word) broadcast to both halves.
-STRATA_DEVFN __half2 scale2(uint32_t w, int hi) {
-  const uint16_t d = (uint16_t)(hi ? (w >> 16) : (w & 0xffffu));
-  return u32_as_h2((uint32_t)d * 0x00010001u);
-}
-
 // Gate/up B operand: token rows n < T of hidden (bf16 -> fp16, exact in the
 // normal range), rows T..NB-1 zero, K permuted within each 16-group like the
 // decoded codes, in the 128-byte-swizzled K-major layout (atoms of 64 K x NB
 // rows, 128 bytes per row, 16-byte piece c of row n at c ^ (n & 7)).  Thread
-// `tid` of `nthr` fills the (row, 32-block) items tid, tid + nthr, ...; each
-// batch issues all of its loads before any conversion, so the fill costs a
-// few L2 round trips.
+// `tid` of `nthr` fills items tid, tid + nthr, ...; each batch issues all of
+// its loads before any conversion, so the fill costs a few L2 round trips.
 template <int FMT>
 STRATA_DEVFN void fill_tokens(uint8_t* bsm, const uint16_t* __restrict__ hidden, int T, int H,
                               int NB, int tid, int nthr) {
-  constexpr int kBatch = 2;
-  const int nb = H / 32, total = NB * nb;
+  constexpr int kBatch = 4;
+  const int ng = H / 16, total = NB * ng;
   for (int i0 = tid; i0 < total; i0 += kBatch * nthr) {
-    uint4 a[kBatch][4];
+    uint4 a[kBatch], b[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int idx = i0 + u * nthr;
-      const int n = idx / nb, b = idx - n * nb;
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        a[u][v] = make_uint4(0, 0, 0, 0);
-        if (idx < total && n < T)
-          a[u][v] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 32 * b + 8 * v);
+      const int n = idx / ng, g = idx - n * ng;
+      a[u] = b[u] = make_uint4(0, 0, 0, 0);
+      if (idx < total && n < T) {
+        a[u] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 16 * g);
+        b[u] = *reinterpret_cast<const uint4*>(hidden + (size_t)n * H + 16 * g + 8);
       }
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int idx = i0 + u * nthr;
       if (idx >= total) break;
-      const int n = idx / nb, b = idx - n * nb;
+      const int n = idx / ng, g = idx - n * ng;
+      const uint32_t w[8] = {a[u].x, a[u].y, a[u].z, a[u].w, b[u].x, b[u].y, b[u].z, b[u].w};
+      uint16_t e[16];
 #pragma unroll
-      for (int gg = 0; gg < 2; ++gg) {  // the block's two 16-groups
-        const uint32_t w[8] = {a[u][2 * gg].x, a[u][2 * gg].y, a[u][2 * gg].z, a[u][2 * gg].w,
-                               a[u][2 * gg + 1].x, a[u][2 * gg + 1].y, a[u][2 * gg + 1].z,
-                               a[u][2 * gg + 1].w};
-        uint16_t e[16];
-#pragma unroll
-        for (int kk = 0; kk < 16; ++kk) {
-          const uint16_t bf = (uint16_t)((kk & 1) ? (w[kk >> 1] >> 16) : (w[kk >> 1] & 0xffffu));
-          e[group_slot<FMT>(kk)] = bf16_to_f16_bits(bf);
-        }
-        uint32_t o[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) o[j] = (uint32_t)e[2 * j] | ((uint32_t)e[2 * j + 1] << 16);
-        const int g = 2 * b + gg;  // 16-group index along K
-        const int pc = (g & 3) * 2;
-        uint8_t* row = bsm + (size_t)(g >> 2) * (NB * 128) + n * 128;
-        *reinterpret_cast<uint4*>(row + ((pc ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-        *reinterpret_cast<uint4*>(row + (((pc + 1) ^ (n & 7)) << 4)) =
-            make_uint4(o[4], o[5], o[6], o[7]);
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint16_t bf = (uint16_t)((kk & 1) ? (w[kk >> 1] >> 16) : (w[kk >> 1] & 0xffffu));
+        e[group_slot<FMT>(kk)] = bf16_to_f16_bits(bf);
       }
+      uint32_t o[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) o[j] = (uint32_t)e[2 * j] | ((uint32_t)e[2 * j + 1] << 16);
+      const int pc = (g & 3) * 2;
+      uint8_t* row = bsm + (size_t)(g >> 2) * (NB * 128) + n * 128;
+      *reinterpret_cast<uint4*>(row + ((pc ^ (n & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+      *reinterpret_cast<uint4*>(row + (((pc + 1) ^ (n & 7)) << 4)) =
+          make_uint4(o[4], o[5], o[6], o[7]);
     }
   }
 }
 
+
 // ---------------------------------------------------------------- kernel
-template <int MODE, int FMT, int NB>
+template <int MODE, int FMT>
 __global__ void __launch_bounds__(kTcThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes (4-D)
+decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
+                 const __grid_constant__ CUtensorMap mu,   // up codes
+                 const __grid_constant__ CUtensorMap msg,  // gate scales
+                 const __grid_constant__ CUtensorMap msu,  // up scales
                  const __grid_constant__ CUtensorMap md,   // down codes
                  const __grid_constant__ CUtensorMap mh,   // h [P, I]
                  const TcParams p) {
   constexpr bool kGU = MODE != 1, kDN = MODE != 0;
-  constexpr int KC = tc_kc(FMT);                                 // K per chunk
+  constexpr int CBR = tc_cbr<FMT>();
   constexpr int PIECE_K = (FMT == STRATA_FMT_Q2_32) ? 64 : 32;  // K per 16-byte code piece
-  constexpr int NPH = kTcKH / PIECE_K;                           // pieces per stage
-  constexpr int TP = NB;  // token columns of B (pairs of a down tile) at most
+  constexpr int NPC = CBR / 16;                                  // pieces per full chunk
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const TcLayout L = tc_layout(MODE, FMT, NB, p.H, p.I, p.S, p.maxT, p.hbn, p.sbn);
+  const TcLayout L = tc_layout(MODE, FMT, p.NB, p.H, p.I, p.S, p.maxT);
   const int S = p.S;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* empty = full + kTcMaxStages;
-  uint64_t* afull = empty + kTcMaxStages;
-  uint64_t* afree = afull + kTcTS;
-  uint64_t* accfull = afree + kTcTS;
-  uint64_t* accfree = accfull + 2;
-  uint64_t* sfull = accfree + 2;
+  uint64_t* tfull = empty + kTcMaxStages;
+  uint64_t* tempty = tfull + kTcTS;
+  uint64_t* afull = tempty + kTcTS;
+  uint64_t* aempty = afull + 2;
+  uint64_t* sfull = aempty + 2;
   uint64_t* sempty = sfull + 2;
   uint64_t* bfull = sempty + 2;
   uint64_t* bempty = bfull + 2;
@@ -267,8 +272,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int H = p.H, I = p.I, T = p.T;
-  const int nchA = (H + KC - 1) / KC;  // H % 256 == 0, I % 128 == 0: a last chunk may
-  const int nchB = (I + KC - 1) / KC;  // hold fewer stages
+  const int nchA = H / kTcKC;                // H % 256 == 0
+  const int nchB = (I + kTcKC - 1) / kTcKC;  // I % 128 == 0: the last chunk may be 128 wide
   const int tpeA = I / 64, tpeB = H / 128;   // tiles per expert
   const Planes PL = plane_offsets(FMT, H, I);
   const int G = gridDim.x, cta = blockIdx.x;
@@ -276,22 +281,22 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 128);  // the decoder group that owns the chunk
+      mbar_init(&empty[s], 128);
     }
     for (int t = 0; t < kTcTS; ++t) {
-      mbar_init(&afull[t], 128);  // the group's decoders stored the half
-      mbar_init(&afree[t], 1);    // the MMA warp's commit: the half's MMAs are done
+      mbar_init(&tfull[t], 128);
+      mbar_init(&tempty[t], 1);
     }
     for (int a = 0; a < 2; ++a) {
-      mbar_init(&accfull[a], 1);   // the MMA warp's commit after a tile's last MMA
-      mbar_init(&accfree[a], 128); // the tile-end warps read the accumulator
+      mbar_init(&afull[a], 1);
+      mbar_init(&aempty[a], 128);
       mbar_init(&sfull[a], 1);
       mbar_init(&sempty[a], 128 * kTcGroups);
       mbar_init(&bfull[a], 1);
-      mbar_init(&bempty[a], 1);    // the MMA warp's commit after the h block's last MMA
+      mbar_init(&bempty[a], 1);
     }
     mbar_init(tbl_ready, 128);
-    mbar_init(done, 1);  // the MMA warp's last commit
+    mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -302,6 +307,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
   if (threadIdx.x == kTcProdWarp * 32) {
     if constexpr (kGU) {
       prefetch_tensormap(&mg);
+      prefetch_tensormap(&mu);
+      prefetch_tensormap(&msg);
+      prefetch_tensormap(&msu);
     }
     if constexpr (kDN) {
       prefetch_tensormap(&md);
@@ -365,80 +373,66 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
     u = j / tpeB;
     rb = j - u * tpeB;
   };
-  auto is_a = [&](int i) { return kGU && (MODE == 0 || i < nA); };
-  // buffer and phase parity of the q-th h block (one or two buffers)
-  auto hb_idx = [&](int q) { return p.hbn == 2 ? (q & 1) : 0; };
-  auto hb_par = [&](int q) { return (uint32_t)(p.hbn == 2 ? ((q >> 1) & 1) : (q & 1)); };
-  // the same for the scale buffer of tile i
-  auto sb_idx = [&](int i) { return p.sbn == 2 ? (i & 1) : 0; };
-  auto sb_par = [&](int i) { return (uint32_t)(p.sbn == 2 ? ((i >> 1) & 1) : (i & 1)); };
-  // the last down tile on an expert's h block (the buffer is then released)
-  auto last_on_h = [&](int i) { return i + 1 == tcount || tbl[i + 1].e != tbl[i].e; };
 
   if (warp == kTcProdWarp) {
-    // ------------------------------------------------ TMA producer: the
-    // whole warp runs the loop (converged); one elected lane issues
-    {
+    // ------------------------------------------------ TMA producer
+    if (elect_one()) {
       int gc = 0, bseq = -1, prev_e = -1;
-      // the next stage, once its previous chunk has been read
-      auto next_stage = [&]() {
+      auto next_stage = [&](uint32_t tx) {
         const int s = gc % S;
         mbar_wait_guarded(&empty[s], ((gc / S) & 1) ^ 1, p.status, abort_flag);
-        __syncwarp();
+        mbar_arrive_expect_tx(&full[s], tx);
         ++gc;
         return s;
       };
       // the expert's h rows [s0, s0 + NB) into the next B buffer
-      auto load_h = [&](int s0) {
+      auto load_h = [&](int e) {
         ++bseq;
-        const int b = hb_idx(bseq);
-        mbar_wait_guarded(&bempty[b], hb_par(bseq) ^ 1u, p.status, abort_flag);
-        __syncwarp();
-        const uint32_t ab = (uint32_t)NB * 128u;
-        mbar_arrive_expect_tx_warp(&bfull[b], ab * (uint32_t)(I / 64));
+        const int b = bseq & 1;
+        const int s0 = p.shared_mode ? 0 : p.offsets[e];
+        mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
+        const uint32_t ab = (uint32_t)p.NB * 128u;
+        mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
         for (int a = 0; a < I / 64; ++a)
-          tma_load_2d_warp(smem + L.hb + b * L.hb_bytes + a * ab, &mh, 64 * a, s0, &bfull[b]);
-      };
-      // the block scales of tile i (rows contiguous in their plane: one bulk
-      // copy per plane) into scale buffer i % 2
-      auto load_scales = [&](int i, const uint8_t* src0, const uint8_t* src1, uint32_t bytes) {
-        const int sb = sb_idx(i);
-        mbar_wait_guarded(&sempty[sb], sb_par(i) ^ 1u, p.status, abort_flag);
-        __syncwarp();
-        mbar_arrive_expect_tx_warp(&sfull[sb], src1 ? 2u * bytes : bytes);
-        bulk_g2s_warp(smem + L.sbuf + sb * L.s_bytes, src0, bytes, &sfull[sb]);
-        if (src1) bulk_g2s_warp(smem + L.sbuf + sb * L.s_bytes + bytes, src1, bytes, &sfull[sb]);
+          tma_load_2d(smem + L.hb + b * L.hb_bytes + a * ab, &mh, 64 * a, s0, &bfull[b]);
       };
       for (int i = 0; i < tcount; ++i) {
-        if (is_a(i)) {
+        if (kGU && (MODE == 0 || i < nA)) {
           int u, rb;
           tile_a(i, u, rb);
           const int e = expert_of(u);
-          // gate rows rb*64.. then the same up rows, every K block
-          const uint8_t* ex = p.wbase + (uint64_t)e * p.stride;
-          const uint64_t so = (uint64_t)rb * 64u * (uint64_t)(H / 16);
-          load_scales(i, ex + PL.scales[0] + so, ex + PL.scales[1] + so, 4u * H);
           for (int c = 0; c < nchA; ++c) {
-            const int s = next_stage();
+            const int s = next_stage(L.codes_bytes + 128u * 16u);
             uint8_t* st = smem + s * L.stage_bytes;
-            // gate rows rb*64.. then the same up rows: one box over both planes
-            tma_stage1_4d_warp(&full[s], L.codes_bytes, st, &mg, c * kTcCBR, rb * 64, 0, e);
+            // gate rows rb*64.. then the same up rows: one box over both
+            // planes for the codes, one for the scales
+            tma_load_4d(st, &mg, c * CBR, rb * 64, 0, e, &full[s]);
+            tma_load_4d(st + L.codes_bytes, &msg, c * 8, rb * 64, 0, e, &full[s]);
           }
           continue;
         }
         if constexpr (kDN) {
           const int ib = i - nA;  // down-tile sequence number
-          if (ib == 0) mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
-          const int u = tbl[i].u, rb = tbl[i].rb, e = tbl[i].e;
+          int u, rb;
+          if constexpr (MODE == 1) {
+            tile_b1(i, u, rb);
+          } else {
+            if (ib == 0) mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
+            u = tbl[i].u;
+            rb = tbl[i].rb;
+          }
+          const int e = expert_of(u);
           // the tile's scales: rows rb*128.. of the down plane, all of K
-          load_scales(i,
-                      p.wbase + (uint64_t)e * p.stride + PL.scales[2] +
-                          (uint64_t)rb * 128u * (uint64_t)(I / 16),
-                      nullptr, 8u * I);
+          const int sb = ib & 1;
+          mbar_wait_guarded(&sempty[sb], ((ib >> 1) & 1) ^ 1, p.status, abort_flag);
+          mbar_arrive_expect_tx(&sfull[sb], 8u * I);
+          bulk_g2s(smem + L.sbuf + sb * L.s_bytes,
+                   p.wbase + (uint64_t)e * p.stride + PL.scales[2] +
+                       (uint64_t)rb * 128u * (uint64_t)(I / 16),
+                   8u * I, &sfull[sb]);
           auto issue_b = [&](int c) {
-            const int s = next_stage();
-            tma_stage1_3d_warp(&full[s], L.codes_bytes, smem + s * L.stage_bytes, &md,
-                               c * kTcCBR, rb * 128, e);
+            const int s = next_stage(L.codes_bytes);
+            tma_load_3d(smem + s * L.stage_bytes, &md, c * CBR, rb * 128, e, &full[s]);
           };
           const bool new_h = ib == 0 || e != prev_e;
           if constexpr (MODE == 1) {
@@ -447,7 +441,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
             for (int c = 0; c < pre; ++c) issue_b(c);
             if (new_h) {
               if (bseq < 0) pdl_wait_prior();  // h is written by the preceding grid
-              load_h(tbl[i].s0);
+              load_h(e);
             }
             for (int c = pre; c < nchB; ++c) issue_b(c);
           } else {
@@ -457,63 +451,41 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
               // has counted itself; then read it through the async proxy
               gmem_wait_geq(p.sync + u, tpeA, p.status, abort_flag);
               fence_proxy_async_global();
-              __syncwarp();
-              load_h(tbl[i].s0);
+              load_h(e);
             }
           }
           prev_e = e;
         }
       }
-      // Before the CTA can exit, every copy it issued has landed (normally
-      // the consumers have seen them all; after a timed-out wait this waits,
-      // bounded, for the copies still in flight).
-      constexpr long long kDrain = 20000000;  // about 10 ms per copy
-      for (int x = max(0, gc - S); x < gc; ++x)
-        mbar_wait_bounded(&full[x % S], (x / S) & 1, p.status, kDrain);
-      for (int x = max(0, tcount - p.sbn); x < tcount; ++x)
-        mbar_wait_bounded(&sfull[sb_idx(x)], sb_par(x), p.status, kDrain);
-      for (int x = max(0, bseq - p.hbn + 1); x <= bseq; ++x)
-        mbar_wait_bounded(&bfull[hb_idx(x)], hb_par(x), p.status, kDrain);
     }
     __syncwarp();
   } else {
-    // ---- everyone else: the tile-end warps build the tile table at once;
-    // the decoders and the MMA warp fill the gate/up B operand meanwhile
-    constexpr int kFillers = (kTcWarps - 5) * 32;  // warps 4..11 and the MMA warp
-    if (warp >= 4) {
-      if constexpr (kGU) {
-        const int ftid = warp < kTcProdWarp ? (int)threadIdx.x - 128 : (int)threadIdx.x - 160;
-        fill_tokens<FMT>(smem + L.b, p.hidden, T, H, NB, ftid, kFillers);
-        fence_proxy_async_smem();
-        named_bar_sync(2, kFillers);
-      }
-    } else {
+    // ---- everyone else: the gate/up B operand, then (epilogue warps) the
+    // tile table
+    if constexpr (kGU) {
+      // the producer warp is not among the fillers: renumber the warps after it
+      const int ftid = warp < kTcProdWarp ? (int)threadIdx.x : (int)threadIdx.x - 32;
+      fill_tokens<FMT>(smem + L.b, p.hidden, T, H, p.NB, ftid, (kTcWarps - 1) * 32);
+      fence_proxy_async_smem();
+      named_bar_sync(2, (kTcWarps - 1) * 32);
+    }
+    if (warp < 4) {
       const int r = threadIdx.x;
-      // fused: per round k of down tiles, the CTAs with more than k of them,
-      // in all and below this one
-      int* gt_all = reinterpret_cast<int*>(smem + L.xch);
-      int* gt_below = gt_all + p.maxT;
+      int* bcnt = reinterpret_cast<int*>(smem + L.xch);  // fused: down tiles of every CTA
       if constexpr (MODE == 2) {
-        for (int k = r; k < 2 * p.maxT; k += 128) gt_all[k] = 0;
-        named_bar_sync(1, 128);
-        for (int c2 = r; c2 < G; c2 += 128) {
-          const int b = min(tc_deal_bstart(deal, c2 + 1) - tc_deal_bstart(deal, c2), nB);
-          for (int k = 0; k < b; ++k) {
-            atomicAdd(&gt_all[k], 1);
-            if (c2 < cta) atomicAdd(&gt_below[k], 1);
-          }
-        }
+        for (int c2 = r; c2 < G; c2 += 128)
+          bcnt[c2] = tc_deal_bstart(deal, c2 + 1) - tc_deal_bstart(deal, c2);
         named_bar_sync(1, 128);
       }
       for (int i = r; i < tcount; i += 128) {
         TcTile& t = tbl[i];
         int u, rb;
-        if (is_a(i)) {
+        if (kGU && (MODE == 0 || i < nA)) {
           tile_a(i, u, rb);
         } else if (MODE == 1) {
           tile_b1(i, u, rb);
         } else {
-          const int j = tc_deal_down_tile_counted(deal, gt_all, gt_below, nB, i - nA);
+          const int j = tc_deal_down_tile(deal, bcnt, cta, i - nA);
           u = j / tpeB;
           rb = j - u * tpeB;
         }
@@ -531,15 +503,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
             dev_flag(p.status, STRATA_DEV_BOUNDS);
             t.n = 0;
           }
-          if (t.s0 < 0 || t.s0 + t.n > Pn) {
-            dev_flag(p.status, STRATA_DEV_BOUNDS);
-            t.s0 = 0;
-            t.n = 0;
-          }
         }
-        if (t.n < 0 || t.n > TP) {
+        if (t.n < 0 || t.n > p.NB) {
           dev_flag(p.status, STRATA_DEV_BOUNDS);
-          t.n = t.n < 0 ? 0 : TP;
+          t.n = t.n < 0 ? 0 : p.NB;
         }
       }
       named_bar_sync(1, 128);
@@ -562,49 +529,38 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
   }
 
   if (warp < 4) {
-    // ------------------------------------------------ tile ends: the tile's
-    // accumulator, then SwiGLU / h / y
+    // ------------------------------------------------ epilogue
     mbar_wait_backoff(tbl_ready, 0, p.status, abort_flag);
-    const int r = threadIdx.x;  // tile row = TMEM lane (warp w reads lanes 32w..)
+    const int r = threadIdx.x;  // tile row = TMEM lane
     float* xch = reinterpret_cast<float*>(smem + L.xch);
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
     for (int i = 0; i < tcount; ++i) {
       const TcTile& ti = tbl[i];
-      const int n = ti.n;
       const int a = i & 1;
-      mbar_wait_backoff(&accfull[a], (i >> 1) & 1, p.status, abort_flag);
+      mbar_wait_backoff(&afull[a], (i >> 1) & 1, p.status, abort_flag);
       tc_fence_after();
-      uint32_t D[16];
-      tmem_ld16_wait(tmem_base + lane_off + (uint32_t)(kTcAccCol0 + 16 * a), D);
-      // the accumulator is in registers: the MMA warp may start tile i + 2 in it
+      uint32_t v[16];
+      tmem_ld16(tmem_base + ((uint32_t)(32 * warp) << 16) + (uint32_t)(a * 32), v);
+      tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(&accfree[a]);
-      // column of pair j: its token (gate/up: B holds every token) or j (down)
-      auto val = [&](int j) {
-        const int col = is_a(i) ? ti.tok[j] : j;
-        float v = 0.f;
+      mbar_arrive(&aempty[a]);
+      if (kGU && (MODE == 0 || i < nA)) {
+        float* xr = xch + r * 17;  // rows 0-63 gate, 64-127 up
 #pragma unroll
-        for (int c = 0; c < 16; ++c) v = (c == col) ? __uint_as_float(D[c]) : v;
-        return v;
-      };
-      if (is_a(i)) {
-        // SwiGLU: rows 0-63 gate, 64-127 the same up rows
-        if (r >= 64) {
-          for (int j = 0; j < n; ++j) xch[(r - 64) * 17 + j] = val(j);
-        }
+        for (int j = 0; j < 16; ++j) xr[j] = __uint_as_float(v[j]);
         named_bar_sync(1, 128);
-        if (r < 64) {
-          const int ii = ti.rb * 64 + r;  // row of I
+        for (int idx = r; idx < ti.n * 64; idx += 128) {
+          const int j = idx >> 6, l = idx & 63;
+          const int t = ti.tok[j];
+          const float gv = xch[l * 17 + t], uv = xch[(64 + l) * 17 + t];
+          const float h = silu_f32(gv) * uv;
+          const int ii = ti.rb * 64 + l;
           const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
-          for (int j = 0; j < n; ++j) {
-            const float hv = silu_f32(val(j)) * xch[r * 17 + j];
-            p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(__float2half_rn(hv));
-          }
-          if constexpr (MODE == 2) {
-            // publish this thread's h stores (to the TMA reads of other CTAs)
-            fence_proxy_async_global();
-            __threadfence();
-          }
+          p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(__float2half_rn(h));
+        }
+        if constexpr (MODE == 2) {
+          // publish this thread's h stores (to the TMA reads of other CTAs)
+          fence_proxy_async_global();
+          __threadfence();
         }
         named_bar_sync(1, 128);
         if constexpr (MODE == 2) {
@@ -612,161 +568,168 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate and up codes 
         }
       } else if constexpr (kDN) {
         const int row = ti.rb * 128 + r;
-        for (int j = 0; j < n; ++j) p.y[(size_t)(ti.s0 + j) * H + row] = val(j);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j < ti.n) p.y[(size_t)(ti.s0 + j) * H + row] = __uint_as_float(v[j]);
       }
     }
   } else if (warp < kTcProdWarp) {
     // ------------------------------------------------ decoders
-    const int g = (warp - kTcDecWarp0) >> 2;
+    const int g = (warp - 4) >> 2;
     const int qd = warp & 3;
     const int r = 32 * qd + lane;  // tile row = TMEM lane
-    const uint32_t swz = (uint32_t)r & 7u;  // 128-byte swizzle of the stage rows
-    const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+    const uint32_t swz = ((uint32_t)(r * CBR) >> 7) & (uint32_t)(NPC - 1);
+    const uint32_t tl = tmem_base + ((uint32_t)(32 * qd) << 16) + kTcACol0;
     const Q4Table T4 = q4_table();
     int gc = 0;
-    int q = 0;          // this group's next tensor-memory stage (0..kTcSPG-1), round robin
-    uint32_t fpar = 0;  // bit q: parity of the next wait on afree[kTcSPG g + q]
     for (int i = 0; i < tcount; ++i) {
-      const bool isA = is_a(i);
+      const bool isA = kGU && (MODE == 0 || i < nA);
+      const int ib = i - nA;
       const int K = isA ? H : I;
       const int nch = isA ? nchA : nchB;
-      // this row's block scales of the tile (every K block)
-      mbar_wait_guarded(&sfull[sb_idx(i)], sb_par(i), p.status, abort_flag);
-      const uint8_t* srow = smem + L.sbuf + sb_idx(i) * L.s_bytes + r * ((isA ? H : I) / 16);
+      const uint8_t* srow = nullptr;
+      if (!isA) {
+        mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
+        srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
+      }
       for (int c = 0; c < nch; ++c, ++gc) {
         if (gc % kTcGroups != g) continue;
         const int s = gc % S;
         mbar_wait_guarded(&full[s], (gc / S) & 1, p.status, abort_flag);
-        const uint8_t* st = smem + s * L.stage_bytes + r * kTcCBR;
-        const int nh = min(KC, K - c * KC) / kTcKH;  // K is a multiple of kTcKH
-        // one tensor-memory stage (128 K) at a time; a single copy of the
-        // body keeps the loop inside the instruction cache
-#pragma unroll 1
-        for (int h = 0; h < nh; ++h) {
-          // this row's codes of the stage: NPH 16-byte pieces of the
-          // 128-byte swizzled row, and the four blocks' scales
-          uint4 cw[NPH];
+        const uint8_t* st = smem + s * L.stage_bytes;
+        const int kv = min(kTcKC, K - c * kTcKC);  // 256, or 128 for a ragged last chunk
+        const int np = kv / PIECE_K;
+        uint4 cw[NPC];
 #pragma unroll
-          for (int pp = 0; pp < NPH; ++pp)
-            cw[pp] = lds128(st + (((uint32_t)(h * NPH + pp) ^ swz) << 4));
-          const uint2 sc = lds64(srow + 2 * (c * (KC / 32) + 4 * h));
-          const uint32_t scw[2] = {sc.x, sc.y};
-          // the stage's four blocks (64 codes per 16-byte piece for 2-bit,
-          // 32 for 4-bit), each times its scale, into R = 64 fp16 pairs
-          uint32_t R[64];
-          if constexpr (FMT == STRATA_FMT_Q2_32) {
-#pragma unroll
-            for (int pp = 0; pp < NPH; ++pp) {  // one piece: blocks 2pp, 2pp + 1
-              const uint4 v = cw[pp];
-              const __half2 d0 = scale2(scw[pp], 0), d1 = scale2(scw[pp], 1);
-              dq_q2_group(v.x, d0, *reinterpret_cast<uint32_t(*)[8]>(R + 32 * pp));
-              dq_q2_group(v.y, d0, *reinterpret_cast<uint32_t(*)[8]>(R + 32 * pp + 8));
-              dq_q2_group(v.z, d1, *reinterpret_cast<uint32_t(*)[8]>(R + 32 * pp + 16));
-              dq_q2_group(v.w, d1, *reinterpret_cast<uint32_t(*)[8]>(R + 32 * pp + 24));
-            }
-          } else {
-#pragma unroll
-            for (int pp = 0; pp < NPH; ++pp) {  // one piece: block pp
-              const uint4 v = cw[pp];
-              const __half2 d = scale2(scw[pp >> 1], pp & 1);
-              dq_q4_group(v.x, v.y, d, T4, *reinterpret_cast<uint32_t(*)[8]>(R + 16 * pp));
-              dq_q4_group(v.z, v.w, d, T4, *reinterpret_cast<uint32_t(*)[8]>(R + 16 * pp + 8));
-            }
+        for (int pc = 0; pc < NPC; ++pc)
+          cw[pc] = (pc < np) ? lds128(st + r * CBR + ((pc ^ swz) << 4)) : make_uint4(0, 0, 0, 0);
+        uint32_t sc[4];
+        if (isA) {
+          const uint4 v = lds128(st + L.codes_bytes + r * 16);
+          sc[0] = v.x;
+          sc[1] = v.y;
+          sc[2] = v.z;
+          sc[3] = v.w;
+        } else {
+          const uint2 lo = lds64(srow + c * 16);
+          sc[0] = lo.x;
+          sc[1] = lo.y;
+          sc[2] = 0;
+          sc[3] = 0;
+          if (kv > 128) {
+            const uint2 hi = lds64(srow + c * 16 + 8);
+            sc[2] = hi.x;
+            sc[3] = hi.y;
           }
-          const int stg = kTcSPG * g + q;
-          // the stage's previous MMAs have read it
-          mbar_wait_guarded(&afree[stg], ((fpar >> q) & 1u) ^ 1u, p.status, abort_flag);
-          fpar ^= 1u << q;
-          tc_fence_after();
-          const uint32_t ta = tmem_base + lane_off + (uint32_t)(stg * kTcStageCols);
-          tmem_st32(ta, *reinterpret_cast<const uint32_t(*)[32]>(R));
-          tmem_st32(ta + 32, *reinterpret_cast<const uint32_t(*)[32]>(R + 32));
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&afull[stg]);  // every row of the stage stored: the MMA warp may go
-          q = q + 1 == kTcSPG ? 0 : q + 1;
         }
-        // The stage's reads are done: order those generic-proxy reads before
-        // the producer's next TMA (async-proxy) write into it, which the
-        // barrier alone does not.
+        // The stage is released before its loads are consumed: order those
+        // generic-proxy reads before the producer's next TMA (async-proxy)
+        // write into the stage, which the barrier alone does not.
         fence_proxy_async_smem();
         mbar_arrive(&empty[s]);
+        const int t = gc % kTcTS;
+        mbar_wait_guarded(&tempty[t], ((gc / kTcTS) & 1) ^ 1, p.status, abort_flag);
+        tc_fence_after();
+        const uint32_t ta = tl + (uint32_t)t * 128u;
+        if constexpr (FMT == STRATA_FMT_Q2_32) {
+#pragma unroll
+          for (int pc = 0; pc < NPC; ++pc) {
+            if (pc < np) {
+              uint32_t R[32];
+              const uint32_t d0 = dup_lo(sc[pc]), d1 = dup_hi(sc[pc]);
+              dq_q2_word(cw[pc].x, d0, R);
+              dq_q2_word(cw[pc].y, d0, R + 8);
+              dq_q2_word(cw[pc].z, d1, R + 16);
+              dq_q2_word(cw[pc].w, d1, R + 24);
+              tmem_st32(ta + pc * 32, R);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int pc = 0; pc < NPC; ++pc) {
+            if (pc < np) {
+              uint32_t R[16], R0[8], R1[8];
+              const __half2 d2 =
+                  u32_as_h2((pc & 1) ? dup_hi(sc[pc >> 1]) : dup_lo(sc[pc >> 1]));
+              dq_q4_group(cw[pc].x, cw[pc].y, d2, T4, R0);
+              dq_q4_group(cw[pc].z, cw[pc].w, d2, T4, R1);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) {
+                R[j] = R0[j];
+                R[8 + j] = R1[j];
+              }
+              tmem_st16(ta + pc * 16, R);
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&tfull[t]);
       }
-      fence_proxy_async_smem();  // scale reads before the next bulk copy into the buffer
-      mbar_arrive(&sempty[sb_idx(i)]);
+      if (!isA) {
+        fence_proxy_async_smem();  // same for the scale block and its next bulk copy
+        mbar_arrive(&sempty[ib & 1]);
+      }
     }
   } else if (warp == kTcMmaWarp) {
-    // ------------------------------------------------ MMA issue: every half
-    // chunk of both groups in chunk order, once its decoders have stored it;
-    // a tile's halves accumulate into one accumulator (tiles alternate
-    // between two).  The whole warp runs the loop; one elected lane issues.
-    const uint32_t idesc = idesc_f16_f32(16);
-    const uint32_t sbo = NB == 16 ? 1024u : 0u;
-    // descriptor start-address step (16-byte units): one 64-K atom of B
-    const uint32_t d_atom = ((uint32_t)NB * 128u) >> 4;
-    const uint32_t bhi = smem_desc_k128_hi(sbo);
-    // warp-uniform by construction (one lane's value), so the issue operands
-    // stay in uniform registers
-    const uint32_t tbase = __shfl_sync(0xffffffffu, tmem_base, 0);
-    uint32_t apar = 0;  // bit stg: parity of the next wait on afull[stg]
-    uint32_t qpack = 0;  // 2 bits per group: its next stage (as its decoders count)
-    int gc = 0, bseq = -1, prev_e = -1;
-    bool ok = true;
-    for (int i = 0; i < tcount && ok; ++i) {
-      const bool isA = is_a(i);
-      const int K = isA ? H : I;
-      const int nch = isA ? nchA : nchB;
-      const int a = i & 1;
-      if (!isA) {
-        const int ib = i - nA;
-        if (ib == 0) ok = mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
-        const int e = tbl[i].e;
-        if (ib == 0 || e != prev_e) {
-          // a new h block: its rows have landed
-          ++bseq;
-          ok = ok && mbar_wait_guarded(&bfull[hb_idx(bseq)], hb_par(bseq), p.status, abort_flag);
+    // ------------------------------------------------ MMA issue (one thread)
+    if constexpr (MODE == 1) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
+    if (elect_one()) {
+      const uint32_t idesc = idesc_f16_f32(16);
+      const uint32_t sbo = p.NB == 16 ? 1024u : 0u;
+      const uint32_t ab = (uint32_t)p.NB * 128u;
+      // descriptor start-address steps (16-byte units): one 64-K atom, one K16 step
+      const uint32_t d_atom = ab >> 4, d_k16 = 32 >> 4;
+      const uint32_t bhi = smem_desc_k128_hi(sbo);
+      int gc = 0, bseq = -1, prev_e = -1;
+      for (int i = 0; i < tcount; ++i) {
+        const bool isA = kGU && (MODE == 0 || i < nA);
+        uint32_t bbase = smem_addr(smem + L.b);
+        int b = 0;
+        if (!isA) {
+          if (MODE == 2 && i == nA) mbar_wait_guarded(tbl_ready, 0, p.status, abort_flag);
+          const int e = tbl[i].e;
+          if (i == nA || e != prev_e) {
+            ++bseq;
+            mbar_wait_guarded(&bfull[bseq & 1], (bseq >> 1) & 1, p.status, abort_flag);
+            tc_fence_after();
+          }
+          prev_e = e;
+          b = bseq & 1;
+          bbase = smem_addr(smem + L.hb) + (uint32_t)b * L.hb_bytes;
         }
-        prev_e = e;
-      }
-      // the tile-end warps have read this accumulator's tile before last
-      ok = ok && mbar_wait_guarded(&accfree[a], (((i >> 1) & 1) ^ 1u), p.status, abort_flag);
-      // B: every token (gate/up) or the expert's h block (down)
-      const uint32_t bbase = isA ? smem_addr(smem + L.b)
-                                 : smem_addr(smem + L.hb) + (uint32_t)hb_idx(bseq) * L.hb_bytes;
-      const uint32_t blo0 = __shfl_sync(0xffffffffu, smem_desc_k128_lo(bbase), 0);
-      const uint32_t dt = tbase + (uint32_t)(kTcAccCol0 + 16 * a);
-      for (int c = 0; c < nch && ok; ++c, ++gc) {
-        const int g = gc % kTcGroups;
-        const int nh = min(KC, K - c * KC) / kTcKH;
-        // B: the chunk starts KC / 64 atoms of 64 K in, a stage two atoms later
-        const uint32_t blo = blo0 + (uint32_t)c * (uint32_t)(KC / 64) * d_atom;
-#pragma unroll
-        for (int h = 0; h < KC / kTcKH; ++h) {
-          if (h >= nh) break;
-          const int qg = (int)((qpack >> (2 * g)) & 3u);
-          const int stg = kTcSPG * g + qg;
-          qpack ^= (uint32_t)(qg ^ (qg + 1 == kTcSPG ? 0 : qg + 1)) << (2 * g);
-          ok = mbar_wait_guarded(&afull[stg], (apar >> stg) & 1u, p.status, abort_flag);
-          apar ^= 1u << stg;
-          if (!ok) break;
-          __syncwarp();
+        const int K = isA ? H : I;
+        const int nch = isA ? nchA : nchB;
+        const int a = i & 1;
+        mbar_wait_guarded(&aempty[a], ((i >> 1) & 1) ^ 1, p.status, abort_flag);
+        tc_fence_after();
+        const uint32_t d = tmem_base + (uint32_t)(a * 32);
+        // B descriptor of the chunk's first K16 step; the steps inside a
+        // chunk are constant offsets from it (the loop is unrolled)
+        uint32_t bd = smem_desc_k128_lo(bbase);
+        for (int c = 0; c < nch; ++c, ++gc, bd += 4 * d_atom) {
+          const int t = gc % kTcTS;
+          mbar_wait_guarded(&tfull[t], (gc / kTcTS) & 1, p.status, abort_flag);
           tc_fence_after();
-          // the half's eight K16 steps; the first of the tile overwrites
-          mma_half_ts_warp<NB * 8>(dt, tbase + (uint32_t)(stg * kTcStageCols),
-                                   blo + (uint32_t)h * 2u * d_atom, bhi, idesc,
-                                   (uint32_t)(c > 0 || h > 0));
-          mma_commit_warp(&afree[stg]);
+          const bool half = K - c * kTcKC < kTcKC;  // ragged last chunk: 128 K
+          const uint32_t at = tmem_base + kTcACol0 + (uint32_t)t * 128u;
+#pragma unroll
+          for (int kk = 0; kk < kTcKC / 16; ++kk) {
+            if (kk < kTcKC / 32 || !half)
+              mma_f16_ts(d, at + (uint32_t)kk * 8u, bd + (kk >> 2) * d_atom + (kk & 3) * d_k16,
+                         bhi, idesc, (c > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&tempty[t]);
+        }
+        mma_commit(&afull[a]);
+        if (!isA) {
+          if (i + 1 == tcount || tbl[i + 1].e != tbl[i].e) mma_commit(&bempty[b]);
         }
       }
-      if (!ok) break;
-      mma_commit_warp(&accfull[a]);  // the tile's accumulator, once its MMAs are done
-      // the h block is free once the MMAs of its expert's last tile are done
-      if (!isA && last_on_h(i)) mma_commit_warp(&bempty[hb_idx(bseq)]);
+      mma_commit(done);
+      // every MMA retired before the tensor memory is released (bounded)
+      mbar_wait_bounded(done, 0, p.status);
     }
-    // every MMA retired before the tensor memory is released (bounded)
-    __syncwarp();
-    mma_commit_warp(done);
-    mbar_wait_bounded(done, 0, p.status);
     __syncwarp();
   }
   tc_fence_before();
@@ -802,8 +765,8 @@ int tc_max_tiles(int mode, int Umax, int H, int I, int grid) {
 // group count: chunk c uses stage c % S and group c % kTcGroups, so every
 // use of a stage belongs to one group and its barrier phases are awaited in
 // order (a waiter two phases ahead would see its parity as complete).
-int tc_stages(int mode, int fmt, int NB, int H, int I, int maxT, int hbn, int sbn) {
-  const TcLayout L0 = tc_layout(mode, fmt, NB, H, I, 0, maxT, hbn, sbn);
+int tc_stages(int mode, int fmt, int NB, int H, int I, int maxT) {
+  const TcLayout L0 = tc_layout(mode, fmt, NB, H, I, 0, maxT);
   const long long room = (long long)kTcSmemBudget - 1024 - (long long)L0.total;
   if (room <= 0) return 0;
   const int s = (int)std::min<long long>(kTcMaxStages, room / L0.stage_bytes);
@@ -823,36 +786,17 @@ void pdl_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int grid, in
   cfg.numAttrs = 1;
 }
 
-template <int MODE, int FMT, int NB>
-cudaError_t launch_tc(const CUtensorMap (&m)[3], const TcParams& prm, int grid, cudaStream_t st) {
-  auto kern = decode_tc_kernel<MODE, FMT, NB>;
-  const size_t smem =
-      1024 + tc_layout(MODE, FMT, NB, prm.H, prm.I, prm.S, prm.maxT, prm.hbn, prm.sbn).total;
+template <int MODE, int FMT>
+cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, cudaStream_t st) {
+  auto kern = decode_tc_kernel<MODE, FMT>;
+  const size_t smem = 1024 + tc_layout(MODE, FMT, prm.NB, prm.H, prm.I, prm.S, prm.maxT).total;
   cudaError_t e =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   pdl_config(cfg, attr, grid, kTcThreads, smem, st);
-  return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], prm);
-}
-
-template <int MODE, int NB>
-cudaError_t launch_tc_fmt(int fmt, const CUtensorMap (&m)[3], const TcParams& prm, int grid,
-                          cudaStream_t st) {
-  if (fmt == STRATA_FMT_Q2_32) return launch_tc<MODE, STRATA_FMT_Q2_32, NB>(m, prm, grid, st);
-  return launch_tc<MODE, STRATA_FMT_Q4CB_32, NB>(m, prm, grid, st);
-}
-
-// B rows NB (8: rows 8-15 of the N = 16 MMA repeat rows 0-7) from the call's
-// token count.
-inline int tc_nb(int T) { return T <= 8 ? 8 : 16; }
-
-template <int MODE>
-cudaError_t launch_tc_nb(int T, int fmt, const CUtensorMap (&m)[3], const TcParams& prm,
-                         int grid, cudaStream_t st) {
-  if (T <= 8) return launch_tc_fmt<MODE, 8>(fmt, m, prm, grid, st);
-  return launch_tc_fmt<MODE, 16>(fmt, m, prm, grid, st);
+  return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], prm);
 }
 
 cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
@@ -862,40 +806,18 @@ cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
   return cudaLaunchKernelEx(&cfg, tc_sync_reset_kernel, sync, n);
 }
 
-// Stages, h buffers and scale buffers of one kernel form: two h buffers
-// unless that leaves fewer than `want` stages, then two scale buffers unless
-// that leaves fewer than kTcGroups.
-constexpr int kTcWantStages = 6;
-void tc_plan(int mode, int fmt, int T, int H, int I, int maxT, int want, int& S, int& hbn,
-             int& sbn) {
-  hbn = 2;
-  sbn = 2;
-  S = tc_stages(mode, fmt, tc_nb(T), H, I, maxT, hbn, sbn);
-  if (mode != 0 && S < want) {
-    hbn = 1;
-    S = tc_stages(mode, fmt, tc_nb(T), H, I, maxT, hbn, sbn);
-  }
-  if (S < kTcGroups) {
-    sbn = 1;
-    S = tc_stages(mode, fmt, tc_nb(T), H, I, maxT, hbn, sbn);
-  }
-}
-
-bool tc_fused_fits(int T, int H, int I, int Umax, int fmt, int grid) {
-  if (grid > kTcMaxGrid) return false;
-  int S, hbn, sbn;
-  tc_plan(2, fmt, T, H, I, tc_max_tiles(2, Umax, H, I, grid), kTcFusedMinStages, S, hbn, sbn);
-  return S >= kTcFusedMinStages;
+bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
+  return grid <= kTcMaxGrid &&
+         tc_stages(2, fmt, NB, H, I, tc_max_tiles(2, Umax, H, I, grid)) >= kTcFusedMinStages;
 }
 
 }  // namespace
 
 bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid) {
   if (T < 1 || T > kDecodeMaxTokens || H % 256 || I % 128 || grid < 1 || Umax < 1) return false;
-  int S0, S1, hbn, sbn;
-  tc_plan(0, fmt, T, H, I, tc_max_tiles(0, Umax, H, I, grid), kTcWantStages, S0, hbn, sbn);
-  tc_plan(1, fmt, T, H, I, tc_max_tiles(1, Umax, H, I, grid), kTcWantStages, S1, hbn, sbn);
-  return S0 >= kTcGroups && S1 >= kTcGroups;
+  const int NB = T <= 8 ? 8 : 16;
+  return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, Umax, H, I, grid)) >= kTcGroups &&
+         tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, Umax, H, I, grid)) >= kTcGroups;
 }
 
 cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
@@ -903,35 +825,47 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   const long long P = a.shared_mode ? a.T : (long long)a.T * a.k;
   const int Umax = a.shared_mode ? 1 : (int)std::min<long long>(a.E, P);
   if (!decode_tc_supported(a.T, a.H, a.I, Umax, a.fmt, a.num_sms)) return cudaErrorNotSupported;
-  const int NB = tc_nb(a.T);
+  const int NB = a.T <= 8 ? 8 : 16;
   const Planes PL = plane_offsets(a.fmt, a.H, a.I);
+  const bool q2 = a.fmt == STRATA_FMT_Q2_32;
+  const cuuint32_t cbr = q2 ? kTcKC / 4 : kTcKC / 2;
+  const CUtensorMapSwizzle sw = cbr == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   const cuuint64_t rowH = codes_row_bytes(a.fmt, a.H), rowI = codes_row_bytes(a.fmt, a.I);
-  // Codes in boxes of 128-byte rows (a TMA box costs about the same per box,
-  // so boxes are 16 KB): gate and up as one 4-D map whose third dimension
-  // steps from the gate plane to the up plane (64 + 64 rows per box), down
-  // 128 rows per box; and h.
-  CUtensorMap m[3];
+  CUtensorMap m[6];  // gate codes, up codes, gate scales, up scales, down codes, h
+  // gate and up as one 4-D map each for codes and scales: the third
+  // dimension steps from the gate plane to the up plane, so one box carries
+  // the tile's 64 gate rows and the same 64 up rows (fewer, larger boxes)
   {
     const cuuint64_t dims[4] = {rowH, (cuuint64_t)a.I, 2, (cuuint64_t)E};
     const cuuint64_t str[3] = {rowH, PL.codes[1] - PL.codes[0], a.stride};
-    const cuuint32_t box[4] = {(cuuint32_t)kTcCBR, 64, 2, 1};
+    const cuuint32_t box[4] = {cbr, 64, 2, 1};
     if (!make_tmap(&m[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, a.wbase + PL.codes[0], dims, str, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+                   sw))
       return cudaErrorInvalidValue;
+    m[1] = m[0];
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)a.H / 32, (cuuint64_t)a.I, 2, (cuuint64_t)E};
+    const cuuint64_t str[3] = {(cuuint64_t)a.H / 16, PL.scales[1] - PL.scales[0], a.stride};
+    const cuuint32_t box[4] = {8, 64, 2, 1};
+    if (!make_tmap(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, a.wbase + PL.scales[0], dims, str,
+                   box, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    m[3] = m[2];
   }
   {
     const cuuint64_t dims[3] = {rowI, (cuuint64_t)a.H, (cuuint64_t)E};
     const cuuint64_t str[2] = {rowI, a.stride};
-    const cuuint32_t box[3] = {(cuuint32_t)kTcCBR, 128, 1};
-    if (!make_tmap(&m[1], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[2], dims, str, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    const cuuint32_t box[3] = {cbr, 128, 1};
+    if (!make_tmap(&m[4], CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[2], dims, str, box,
+                   sw))
       return cudaErrorInvalidValue;
   }
   {
     const cuuint64_t dims[2] = {(cuuint64_t)a.I, (cuuint64_t)P};
     const cuuint64_t str[1] = {(cuuint64_t)a.I * 2};
     const cuuint32_t box[2] = {64, (cuuint32_t)NB};
-    if (!make_tmap(&m[2], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.hbuf, dims, str, box,
+    if (!make_tmap(&m[5], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.hbuf, dims, str, box,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return cudaErrorInvalidValue;
   }
@@ -952,19 +886,26 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   prm.y = a.y;
   prm.status = a.status;
   prm.sync = a.sync;
+  prm.NB = NB;
   cudaError_t e;
-  if (a.sync && tc_fused_fits(a.T, a.H, a.I, Umax, a.fmt, a.num_sms)) {
+  if (a.sync && tc_fused_fits(NB, a.H, a.I, Umax, a.fmt, a.num_sms)) {
     prm.maxT = tc_max_tiles(2, Umax, a.H, a.I, a.num_sms);
-    tc_plan(2, a.fmt, a.T, a.H, a.I, prm.maxT, kTcFusedMinStages, prm.S, prm.hbn, prm.sbn);
+    prm.S = tc_stages(2, a.fmt, NB, a.H, a.I, prm.maxT);
     if ((e = launch_sync_reset(a.sync, Umax, st)) != cudaSuccess) return e;
-    return launch_tc_nb<2>(a.T, a.fmt, m, prm, a.num_sms, st);
+    if (q2) return launch_tc<2, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
+    return launch_tc<2, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
   }
   prm.maxT = tc_max_tiles(0, Umax, a.H, a.I, a.num_sms);
-  tc_plan(0, a.fmt, a.T, a.H, a.I, prm.maxT, kTcWantStages, prm.S, prm.hbn, prm.sbn);
-  if ((e = launch_tc_nb<0>(a.T, a.fmt, m, prm, a.num_sms, st)) != cudaSuccess) return e;
+  prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);
+  if (q2)
+    e = launch_tc<0, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
+  else
+    e = launch_tc<0, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+  if (e != cudaSuccess) return e;
   prm.maxT = tc_max_tiles(1, Umax, a.H, a.I, a.num_sms);
-  tc_plan(1, a.fmt, a.T, a.H, a.I, prm.maxT, kTcWantStages, prm.S, prm.hbn, prm.sbn);
-  return launch_tc_nb<1>(a.T, a.fmt, m, prm, a.num_sms, st);
+  prm.S = tc_stages(1, a.fmt, NB, a.H, a.I, prm.maxT);
+  if (q2) return launch_tc<1, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
+  return launch_tc<1, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
 }
 
 }  // namespace strata

@@ -108,6 +108,27 @@ STRATA_DEVFN void tma_load_2d(void* dst, const CUtensorMap* map, int c0, int c1,
       : "memory");
 }
 
+// 3-D tiled load (c0 innermost), no multicast.
+STRATA_DEVFN void tma_load_3d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// 4-D tiled load (c0 innermost), no multicast.
+STRATA_DEVFN void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
+                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+      "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Warp-converged forms of the copy issue: every lane of a converged warp
 // executes the statement and elect.sync picks the one lane that issues, so
 // the warp-uniform operands stay in uniform registers (a lone thread in a
@@ -218,6 +239,15 @@ STRATA_DEVFN void tmem_ld16_wait(uint32_t a0, uint32_t (&r)[16]) {
       : "memory");
 }
 
+STRATA_DEVFN void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
 STRATA_DEVFN void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
@@ -285,6 +315,24 @@ STRATA_DEVFN void mma_commit(uint64_t* bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
           smem_addr(bar))
+      : "memory");
+}
+
+// tcgen05.mma (kind::f16, A from tensor memory at a_tmem: 128 rows x 16 K,
+// two fp16 per 32-bit column, row m in lane m) issued by one thread, with the
+// B descriptor given as its two 32-bit words and joined into the 64-bit
+// operand inside the asm statement, so the compiler does no 64-bit
+// arithmetic on a descriptor.  (A build that added offsets to a 64-bit
+// descriptor in C++ handed some MMAs a descriptor whose high word was lost:
+// B was then read as an unswizzled layout with 16-byte rows.)
+STRATA_DEVFN void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
+                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "mov.b64 bd, {%2, %3};\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
