@@ -74,7 +74,7 @@ constexpr int kTcTmemCols = 512;
 constexpr int kTcMaxStages = 16;
 constexpr int kTcSmemBudget = 227 * 1024;
 constexpr int kTcFusedMinStages = 9;  // fewer: run the two-kernel form
-constexpr int kTcMaxGrid = 1024;      // the fused tile dealing keeps one int per CTA
+constexpr int kTcMaxGrid = 1024;      // grids the fused tile dealing is checked for
 // Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
 // only after the MMAs of its previous one retired, so with at least as many
 // stages as groups no waiter runs two phases ahead of a stage's barrier.
@@ -145,7 +145,6 @@ __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, 
   L.total = off;
   return L;
 }
-static_assert(2 * 64 * 17 * 4 >= 4 * kTcMaxGrid, "dealing scratch fits the exchange buffer");
 
 // ---------------------------------------------------------------- decode
 // One Q2 word (16 codes, element j at bits 2j) -> R[i] = fp16x2 (element i,
@@ -460,21 +459,32 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     }
     __syncwarp();
   } else {
-    // ---- everyone else: the gate/up B operand, then (epilogue warps) the
-    // tile table
-    if constexpr (kGU) {
-      // the producer warp is not among the fillers: renumber the warps after it
-      const int ftid = warp < kTcProdWarp ? (int)threadIdx.x : (int)threadIdx.x - 32;
-      fill_tokens<FMT>(smem + L.b, p.hidden, T, H, p.NB, ftid, (kTcWarps - 1) * 32);
-      fence_proxy_async_smem();
-      named_bar_sync(2, (kTcWarps - 1) * 32);
-    }
-    if (warp < 4) {
+    // ---- everyone else: the epilogue warps build the tile table at once;
+    // the decoders and the MMA warp fill the gate/up B operand meanwhile
+    constexpr int kFillers = (kTcWarps - 5) * 32;  // the warps after 3 but the producer
+    if (warp >= 4) {
+      if constexpr (kGU) {
+        const int ftid = warp < kTcProdWarp ? (int)threadIdx.x - 128 : (int)threadIdx.x - 160;
+        fill_tokens<FMT>(smem + L.b, p.hidden, T, H, p.NB, ftid, kFillers);
+        fence_proxy_async_smem();
+        named_bar_sync(2, kFillers);
+      }
+    } else {
       const int r = threadIdx.x;
-      int* bcnt = reinterpret_cast<int*>(smem + L.xch);  // fused: down tiles of every CTA
+      // fused: per round k of down tiles, the CTAs with more than k of them,
+      // in all and below this one
+      int* gt_all = reinterpret_cast<int*>(smem + L.xch);
+      int* gt_below = gt_all + p.maxT;
       if constexpr (MODE == 2) {
-        for (int c2 = r; c2 < G; c2 += 128)
-          bcnt[c2] = tc_deal_bstart(deal, c2 + 1) - tc_deal_bstart(deal, c2);
+        for (int k = r; k < 2 * p.maxT; k += 128) gt_all[k] = 0;
+        named_bar_sync(1, 128);
+        for (int c2 = r; c2 < G; c2 += 128) {
+          const int b = min(tc_deal_bstart(deal, c2 + 1) - tc_deal_bstart(deal, c2), nB);
+          for (int k = 0; k < b; ++k) {
+            atomicAdd(&gt_all[k], 1);
+            if (c2 < cta) atomicAdd(&gt_below[k], 1);
+          }
+        }
         named_bar_sync(1, 128);
       }
       for (int i = r; i < tcount; i += 128) {
@@ -485,7 +495,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         } else if (MODE == 1) {
           tile_b1(i, u, rb);
         } else {
-          const int j = tc_deal_down_tile(deal, bcnt, cta, i - nA);
+          const int j = tc_deal_down_tile_counted(deal, gt_all, gt_below, nB, i - nA);
           u = j / tpeB;
           rb = j - u * tpeB;
         }
@@ -807,8 +817,10 @@ cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
 }
 
 bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
-  return grid <= kTcMaxGrid &&
-         tc_stages(2, fmt, NB, H, I, tc_max_tiles(2, Umax, H, I, grid)) >= kTcFusedMinStages;
+  const int maxT = tc_max_tiles(2, Umax, H, I, grid);
+  // the dealing counts (two ints per table slot) live in the exchange buffer
+  return grid <= kTcMaxGrid && 8 * maxT <= 2 * 64 * 17 * 4 &&
+         tc_stages(2, fmt, NB, H, I, maxT) >= kTcFusedMinStages;
 }
 
 }  // namespace
