@@ -12,7 +12,7 @@ import os
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libstrata_moe.so")
 
-OK, EINVAL, ECUDA, EUNSUPPORTED, ETIMEOUT, EBOUNDS = range(6)
+OK, EINVAL, ECUDA, EUNSUPPORTED, ETIMEOUT, EBOUNDS, EOVERFLOW = range(7)
 FMT_Q2_32 = 1
 FMT_Q4CB_32 = 2
 DTYPE_F32 = 0

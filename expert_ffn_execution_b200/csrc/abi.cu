@@ -143,6 +143,7 @@ const char* strata_status_string(int32_t s) {
     case STRATA_EUNSUPPORTED: return "unsupported configuration";
     case STRATA_ETIMEOUT: return "device wait timed out";
     case STRATA_EBOUNDS: return "device index out of range";
+    case STRATA_EOVERFLOW: return "fp16 intermediate overflowed";
     default: return "unknown status";
   }
 }
@@ -164,6 +165,7 @@ int32_t strata_read_status(const int32_t* dev_status, void* stream) {
   if (cudaStreamSynchronize(st) != cudaSuccess) return STRATA_ECUDA;
   if (h & STRATA_DEV_TIMEOUT) return STRATA_ETIMEOUT;
   if (h & STRATA_DEV_BOUNDS) return STRATA_EBOUNDS;
+  if (h & STRATA_DEV_OVERFLOW) return STRATA_EOVERFLOW;
   return STRATA_OK;
 }
 

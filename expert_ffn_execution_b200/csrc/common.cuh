@@ -17,6 +17,14 @@ STRATA_DEVFN void dev_flag(int32_t* status, int32_t bit) {
   if (status) atomicOr(status, bit);
 }
 
+// fp16 bits of v (round to nearest); a finite v beyond the fp16 range becomes
+// +-inf and sets STRATA_DEV_OVERFLOW in *status.
+STRATA_DEVFN uint16_t f16_bits_checked(float v, int32_t* status) {
+  const __half h = __float2half_rn(v);
+  if (__hisinf(h) && isfinite(v)) dev_flag(status, STRATA_DEV_OVERFLOW);
+  return __half_as_ushort(h);
+}
+
 // ---------------------------------------------------------------- loads
 // Weights are streamed once: keep them out of L1.
 STRATA_DEVFN uint4 ld_stream_v4(const void* p) {

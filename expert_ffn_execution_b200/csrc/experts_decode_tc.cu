@@ -565,7 +565,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
           const float h = silu_f32(gv) * uv;
           const int ii = ti.rb * 64 + l;
           const int pos = (ii & ~15) + group_slot<FMT>(ii & 15);
-          p.hbuf[(size_t)(ti.s0 + j) * I + pos] = __half_as_ushort(__float2half_rn(h));
+          p.hbuf[(size_t)(ti.s0 + j) * I + pos] = f16_bits_checked(h, p.status);
         }
         if constexpr (MODE == 2) {
           // publish this thread's h stores (to the TMA reads of other CTAs)
@@ -804,8 +804,15 @@ cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, 
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   pdl_config(cfg, attr, grid, kTcThreads, smem, st);
+  if constexpr (MODE == 2) {
+    // The fused grid's CTAs wait on each other's counters: a cooperative
+    // launch guarantees that every CTA is resident, or fails to launch.
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.numAttrs = 2;
+  }
   return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], prm);
 }
 
@@ -904,8 +911,13 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
     prm.maxT = tc_max_tiles(2, Umax, a.H, a.I, a.num_sms);
     prm.S = tc_stages(2, a.fmt, NB, a.H, a.I, prm.maxT);
     if ((e = launch_sync_reset(a.sync, Umax, st)) != cudaSuccess) return e;
-    if (q2) return launch_tc<2, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
-    return launch_tc<2, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+    e = q2 ? launch_tc<2, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st)
+           : launch_tc<2, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+    // Where the grid cannot be resident all at once (SMs held by other work,
+    // a partitioned GPU), the cooperative launch is refused: clear the error
+    // and run the two-kernel form, which needs no co-residency.
+    if (e != cudaErrorCooperativeLaunchTooLarge) return e;
+    (void)cudaGetLastError();
   }
   prm.maxT = tc_max_tiles(0, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);

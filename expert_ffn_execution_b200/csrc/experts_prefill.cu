@@ -261,7 +261,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
             if (n < tl.n) {
               const float gv = __uint_as_float(g[j]), uv = __uint_as_float(uu[j]);
               const float h = silu_f32(gv) * uv;
-              out[(size_t)(tl.s0 + n) * I + mt * kPM + m] = __half_as_ushort(__float2half_rn(h));
+              out[(size_t)(tl.s0 + n) * I + mt * kPM + m] = f16_bits_checked(h, status);
             }
           }
         } else {
@@ -271,7 +271,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
             const int n = c0 + j;
             if (n < tl.n)
               out[(size_t)(tl.s0 + n) * H + mt * kPM + m] =
-                  __half_as_ushort(__float2half_rn(__uint_as_float(g[j])));
+                  f16_bits_checked(__uint_as_float(g[j]), status);
           }
         }
       }

@@ -32,7 +32,8 @@
  *   - `dev_status` (device int32, may be NULL where stated) is a sticky error
  *     word: kernels never trap; on a device-detected problem (a bounded wait
  *     that ran out, an index out of range) they OR a STRATA_DEV_* bit into it
- *     and skip the offending access.  Zero it once; read it with
+ *     and skip the offending access; an fp16 intermediate that overflowed
+ *     (stored as +-inf) is reported the same way.  Zero it once; read it with
  *     strata_read_status.
  *   - bf16 and fp16 values travel as uint16_t bit patterns.
  *   - Shapes: T tokens, H hidden, E experts, I expert width, k experts per
@@ -61,12 +62,16 @@ typedef enum strata_status {
   STRATA_ECUDA = 2,        /* a CUDA launch or API call failed */
   STRATA_EUNSUPPORTED = 3, /* valid but outside what the kernels implement */
   STRATA_ETIMEOUT = 4,     /* device-reported: a bounded wait ran out */
-  STRATA_EBOUNDS = 5       /* device-reported: an index was out of range */
+  STRATA_EBOUNDS = 5,      /* device-reported: an index was out of range */
+  STRATA_EOVERFLOW = 6     /* device-reported: an fp16 intermediate overflowed */
 } strata_status;
 
 /* Bits a kernel ORs into *dev_status. */
 #define STRATA_DEV_TIMEOUT 0x1
 #define STRATA_DEV_BOUNDS 0x2
+/* An fp16 intermediate (the SwiGLU output h of either path, or the prefill
+ * expert output y) exceeded the fp16 range and was stored as +-inf. */
+#define STRATA_DEV_OVERFLOW 0x4
 
 /* ---------------------------------------------------------------- formats
  * Block-quantised expert weights.  Each weight matrix is stored as
@@ -122,7 +127,8 @@ STRATA_API const char* strata_status_string(int32_t status);
 STRATA_API uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t inter);
 /* Reads *dev_status (device) into host memory: enqueues a copy on `stream` and
  * SYNCHRONISES that stream.  Returns STRATA_OK, STRATA_ETIMEOUT,
- * STRATA_EBOUNDS (the first set bit, timeout first) or STRATA_ECUDA. */
+ * STRATA_EBOUNDS, STRATA_EOVERFLOW (the first set bit in that order) or
+ * STRATA_ECUDA. */
 STRATA_API int32_t strata_read_status(const int32_t* dev_status, void* stream);
 
 /* Failure-detection self-test of the bounded device waits (the pages have

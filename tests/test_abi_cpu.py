@@ -38,6 +38,7 @@ def test_abi_version_and_status_strings():
     assert sm.abi_version() == 1
     assert sm.status_string(0) == "ok"
     assert sm.status_string(1) == "invalid argument"
+    assert sm.status_string(6) == "fp16 intermediate overflowed"
     assert sm.status_string(99) == "unknown status"
 
 

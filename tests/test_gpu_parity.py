@@ -21,6 +21,7 @@ if not torch.cuda.is_available():
 import expert_ffn_execution_b200 as sm  # noqa: E402
 import moe_inputs as mi  # noqa: E402
 import oracle  # noqa: E402
+from expert_ffn_execution_b200._binding import EOVERFLOW  # noqa: E402
 from tests.harness import (OUT_REL_L2, TOPK_W_ATOL, check_routing, logit_tol, parallel_rows,  # noqa: E402
                            rel_l2_rows, stratified_tokens)
 
@@ -218,6 +219,40 @@ def test_decode_large_down_scales():
     assert 0.2 < big < 0.9, big  # both forms are exercised
     r.run()
     check_layer(r)
+
+
+@pytest.mark.parametrize("T", [4, 64])
+def test_fp16_overflow_flagged(T):
+    """Gate/up block scales times 2^12 push the SwiGLU output h past the fp16
+    range: h is stored as inf and the call reports STRATA_EOVERFLOW (decode at
+    T = 4, prefill at T = 64)."""
+    c = mi.CONFIGS[1]
+    inp = mi.make_layer(1, T, layer=0, device=DEV)
+    planes, _ = mi.plane_layout(c.fmt, c.H, c.I)
+    for name in ("gate", "up"):
+        _, off, n, _, _, _ = [pl for pl in planes if pl[0] == name and pl[5] == "scales"][0]
+        inp.experts[:, off:off + n].view(torch.float16).mul_(2.0 ** 12)
+    H, E, k, I = c.H, inp.w_router.shape[1], c.k, c.I
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    hid = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offs = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(T * k, dtype=torch.int32, device=DEV)
+    act = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    rw = ws(sm.moe_route_workspace_size(T, H, E, k))
+    sm.moe_route(inp.x, T, H, c.eps, inp.w_router, inp.bias, E, k, hid, ids, w, counts, offs,
+                 perm, inv, act, rw, rw.numel(), st)
+    assert sm.strata_read_status(st) == 0
+    qw = sm.qweights(c.fmt, E, H, I, inp.experts, inp.experts.stride(0))
+    decode = T <= sm.DECODE_MAX_T
+    y = torch.empty(T * k, H, dtype=torch.float32 if decode else torch.float16, device=DEV)
+    ew = ws(sm.moe_experts_workspace_size(qw, T, k))
+    sm.moe_experts(hid, qw, offs, perm, act, T, k, y, ew, ew.numel(), st)
+    torch.cuda.synchronize()
+    assert sm.strata_read_status(st) == EOVERFLOW
 
 
 @pytest.mark.parametrize("config,T", [(1, 4), (4, 8)])
