@@ -10,10 +10,13 @@ include/strata_moe.h):
                down codes | down scales, each plane on a 256-byte boundary;
   gate/up are [I rows x H], down is [H rows x I]; codes are uint8 planes
   ([N][K/4] for the 2-bit format, [N][K/2] for the 4-bit codebook format),
-  scales are fp16 [N][K/32].
+  scales are fp16 [N][K/32], or for the MXFP4 format (4-bit E2M1 codes laid
+  out like the 4-bit codebook format) one E8M0 byte per block, [N][K/32].
 
 Random codes are uniform bytes, which makes every 2-bit code uniform in 0..3
-and every 4-bit code uniform in 0..15.  Scales are U[lo, hi] rounded to fp16.
+and every 4-bit code uniform in 0..15.  Scales are U[lo, hi] rounded to fp16;
+MXFP4 scales are E8M0 exponents e uniform over the integers with 2^(e-127) in
+[lo, hi] (lo and hi powers of two).
 
 Workloads (the five layer configurations this library is measured on):
   C0  H=2560 E=512 I=640 k=10, T=1, 2-bit experts d~U[0.005,0.02], no bias
@@ -23,6 +26,8 @@ Workloads (the five layer configurations this library is measured on):
       d~U[0.0005,0.002]; also T=1 and T=4
   C4  H=4096 E=256 I=2048 k=6, 4-bit codebook routed + shared experts,
       d~U[0.0005,0.002], Zipf(s=1.0) bias, x rounded to bf16; T=1, 4, 8192
+  C6  the C1/C2 layer with MXFP4 routed experts, scales 2^-9..2^-6, Zipf(s=1.1)
+      bias; T=1, 4, 8192 (the native-MXFP4 model tier's expert format)
 x ~ N(0,1) fp32 (then RMSNorm inside the layer); W_r ~ N(0, 0.02) bf16 [H, E].
 Zipf bias: a seeded permutation gives each expert a popularity rank r in
 1..E and bias[e] = -0.5 * s * ln(r_e) (half the log of a Zipf(s) probability,
@@ -37,6 +42,7 @@ import torch
 
 FMT_Q2 = 1
 FMT_Q4CB = 2
+FMT_MXFP4 = 3
 
 
 def _round256(x: int) -> int:
@@ -46,7 +52,7 @@ def _round256(x: int) -> int:
 def plane_layout(fmt: int, H: int, I: int):
     """[(name, offset, nbytes, rows, K, kind)] for the six planes, and the
     blob size.  kind is 'codes' or 'scales'."""
-    if fmt not in (FMT_Q2, FMT_Q4CB):
+    if fmt not in (FMT_Q2, FMT_Q4CB, FMT_MXFP4):
         raise ValueError(f"unknown format {fmt}")
     if H % 32 or I % 32:
         raise ValueError("H and I must be multiples of 32")
@@ -56,7 +62,7 @@ def plane_layout(fmt: int, H: int, I: int):
         nc = rows * (K // 4 if fmt == FMT_Q2 else K // 2)
         planes.append((name, off, nc, rows, K, "codes"))
         off = _round256(off + nc)
-        ns = rows * (K // 32) * 2
+        ns = rows * (K // 32) * (1 if fmt == FMT_MXFP4 else 2)
         planes.append((name, off, ns, rows, K, "scales"))
         off = _round256(off + ns)
     return planes, off
@@ -104,6 +110,8 @@ CONFIGS = {
     5: LayerConfig("C3b", 2560, 512, 640, 10, FMT_Q4CB, (0.0005, 0.002), (1, 4),
                    zipf_s=1.1, shared_fmt=FMT_Q4CB, shared_d_range=(0.0005, 0.002),
                    notes="C3 with 4-bit-codebook routed experts"),
+    6: LayerConfig("C6", 2560, 512, 640, 10, FMT_MXFP4, (2.0**-9, 2.0**-6), (1, 4, 8192),
+                   zipf_s=1.1, notes="C1/C2 layer with MXFP4 routed experts"),
 }
 
 
@@ -142,7 +150,8 @@ def gen_zipf_bias(E: int, s: float, seed: int, device="cpu") -> torch.Tensor:
 def gen_experts(fmt: int, E: int, H: int, I: int, d_range, seed: int, device="cpu",
                 out: torch.Tensor | None = None) -> torch.Tensor:
     """E expert blobs as uint8 [E, expert_bytes]: uniform random code bytes,
-    fp16 scales U[lo, hi].  Writes into `out` if given."""
+    fp16 scales U[lo, hi] (MXFP4: E8M0 bytes for the powers of two in
+    [lo, hi]).  Writes into `out` if given."""
     planes, nbytes = plane_layout(fmt, H, I)
     if out is None:
         out = torch.empty(E, nbytes, dtype=torch.uint8, device=device)
@@ -154,6 +163,11 @@ def gen_experts(fmt: int, E: int, H: int, I: int, d_range, seed: int, device="cp
         if kind == "codes":
             out[:, off:off + n] = torch.randint(0, 256, (E, n), generator=g, device=out.device,
                                                 dtype=torch.uint8)
+        elif fmt == FMT_MXFP4:
+            e_lo = 127 + int(round(math.log2(lo)))
+            e_hi = 127 + int(round(math.log2(hi)))
+            out[:, off:off + n] = torch.randint(e_lo, e_hi + 1, (E, n), generator=g,
+                                                device=out.device, dtype=torch.uint8)
         else:
             cnt = n // 2
             d = torch.rand(E, cnt, generator=g, device=out.device, dtype=torch.float32)

@@ -22,6 +22,7 @@ _LIB_OVERRIDE = os.environ.get("STRATA_ORACLE_LIB")
 
 FMT_Q2 = 1
 FMT_Q4CB = 2
+FMT_MXFP4 = 3
 
 
 def build(force: bool = False) -> str:

@@ -36,11 +36,24 @@
  *                   k, high nibble for odd k; w = d * KV[c] with the 16-entry
  *                   non-linear codebook below (the IQ4_NL table named by the
  *                   Strata walk-through, section 13)
+ *   fmt 3, MXFP4_32: the OCP Microscaling (MX) v1.0 MXFP4 format, the
+ *                   experts of the native-MXFP4 model tier (lcz.me/topic/2153,
+ *                   model tier list, "ds4f-mxfp4"; the llama.cpp MXFP4 GGUF
+ *                   line on the same page).  Element codes as in fmt 2 (one
+ *                   nibble per element, low nibble for even k), each an FP4
+ *                   E2M1 number: bit 3 sign, bits 2-1 exponent (bias 1),
+ *                   bit 0 mantissa, exponent 0 subnormal; the block scale is
+ *                   one E8M0 byte e (no sign, no mantissa): 2^(e-127), e = 255
+ *                   is NaN.  w = e2m1(c) * 2^(e-127).  The scales plane holds
+ *                   one byte per block instead of two.
  *   Expert blob: gate codes | gate scales | up codes | up scales | down codes |
  *   down scales, each plane starting on a 256-byte boundary.  gate and up are
  *   [I rows x H], down is [H rows x I].
- * Dequantisation is exact in fp32: d has 11 significant bits and the code
- * value at most 8, so the product fits in 24 bits.
+ * Dequantisation is exact in fp32 for fmt 1 and 2: d has 11 significant bits
+ * and the code value at most 8, so the product fits in 24 bits.  For fmt 3
+ * the product is formed in double (exact: two significant bits times a power
+ * of two) and rounded once to fp32, which is exact unless it leaves fp32's
+ * range (e >= 253).
  *
  * Pins (tests/test_oracle_pins.py): hand-built blocks with known values,
  * brute-force top-k on tiny inputs, the k = E identical-expert identity with a
@@ -111,9 +124,21 @@ static size_t round_up_256(size_t x) { return (x + 255) & ~(size_t)255; }
 static size_t codes_plane_bytes(int fmt, int rows, int K) {
   return fmt == 1 ? (size_t)rows * (size_t)(K / 4) : (size_t)rows * (size_t)(K / 2);
 }
-static size_t scales_plane_bytes(int rows, int K) {
-  return (size_t)rows * (size_t)(K / 32) * 2;
+/* fp16 scales for fmt 1 and 2, one E8M0 byte for fmt 3 */
+static size_t scales_plane_bytes(int fmt, int rows, int K) {
+  return (size_t)rows * (size_t)(K / 32) * (fmt == 3 ? 1 : 2);
 }
+
+/* OCP MX v1.0 FP4 (E2M1) element value, from the field definition. */
+static double e2m1_value(int c) {
+  const int sign = (c >> 3) & 1, ex = (c >> 1) & 3, man = c & 1;
+  const double mag = ex == 0 ? 0.5 * man                    /* subnormal: m * 2^(1-bias) / 2 */
+                             : ldexp(1.0 + 0.5 * man, ex - 1); /* (1 + m/2) * 2^(ex-bias) */
+  return sign ? -mag : mag;
+}
+
+/* OCP MX v1.0 E8M0 scale value: 2^(e-127); 255 encodes NaN. */
+static double e8m0_value(int e) { return e == 255 ? NAN : ldexp(1.0, e - 127); }
 
 /* Offsets of the six planes of one expert blob.  which: 0 gate, 1 up, 2 down. */
 static void plane_offsets(int fmt, int H, int I, int which, size_t* codes_off,
@@ -125,7 +150,7 @@ static void plane_offsets(int fmt, int H, int I, int which, size_t* codes_off,
     size_t c = off;
     off = round_up_256(off + codes_plane_bytes(fmt, r, k));
     size_t s = off;
-    off = round_up_256(off + scales_plane_bytes(r, k));
+    off = round_up_256(off + scales_plane_bytes(fmt, r, k));
     if (m == which) {
       *codes_off = c;
       *scales_off = s;
@@ -141,7 +166,7 @@ size_t oracle_expert_bytes(int fmt, int H, int I) {
     int r = (m == 2) ? H : I;
     int k = (m == 2) ? I : H;
     off = round_up_256(off + codes_plane_bytes(fmt, r, k));
-    off = round_up_256(off + scales_plane_bytes(r, k));
+    off = round_up_256(off + scales_plane_bytes(fmt, r, k));
   }
   return off;
 }
@@ -152,17 +177,22 @@ int oracle_version(void) { return ORACLE_VERSION; }
  * blob into K floats.  Returns 0, or -1 on a bad argument. */
 int oracle_dequant_row(int fmt, const uint8_t* blob, int H, int I, int which,
                        int row, float* out) {
-  if ((fmt != 1 && fmt != 2) || which < 0 || which > 2 || H % 32 || I % 32) return -1;
+  if (fmt < 1 || fmt > 3 || which < 0 || which > 2 || H % 32 || I % 32) return -1;
   size_t co = 0, so = 0;
   int rows = 0, K = 0;
   plane_offsets(fmt, H, I, which, &co, &so, &rows, &K);
   if (row < 0 || row >= rows) return -1;
   const uint8_t* codes = blob + co + codes_plane_bytes(fmt, 1, K) * (size_t)row;
-  const uint8_t* scales = blob + so + scales_plane_bytes(1, K) * (size_t)row;
+  const uint8_t* scales = blob + so + scales_plane_bytes(fmt, 1, K) * (size_t)row;
   for (int k = 0; k < K; ++k) {
+    float w;
+    if (fmt == 3) {
+      int c = (codes[k / 2] >> (4 * (k % 2))) & 15;
+      out[k] = (float)(e2m1_value(c) * e8m0_value(scales[k / 32]));
+      continue;
+    }
     uint16_t dbits = (uint16_t)(scales[2 * (k / 32)] | (scales[2 * (k / 32) + 1] << 8));
     float d = half_to_float(dbits);
-    float w;
     if (fmt == 1) {
       int c = (codes[k / 4] >> (2 * (k % 4))) & 3;
       w = d * ((float)c - 1.5f);

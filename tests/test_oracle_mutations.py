@@ -34,6 +34,13 @@ MUTATIONS = {
     "gate_up_planes_swapped": ("if (m == which) {", "if (m == (which < 2 ? 1 - which : 2)) {"),
     "scale_block_size": ("uint16_t dbits = (uint16_t)(scales[2 * (k / 32)] | (scales[2 * (k / 32) + 1] << 8));",
                          "uint16_t dbits = (uint16_t)(scales[2 * (k / 64)] | (scales[2 * (k / 64) + 1] << 8));"),
+    "mxfp4_nibble_order": (">> (4 * (k % 2))) & 15;", ">> (4 - 4 * (k % 2))) & 15;"),
+    "mxfp4_e2m1_bias": ("ldexp(1.0 + 0.5 * man, ex - 1)", "ldexp(1.0 + 0.5 * man, ex)"),
+    "mxfp4_e2m1_subnormal": ("ex == 0 ? 0.5 * man", "ex == 0 ? 1.0 * man"),
+    "mxfp4_sign_bit": ("const int sign = (c >> 3) & 1,", "const int sign = (c >> 2) & 1,"),
+    "mxfp4_e8m0_bias": ("ldexp(1.0, e - 127); }", "ldexp(1.0, e - 128); }"),
+    "mxfp4_e8m0_nan": ("e == 255 ? NAN :", "e == 256 ? NAN :"),
+    "mxfp4_scale_width": ("(fmt == 3 ? 1 : 2)", "2"),
 }
 
 

@@ -15,10 +15,16 @@ import numpy as np
 import pytest
 
 import oracle
-from oracle import FMT_Q2, FMT_Q4CB, bf16_bits_to_f32, f32_to_bf16_bits
+from oracle import FMT_MXFP4, FMT_Q2, FMT_Q4CB, bf16_bits_to_f32, f32_to_bf16_bits
 
 KV = np.array([-127, -104, -83, -65, -49, -35, -22, -10, 1, 13, 25, 38, 53, 69, 89, 113],
               np.float64)
+# FP4 E2M1 values of codes 0..15, read off the OCP MX v1.0 element table
+E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6], np.float64)
+
+
+def scale_bytes(fmt):
+    return 1 if fmt == FMT_MXFP4 else 2
 
 
 # ------------------------------------------------------------ independent decoder
@@ -32,7 +38,7 @@ def np_layout(fmt, H, I):
         out[name] = (off, None, rows, K)
         off = r256(off + nc)
         out[name] = (out[name][0], off, rows, K)
-        off = r256(off + rows * K // 32 * 2)
+        off = r256(off + rows * K // 32 * scale_bytes(fmt))
     return out, off
 
 
@@ -40,7 +46,12 @@ def np_dequant(fmt, blob, H, I, name):
     """Vectorised float64 decode of one matrix [rows, K]."""
     lay, _ = np_layout(fmt, H, I)
     co, so, rows, K = lay[name]
-    d = blob[so:so + rows * K // 32 * 2].view(np.float16).astype(np.float64).reshape(rows, K // 32)
+    if fmt == FMT_MXFP4:
+        e = blob[so:so + rows * K // 32].astype(np.int64).reshape(rows, K // 32)
+        d = np.where(e == 255, np.nan, np.ldexp(1.0, e - 127))
+    else:
+        d = blob[so:so + rows * K // 32 * 2].view(np.float16).astype(np.float64).reshape(
+            rows, K // 32)
     if fmt == FMT_Q2:
         b = blob[co:co + rows * K // 4].reshape(rows, K // 4)
         c = np.stack([(b >> (2 * i)) & 3 for i in range(4)], axis=-1).reshape(rows, K)
@@ -48,7 +59,7 @@ def np_dequant(fmt, blob, H, I, name):
     else:
         b = blob[co:co + rows * K // 2].reshape(rows, K // 2)
         c = np.stack([b & 15, b >> 4], axis=-1).reshape(rows, K)
-        v = KV[c]
+        v = (E2M1 if fmt == FMT_MXFP4 else KV)[c]
     return v * np.repeat(d, 32, axis=1)
 
 
@@ -56,6 +67,11 @@ def rand_blob(rng, fmt, H, I, d_lo=0.005, d_hi=0.02):
     lay, n = np_layout(fmt, H, I)
     blob = rng.integers(0, 256, n, dtype=np.uint8)
     for name, (co, so, rows, K) in lay.items():
+        if fmt == FMT_MXFP4:  # E8M0 exponents, d_lo..d_hi read as powers of two
+            e = rng.integers(127 + int(math.log2(d_lo)), 128 + int(math.log2(d_hi)),
+                             rows * K // 32)
+            blob[so:so + rows * K // 32] = e.astype(np.uint8)
+            continue
         d = rng.uniform(d_lo, d_hi, rows * K // 32).astype(np.float16)
         blob[so:so + d.nbytes] = d.view(np.uint8)
     return blob
@@ -83,17 +99,22 @@ def blob_with_first_row(fmt, H, I, which, codes, scale_bits):
     blob = np.zeros(n, np.uint8)
     co, so, rows, K = lay[("gate", "up", "down")[which]]
     blob[co:co + len(codes)] = np.frombuffer(codes, np.uint8)
-    blob[so:so + 2] = np.array([scale_bits], np.uint16).view(np.uint8)
+    if fmt == FMT_MXFP4:
+        blob[so] = scale_bits
+    else:
+        blob[so:so + 2] = np.array([scale_bits], np.uint16).view(np.uint8)
     return blob
 
 
 # ------------------------------------------------------------ dequantisation
-@pytest.mark.parametrize("fmt,fname", [(FMT_Q2, "q2_blocks.txt"), (FMT_Q4CB, "q4cb_blocks.txt")])
+@pytest.mark.parametrize("fmt,fname", [(FMT_Q2, "q2_blocks.txt"), (FMT_Q4CB, "q4cb_blocks.txt"),
+                                      (FMT_MXFP4, "mxfp4_blocks.txt")])
 @pytest.mark.parametrize("which", [0, 1, 2])
 def test_dequant_hand_built_blocks(golden_dir, fmt, fname, which):
     """Known codes and scales decode to the hand-worked values in every matrix.
     Catches: wrong bit/nibble order, wrong offset (-1.5), wrong codebook entry,
-    wrong fp16 decode, wrong plane offsets for gate/up/down."""
+    wrong fp16 decode, wrong plane offsets for gate/up/down; for MXFP4 a wrong
+    E2M1 field split, exponent bias, subnormal value, sign, or E8M0 bias/NaN."""
     H, I = 64, 32
     for name, codes, sbits, expect in read_golden(os.path.join(golden_dir, fname)):
         blob = blob_with_first_row(fmt, H, I, which, codes, sbits)
@@ -103,11 +124,12 @@ def test_dequant_hand_built_blocks(golden_dir, fmt, fname, which):
 
 def test_dequant_matches_independent_decoder():
     """The oracle's row decode equals the numpy decoder on random blobs, all
-    rows of all three matrices, both formats (exact)."""
+    rows of all three matrices, every format (exact)."""
     rng = np.random.default_rng(1)
-    for fmt in (FMT_Q2, FMT_Q4CB):
+    for fmt in (FMT_Q2, FMT_Q4CB, FMT_MXFP4):
         H, I = 96, 64
-        blob = rand_blob(rng, fmt, H, I)
+        blob = rand_blob(rng, fmt, H, I, *((2.0**-9, 2.0**-6) if fmt == FMT_MXFP4
+                                           else (0.005, 0.02)))
         for which, name in enumerate(("gate", "up", "down")):
             ref = np_dequant(fmt, blob, H, I, name)
             got = np.stack([oracle.dequant_row(fmt, blob, H, I, which, r)
@@ -129,6 +151,36 @@ def test_dequant_planes_are_distinct():
     for which, scale in enumerate((1.0, 2.0, 4.0)):
         row = oracle.dequant_row(FMT_Q2, blob, H, I, which, 1)
         assert np.all(row == np.float32(1.5 * scale))
+
+
+def test_mxfp4_sign_and_scale_steps():
+    """MXFP4 properties fixed by the format: setting a code's bit 3 negates
+    the element; adding 1 to a block's E8M0 byte doubles its 32 elements
+    exactly and leaves the other blocks alone; codes 0..7 increase strictly.
+    Catches: sign taken from the wrong bit, a scale indexed by the wrong
+    block, a scale that is not a power of two."""
+    rng = np.random.default_rng(11)
+    H, I = 96, 64
+    blob = rand_blob(rng, FMT_MXFP4, H, I, 2.0**-9, 2.0**-6)
+    lay, _ = np_layout(FMT_MXFP4, H, I)
+    for which, name in enumerate(("gate", "up", "down")):
+        co, so, rows, K = lay[name]
+        r = 3
+        base = oracle.dequant_row(FMT_MXFP4, blob, H, I, which, r).astype(np.float64)
+        neg = blob.copy()
+        neg[co + r * K // 2:co + (r + 1) * K // 2] ^= 0x88
+        np.testing.assert_array_equal(
+            oracle.dequant_row(FMT_MXFP4, neg, H, I, which, r), -base)
+        dbl = blob.copy()
+        dbl[so + r * K // 32 + 1] += 1
+        got = oracle.dequant_row(FMT_MXFP4, dbl, H, I, which, r).astype(np.float64)
+        np.testing.assert_array_equal(got[32:64], 2 * base[32:64])
+        np.testing.assert_array_equal(np.delete(got, np.s_[32:64]), np.delete(base, np.s_[32:64]))
+    mono = blob.copy()
+    co, so, rows, K = lay["gate"]
+    mono[co:co + 4] = [0x10, 0x32, 0x54, 0x76]
+    v = oracle.dequant_row(FMT_MXFP4, mono, H, I, 0, 0)[:8]
+    assert np.all(np.diff(v) > 0) and v[0] == 0
 
 
 # ------------------------------------------------------------ sizes
@@ -161,6 +213,9 @@ def test_blob_sizes_closed_form():
     planes are already 256-byte multiples; 48 x 512 Q2 experts ~ 38 GB."""
     assert oracle.expert_bytes(FMT_Q2, 2560, 640) == 3 * 2560 * 640 * 5 // 16 == 1536000
     assert oracle.expert_bytes(FMT_Q4CB, 2560, 640) == 3 * 2560 * 640 * 9 // 16 == 2764800
+    # MXFP4: 4 bits per element and an 8-bit scale per 32 -> 4.25 bits/weight
+    assert oracle.expert_bytes(FMT_MXFP4, 2560, 640) == 3 * 2560 * 640 * 17 // 32 == 2611200
+    assert oracle.expert_bytes(FMT_MXFP4, 4096, 2048) == 3 * 4096 * 2048 * 17 // 32
     assert oracle.expert_bytes(FMT_Q4CB, 4096, 2048) == 14155776
     assert round(48 * 512 * 1536000 / 2**30, 2) == 35.16  # 37.75 GB
     assert oracle.expert_bytes(FMT_Q2, 64, 32) == np_layout(FMT_Q2, 64, 32)[1]
@@ -286,7 +341,10 @@ def textbook_mlp(fmt, blob, H, I, x_bits):
     return wd @ (g / (1 + np.exp(-g)) * u)
 
 
-@pytest.mark.parametrize("fmt", [FMT_Q2, FMT_Q4CB])
+D_RANGE = {FMT_Q2: (0.005, 0.02), FMT_Q4CB: (0.0005, 0.002), FMT_MXFP4: (2.0**-9, 2.0**-6)}
+
+
+@pytest.mark.parametrize("fmt", [FMT_Q2, FMT_Q4CB, FMT_MXFP4])
 def test_expert_ffn_matches_textbook_mlp(fmt):
     """E = 1: one expert equals the float64 SwiGLU MLP y = Wd (silu(Wg x) * Wu x)
     built from the independent decoder, with H != I so a transposed operand
@@ -294,7 +352,7 @@ def test_expert_ffn_matches_textbook_mlp(fmt):
     rng = np.random.default_rng(6)
     H, I = 96, 64
     for _ in range(3):
-        blob = rand_blob(rng, fmt, H, I, *((0.005, 0.02) if fmt == FMT_Q2 else (0.0005, 0.002)))
+        blob = rand_blob(rng, fmt, H, I, *D_RANGE[fmt])
         x = rand_hidden(rng, 1, H)[0]
         ref = textbook_mlp(fmt, blob, H, I, x)
         y32 = oracle.expert_ffn(fmt, blob, H, I, x, acc64=False).astype(np.float64)
