@@ -6,7 +6,7 @@ under the same name.  Build the library with
 """
 from ._binding import (DECODE_MAX_T, DEV_BOUNDS, DEV_TIMEOUT, DTYPE_BF16, DTYPE_F16, DTYPE_F32,
                        FMT_Q2_32,
-                       FMT_Q4CB_32, QWeights, StrataError, abi_version, exported_symbols, load,
+                       FMT_MXFP4_32, FMT_Q4CB_32, QWeights, StrataError, abi_version, exported_symbols, load,
                        moe_bucket, moe_bucket_workspace_size, moe_combine, moe_experts,
                        moe_experts_static_scratch, moe_gather_rows,
                        moe_experts_workspace_size, moe_layer_forward, moe_layer_workspace_size,

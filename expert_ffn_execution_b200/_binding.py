@@ -15,6 +15,7 @@ LIB_PATH = os.path.join(HERE, "libstrata_moe.so")
 OK, EINVAL, ECUDA, EUNSUPPORTED, ETIMEOUT, EBOUNDS, EOVERFLOW = range(7)
 FMT_Q2_32 = 1
 FMT_Q4CB_32 = 2
+FMT_MXFP4_32 = 3
 DTYPE_F32 = 0
 DTYPE_F16 = 1
 DTYPE_BF16 = 2

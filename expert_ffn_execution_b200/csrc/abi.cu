@@ -33,7 +33,7 @@ uint64_t up256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
 
 bool valid_weights(const strata_qweights* w) {
   if (!w || !w->base) return false;
-  if (w->fmt != STRATA_FMT_Q2_32 && w->fmt != STRATA_FMT_Q4CB_32) return false;
+  if (w->fmt < STRATA_FMT_Q2_32 || w->fmt > STRATA_FMT_MXFP4_32) return false;
   if (w->num_experts < 1 || w->hidden < 128 || w->inter < 128) return false;
   if (w->hidden % 128 || w->inter % 128) return false;
   if (!aligned(w->base, 256) || w->expert_stride % 256) return false;
@@ -43,9 +43,10 @@ bool valid_weights(const strata_qweights* w) {
 }
 
 // Decode-path support: gate/up K steps of 256, down K steps of 128, down
-// tasks of 64 rows.
+// tasks of 64 rows; MXFP4 gate/up scale rows in whole 16-byte units.
 bool decode_supported(const strata_qweights* w) {
-  return w->hidden % 256 == 0 && w->inter % 128 == 0 && w->hidden % 64 == 0;
+  return w->hidden % 256 == 0 && w->inter % 128 == 0 && w->hidden % 64 == 0 &&
+         (w->fmt != STRATA_FMT_MXFP4_32 || w->hidden % 512 == 0);
 }
 
 // Decode scratch: h fp16 [P, I], then one progress counter per active
@@ -149,7 +150,7 @@ const char* strata_status_string(int32_t s) {
 }
 
 uint64_t strata_expert_bytes(int32_t fmt, int32_t hidden, int32_t inter) {
-  if (fmt != STRATA_FMT_Q2_32 && fmt != STRATA_FMT_Q4CB_32) return 0;
+  if (fmt < STRATA_FMT_Q2_32 || fmt > STRATA_FMT_MXFP4_32) return 0;
   if (hidden <= 0 || inter <= 0 || hidden % 32 || inter % 32) return 0;
   uint64_t total = 0;
   plane_offsets(fmt, hidden, inter, &total);

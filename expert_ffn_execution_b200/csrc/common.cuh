@@ -46,6 +46,11 @@ STRATA_DEVFN uint32_t ld_stream_u32(const void* p) {
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
   return v;
 }
+STRATA_DEVFN uint32_t ld_stream_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
 
 // ---------------------------------------------------------------- packing
 STRATA_DEVFN uint32_t h2_as_u32(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }

@@ -134,7 +134,7 @@ __host__ __device__ inline TcLayout tc_layout(int mode, int fmt, int NB, int H, 
   L.hb_bytes = dn ? (uint32_t)NB * (uint32_t)I * 2u : 0u;
   off += 2u * L.hb_bytes;
   L.sbuf = off;
-  L.s_bytes = dn ? up1k(8u * (uint32_t)I) : 0u;
+  L.s_bytes = dn ? up1k(128u * (uint32_t)scales_row_bytes(fmt, I)) : 0u;
   off += 2u * L.s_bytes;
   L.xch = off;
   off += gu ? up1k(2u * 64u * 17u * 4u) : 0u;
@@ -178,6 +178,11 @@ STRATA_DEVFN uint4 lds128(const void* p) {
   asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "r"(smem_addr(p)));
+  return v;
+}
+STRATA_DEVFN uint32_t lds32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(smem_addr(p)));
   return v;
 }
 STRATA_DEVFN uint2 lds64(const void* p) {
@@ -406,7 +411,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
             // gate rows rb*64.. then the same up rows: one box over both
             // planes for the codes, one for the scales
             tma_load_4d(st, &mg, c * CBR, rb * 64, 0, e, &full[s]);
-            tma_load_4d(st + L.codes_bytes, &msg, c * 8, rb * 64, 0, e, &full[s]);
+            // scales: 16 bytes per row, the chunk's 8 fp16 values, or for
+            // MXFP4 the 16 E8M0 bytes of the chunk pair starting at an even
+            // chunk (a box must start on a 16-byte boundary)
+            tma_load_4d(st + L.codes_bytes, &msg, FMT == STRATA_FMT_MXFP4_32 ? (c & ~1) * 8 : c * 8,
+                        rb * 64, 0, e, &full[s]);
           }
           continue;
         }
@@ -424,11 +433,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
           // the tile's scales: rows rb*128.. of the down plane, all of K
           const int sb = ib & 1;
           mbar_wait_guarded(&sempty[sb], ((ib >> 1) & 1) ^ 1, p.status, abort_flag);
-          mbar_arrive_expect_tx(&sfull[sb], 8u * I);
+          const uint32_t sblk = 128u * (uint32_t)scales_row_bytes(FMT, I);
+          mbar_arrive_expect_tx(&sfull[sb], sblk);
           bulk_g2s(smem + L.sbuf + sb * L.s_bytes,
-                   p.wbase + (uint64_t)e * p.stride + PL.scales[2] +
-                       (uint64_t)rb * 128u * (uint64_t)(I / 16),
-                   8u * I, &sfull[sb]);
+                   p.wbase + (uint64_t)e * p.stride + PL.scales[2] + (uint64_t)rb * sblk, sblk,
+                   &sfull[sb]);
           auto issue_b = [&](int c) {
             const int s = next_stage(L.codes_bytes);
             tma_load_3d(smem + s * L.stage_bytes, &md, c * CBR, rb * 128, e, &full[s]);
@@ -600,7 +609,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
       const uint8_t* srow = nullptr;
       if (!isA) {
         mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
-        srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (I / 16);
+        srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (int)scales_row_bytes(FMT, I);
       }
       for (int c = 0; c < nch; ++c, ++gc) {
         if (gc % kTcGroups != g) continue;
@@ -614,7 +623,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         for (int pc = 0; pc < NPC; ++pc)
           cw[pc] = (pc < np) ? lds128(st + r * CBR + ((pc ^ swz) << 4)) : make_uint4(0, 0, 0, 0);
         uint32_t sc[4];
-        if (isA) {
+        if constexpr (FMT == STRATA_FMT_MXFP4_32) {
+          // 8 E8M0 bytes, one per 32-K piece
+          if (isA) {
+            const uint2 v = lds64(st + L.codes_bytes + r * 16 + (c & 1) * 8);
+            sc[0] = v.x;
+            sc[1] = v.y;
+          } else {  // rows of I/32 bytes: 4-byte aligned
+            sc[0] = lds32(srow + c * 8);
+            sc[1] = kv > 128 ? lds32(srow + c * 8 + 4) : 0u;
+          }
+          sc[2] = sc[3] = 0;
+        } else if (isA) {
           const uint4 v = lds128(st + L.codes_bytes + r * 16);
           sc[0] = v.x;
           sc[1] = v.y;
@@ -652,6 +672,19 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
               dq_q2_word(cw[pc].z, d1, R + 16);
               dq_q2_word(cw[pc].w, d1, R + 24);
               tmem_st32(ta + pc * 32, R);
+            }
+          }
+        } else if constexpr (FMT == STRATA_FMT_MXFP4_32) {
+#pragma unroll
+          for (int pc = 0; pc < NPC; ++pc) {
+            if (pc < np) {
+              uint32_t R[16];
+              const uint32_t d2 = mx_scale_h2((sc[pc >> 2] >> (8 * (pc & 3))) & 0xFFu);
+              dq_mx_word(cw[pc].x, d2, R);
+              dq_mx_word(cw[pc].y, d2, R + 4);
+              dq_mx_word(cw[pc].z, d2, R + 8);
+              dq_mx_word(cw[pc].w, d2, R + 12);
+              tmem_st16(ta + pc * 16, R);
             }
           }
         } else {
@@ -816,6 +849,17 @@ cudaError_t launch_tc(const CUtensorMap (&m)[6], const TcParams& prm, int grid, 
   return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], m[5], prm);
 }
 
+template <int MODE>
+cudaError_t launch_tc_fmt(int fmt, const CUtensorMap (&m)[6], const TcParams& prm, int grid,
+                          cudaStream_t st) {
+  switch (fmt) {
+    case STRATA_FMT_Q2_32: return launch_tc<MODE, STRATA_FMT_Q2_32>(m, prm, grid, st);
+    case STRATA_FMT_Q4CB_32: return launch_tc<MODE, STRATA_FMT_Q4CB_32>(m, prm, grid, st);
+    case STRATA_FMT_MXFP4_32: return launch_tc<MODE, STRATA_FMT_MXFP4_32>(m, prm, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
 cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
@@ -834,6 +878,8 @@ bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
 
 bool decode_tc_supported(int T, int H, int I, int Umax, int fmt, int grid) {
   if (T < 1 || T > kDecodeMaxTokens || H % 256 || I % 128 || grid < 1 || Umax < 1) return false;
+  // MXFP4 gate/up scale rows (H/32 bytes) are a tensor-map stride: whole 16 bytes
+  if (fmt == STRATA_FMT_MXFP4_32 && H % 512) return false;
   const int NB = T <= 8 ? 8 : 16;
   return tc_stages(0, fmt, NB, H, I, tc_max_tiles(0, Umax, H, I, grid)) >= kTcGroups &&
          tc_stages(1, fmt, NB, H, I, tc_max_tiles(1, Umax, H, I, grid)) >= kTcGroups;
@@ -846,8 +892,7 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   if (!decode_tc_supported(a.T, a.H, a.I, Umax, a.fmt, a.num_sms)) return cudaErrorNotSupported;
   const int NB = a.T <= 8 ? 8 : 16;
   const Planes PL = plane_offsets(a.fmt, a.H, a.I);
-  const bool q2 = a.fmt == STRATA_FMT_Q2_32;
-  const cuuint32_t cbr = q2 ? kTcKC / 4 : kTcKC / 2;
+  const cuuint32_t cbr = a.fmt == STRATA_FMT_Q2_32 ? kTcKC / 4 : kTcKC / 2;
   const CUtensorMapSwizzle sw = cbr == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
   const cuuint64_t rowH = codes_row_bytes(a.fmt, a.H), rowI = codes_row_bytes(a.fmt, a.I);
   CUtensorMap m[6];  // gate codes, up codes, gate scales, up scales, down codes, h
@@ -864,11 +909,14 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
     m[1] = m[0];
   }
   {
+    // 16 bytes per row and box: 8 fp16 scales, or 16 E8M0 bytes (two chunks)
+    const bool mx = a.fmt == STRATA_FMT_MXFP4_32;
     const cuuint64_t dims[4] = {(cuuint64_t)a.H / 32, (cuuint64_t)a.I, 2, (cuuint64_t)E};
-    const cuuint64_t str[3] = {(cuuint64_t)a.H / 16, PL.scales[1] - PL.scales[0], a.stride};
-    const cuuint32_t box[4] = {8, 64, 2, 1};
-    if (!make_tmap(&m[2], CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, a.wbase + PL.scales[0], dims, str,
-                   box, CU_TENSOR_MAP_SWIZZLE_NONE))
+    const cuuint64_t str[3] = {scales_row_bytes(a.fmt, a.H), PL.scales[1] - PL.scales[0],
+                               a.stride};
+    const cuuint32_t box[4] = {mx ? 16u : 8u, 64, 2, 1};
+    if (!make_tmap(&m[2], mx ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 4,
+                   a.wbase + PL.scales[0], dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE))
       return cudaErrorInvalidValue;
     m[3] = m[2];
   }
@@ -911,8 +959,7 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
     prm.maxT = tc_max_tiles(2, Umax, a.H, a.I, a.num_sms);
     prm.S = tc_stages(2, a.fmt, NB, a.H, a.I, prm.maxT);
     if ((e = launch_sync_reset(a.sync, Umax, st)) != cudaSuccess) return e;
-    e = q2 ? launch_tc<2, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st)
-           : launch_tc<2, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+    e = launch_tc_fmt<2>(a.fmt, m, prm, a.num_sms, st);
     // Where the grid cannot be resident all at once (SMs held by other work,
     // a partitioned GPU), the cooperative launch is refused: clear the error
     // and run the two-kernel form, which needs no co-residency.
@@ -921,15 +968,10 @@ cudaError_t launch_experts_decode_tc(const DecodeArgs& a, cudaStream_t st) {
   }
   prm.maxT = tc_max_tiles(0, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(0, a.fmt, NB, a.H, a.I, prm.maxT);
-  if (q2)
-    e = launch_tc<0, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
-  else
-    e = launch_tc<0, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
-  if (e != cudaSuccess) return e;
+  if ((e = launch_tc_fmt<0>(a.fmt, m, prm, a.num_sms, st)) != cudaSuccess) return e;
   prm.maxT = tc_max_tiles(1, Umax, a.H, a.I, a.num_sms);
   prm.S = tc_stages(1, a.fmt, NB, a.H, a.I, prm.maxT);
-  if (q2) return launch_tc<1, STRATA_FMT_Q2_32>(m, prm, a.num_sms, st);
-  return launch_tc<1, STRATA_FMT_Q4CB_32>(m, prm, a.num_sms, st);
+  return launch_tc_fmt<1>(a.fmt, m, prm, a.num_sms, st);
 }
 
 }  // namespace strata

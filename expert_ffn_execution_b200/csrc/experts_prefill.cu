@@ -93,7 +93,9 @@ STRATA_DEVFN void load_chunk(PChunk<FMT>& r, const uint8_t* codes_row, const uin
   constexpr int CB = (FMT == STRATA_FMT_Q2_32) ? 16 : 32;
 #pragma unroll
   for (int i = 0; i < CB / 16; ++i) r.c[i] = ld_stream_v4(codes_row + kc * CB + 16 * i);
-  r.s = ld_stream_u32(scales_row + kc * 4);
+  // two block scales: fp16 pairs, or two E8M0 bytes
+  r.s = FMT == STRATA_FMT_MXFP4_32 ? ld_stream_u16(scales_row + kc * 2)
+                                   : ld_stream_u32(scales_row + kc * 4);
 }
 
 // Decode one row's chunk and store it, swizzled, into a [128 x 64] fp16 tile.
@@ -101,8 +103,9 @@ template <int FMT>
 STRATA_DEVFN void store_chunk(const PChunk<FMT>& r, uint8_t* tile, int row, const Q4Table& T4) {
   uint8_t* rbase = tile + row * 128;
   const int sw = row & 7;
-  const __half2 d0 = u32_as_h2(__byte_perm(r.s, 0, 0x1010));
-  const __half2 d1 = u32_as_h2(__byte_perm(r.s, 0, 0x3232));
+  const bool mx = FMT == STRATA_FMT_MXFP4_32;
+  const __half2 d0 = u32_as_h2(mx ? mx_scale_h2(r.s & 0xFFu) : __byte_perm(r.s, 0, 0x1010));
+  const __half2 d1 = u32_as_h2(mx ? mx_scale_h2((r.s >> 8) & 0xFFu) : __byte_perm(r.s, 0, 0x3232));
 #pragma unroll
   for (int g = 0; g < 4; ++g) {  // 16 elements per group, two 16-byte chunks
     uint32_t R[8];
@@ -110,6 +113,10 @@ STRATA_DEVFN void store_chunk(const PChunk<FMT>& r, uint8_t* tile, int row, cons
     if constexpr (FMT == STRATA_FMT_Q2_32) {
       const uint32_t w = (g == 0) ? r.c[0].x : (g == 1) ? r.c[0].y : (g == 2) ? r.c[0].z : r.c[0].w;
       dq_q2_natural(w, d2, R);
+    } else if constexpr (FMT == STRATA_FMT_MXFP4_32) {
+      const uint4& v = r.c[g >> 1];
+      dq_mx_word((g & 1) ? v.z : v.x, h2_as_u32(d2), R);
+      dq_mx_word((g & 1) ? v.w : v.y, h2_as_u32(d2), R + 4);
     } else {
       const uint4& v = r.c[g >> 1];
       dq_q4_group((g & 1) ? v.z : v.x, (g & 1) ? v.w : v.y, d2, T4, R);
@@ -283,9 +290,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
     const int pg = (warp - 4) >> 2;   // group: takes chunks j = pg, pg + 2, ...
     const int r = threadIdx.x & 127;  // weight row within the tile
     const Q4Table T4 = q4_table();
-    const uint64_t crow = codes_row_bytes(FMT, K), srow = (uint64_t)(K / 32) * 2;
+    const uint64_t crow = codes_row_bytes(FMT, K), srow = scales_row_bytes(FMT, K);
     constexpr int NA = C::NA;
-    constexpr int PD = (FMT == STRATA_FMT_Q4CB_32 && NA == 2) ? 3 : 4;  // register budget
+    constexpr int PD = (FMT != STRATA_FMT_Q2_32 && NA == 2) ? 3 : 4;  // register budget
     const int nunits = (total > (int)blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
     const int nchunks = nunits * KC;
     // flat chunk sequence of this CTA: j -> unit blockIdx.x + (j / KC) * grid, chunk j % KC
@@ -490,6 +497,11 @@ cudaError_t launch_experts_prefill(const PrefillArgs& a, cudaStream_t st) {
   if (a.fmt == STRATA_FMT_Q2_32) {
     if ((e = launch_gemm<0, STRATA_FMT_Q2_32>(mx, a, tiles, count, h, st)) != cudaSuccess) return e;
     return launch_gemm<1, STRATA_FMT_Q2_32>(mh, a, tiles, count, a.y, st);
+  }
+  if (a.fmt == STRATA_FMT_MXFP4_32) {
+    if ((e = launch_gemm<0, STRATA_FMT_MXFP4_32>(mx, a, tiles, count, h, st)) != cudaSuccess)
+      return e;
+    return launch_gemm<1, STRATA_FMT_MXFP4_32>(mh, a, tiles, count, a.y, st);
   }
   if ((e = launch_gemm<0, STRATA_FMT_Q4CB_32>(mx, a, tiles, count, h, st)) != cudaSuccess) return e;
   return launch_gemm<1, STRATA_FMT_Q4CB_32>(mh, a, tiles, count, a.y, st);

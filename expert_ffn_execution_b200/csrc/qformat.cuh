@@ -2,9 +2,10 @@
 //
 // Storage (include/strata_moe.h): per matrix, output-feature rows with K
 // contiguous; a codes plane (Q2_32: K/4 bytes per row, element k at byte k/4,
-// bits 2(k%4)..; Q4CB_32: K/2 bytes per row, low nibble = even k) and an fp16
-// scales plane [rows][K/32].  Blob = gate codes|scales, up codes|scales, down
-// codes|scales, each plane on a 256-byte boundary.
+// bits 2(k%4)..; Q4CB_32 and MXFP4_32: K/2 bytes per row, low nibble = even
+// k) and a scales plane [rows][K/32] (fp16; MXFP4_32: E8M0 bytes).  Blob =
+// gate codes|scales, up codes|scales, down codes|scales, each plane on a
+// 256-byte boundary.
 //
 // Register-level decode for the mma.sync decode path.  A "group" is 16
 // consecutive K elements of one row.  Decoding a group yields eight fp16x2
@@ -31,6 +32,10 @@ __host__ __device__ inline uint64_t codes_row_bytes(int fmt, int K) {
   return fmt == STRATA_FMT_Q2_32 ? uint64_t(K) / 4 : uint64_t(K) / 2;
 }
 
+__host__ __device__ inline uint64_t scales_row_bytes(int fmt, int K) {
+  return fmt == STRATA_FMT_MXFP4_32 ? uint64_t(K) / 32 : uint64_t(K) / 16;
+}
+
 __host__ __device__ inline Planes plane_offsets(int fmt, int H, int I, uint64_t* total = nullptr) {
   Planes p;
   uint64_t off = 0;
@@ -40,7 +45,7 @@ __host__ __device__ inline Planes plane_offsets(int fmt, int H, int I, uint64_t*
     p.codes[m] = off;
     off = round_up_256(off + uint64_t(rows) * codes_row_bytes(fmt, K));
     p.scales[m] = off;
-    off = round_up_256(off + uint64_t(rows) * uint64_t(K / 32) * 2);
+    off = round_up_256(off + uint64_t(rows) * scales_row_bytes(fmt, K));
   }
   if (total) *total = off;
   return p;
@@ -118,6 +123,30 @@ STRATA_DEVFN void dq_q4_group(uint32_t w0, uint32_t w1, __half2 d2, const Q4Tabl
     R[2 * i + 1] =
         h2_as_u32(__hmul2(__hsub2(u32_as_h2(__byte_perm(u[i], 0x64646464u, 0x4342u)), C), d2));
   }
+}
+
+// ---------------------------------------------------------------- MXFP4_32
+// E8M0 scale byte e -> fp16x2 (2^(e-127), same): the fp32 whose exponent
+// field is e is 2^(e-127) (0 for e = 0, +inf for e = 255); the one rounding
+// to fp16 keeps it exact for e in 103..142.
+STRATA_DEVFN uint32_t mx_scale_h2(uint32_t e) {
+  return h2_as_u32(__float2half2_rn(__uint_as_float(e << 23)));
+}
+
+// One word of MXFP4 codes (elements 0..7, low nibble first) times the block
+// scale: R[i] = (element 2i, element 2i+1) * d.  The sm_100 conversion
+// cvt.rn.f16x2.e2m1x2 turns one code byte into its two E2M1 values in fp16
+// (exact: they have two significant bits), low nibble in the low half; the
+// multiply by the power of two d is exact while the product is in fp16 range.
+STRATA_DEVFN void dq_mx_word(uint32_t w, uint32_t d2, uint32_t* R) {
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t.reg .b32 v0, v1, v2, v3;\n\t"
+      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 v0, q0;\n\tcvt.rn.f16x2.e2m1x2 v1, q1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 v2, q2;\n\tcvt.rn.f16x2.e2m1x2 v3, q3;\n\t"
+      "mul.rn.f16x2 %0, v0, %5;\n\tmul.rn.f16x2 %1, v1, %5;\n\t"
+      "mul.rn.f16x2 %2, v2, %5;\n\tmul.rn.f16x2 %3, v3, %5;\n\t}"
+      : "=r"(R[0]), "=r"(R[1]), "=r"(R[2]), "=r"(R[3])
+      : "r"(w), "r"(d2));
 }
 
 }  // namespace strata

@@ -76,7 +76,8 @@ typedef enum strata_status {
 /* ---------------------------------------------------------------- formats
  * Block-quantised expert weights.  Each weight matrix is stored as
  * output-feature rows with the K (input) dimension contiguous; blocks are 32
- * consecutive K elements of one row with one IEEE fp16 scale d per block.
+ * consecutive K elements of one row with one scale d per block (IEEE fp16,
+ * or an E8M0 byte for MXFP4).
  *
  *   STRATA_FMT_Q2_32   2-bit code c in 0..3; w = d * (c - 1.5).
  *                      Codes plane uint8 [N][K/4]: element k is byte k/4,
@@ -90,7 +91,20 @@ typedef enum strata_status {
  *                      IQ4_NL in section 13).  Codes plane uint8 [N][K/2]:
  *                      element k is byte k/2, low nibble for even k, high
  *                      nibble for odd k.  4.5 bits per weight.
- *   Scales plane (both formats): fp16 [N][K/32], little-endian.
+ *   STRATA_FMT_MXFP4_32 the OCP Microscaling (MX) v1.0 MXFP4 format, in
+ *                      which the native-MXFP4 model tier ships its experts
+ *                      (lcz.me/topic/2153, model tier list, "ds4f-mxfp4").
+ *                      4-bit code c is an FP4 E2M1 number (bit 3 sign, bits
+ *                      2-1 exponent with bias 1, bit 0 mantissa, exponent 0
+ *                      subnormal: codes 0..7 are 0,0.5,1,1.5,2,3,4,6); the
+ *                      block scale is one E8M0 byte e, d = 2^(e-127).
+ *                      w = e2m1(c) * d.  Codes plane as for Q4CB_32.
+ *                      4.25 bits per weight.  The kernels form w in fp16,
+ *                      which is exact for e in 104..140; outside it w is
+ *                      fp16-rounded (flushed towards 0 below, +-inf above;
+ *                      e = 255, NaN in the format, gives non-finite w).
+ *   Scales plane: fp16 [N][K/32], little-endian (Q2_32, Q4CB_32), or
+ *   uint8 E8M0 [N][K/32] (MXFP4_32).
  *
  * One expert blob, in this order, every plane starting on a 256-byte boundary:
  *   gate codes [I][H..] | gate scales | up codes [I][H..] | up scales |
@@ -98,9 +112,13 @@ typedef enum strata_status {
  * strata_expert_bytes() gives its size: 1,536,000 B for Q2_32 at H=2560,
  * I=640 (the pages' own 2.25-bit Q2_0 blob is 1,382,400 B, lcz.me/topic/2153
  * section 3.4; its bit layout is not on the pages), 2,764,800 B for Q4CB_32
- * at H=2560, I=640 and 14,155,776 B at H=4096, I=2048. */
+ * at H=2560, I=640 and 14,155,776 B at H=4096, I=2048, 2,611,200 B for
+ * MXFP4_32 at H=2560, I=640.  The decode path (T <= STRATA_DECODE_MAX_T)
+ * takes MXFP4_32 weights only with H a multiple of 512 (its scale rows are
+ * then whole 16-byte units); other H return STRATA_EUNSUPPORTED there. */
 #define STRATA_FMT_Q2_32 1
 #define STRATA_FMT_Q4CB_32 2
+#define STRATA_FMT_MXFP4_32 3
 
 /* Element types of expert outputs y (and of moe_gather_rows rows). */
 #define STRATA_DTYPE_F32 0

@@ -42,11 +42,13 @@ def test_abi_version_and_status_strings():
     assert sm.status_string(99) == "unknown status"
 
 
-@pytest.mark.parametrize("fmt,H,I", [(1, 2560, 640), (2, 2560, 640), (2, 4096, 2048), (1, 128, 128)])
+@pytest.mark.parametrize("fmt,H,I", [(1, 2560, 640), (2, 2560, 640), (2, 4096, 2048), (1, 128, 128),
+                                     (3, 2560, 640), (3, 4096, 2048), (3, 128, 128)])
 def test_expert_bytes_agree(fmt, H, I):
     assert sm.strata_expert_bytes(fmt, H, I) == moe_inputs.expert_bytes(fmt, H, I)
     assert sm.strata_expert_bytes(fmt, H, I) == oracle.expert_bytes(fmt, H, I)
-    assert sm.strata_expert_bytes(3, H, I) == 0
+    assert sm.strata_expert_bytes(4, H, I) == 0
+    assert sm.strata_expert_bytes(0, H, I) == 0
     assert sm.strata_expert_bytes(fmt, H + 16, I) == 0
 
 

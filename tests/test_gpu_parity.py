@@ -21,7 +21,7 @@ if not torch.cuda.is_available():
 import expert_ffn_execution_b200 as sm  # noqa: E402
 import moe_inputs as mi  # noqa: E402
 import oracle  # noqa: E402
-from expert_ffn_execution_b200._binding import EOVERFLOW  # noqa: E402
+from expert_ffn_execution_b200._binding import EOVERFLOW, EUNSUPPORTED  # noqa: E402
 from tests.harness import (OUT_REL_L2, TOPK_W_ATOL, check_routing, logit_tol, parallel_rows,  # noqa: E402
                            rel_l2_rows, stratified_tokens)
 
@@ -180,11 +180,12 @@ def check_layer(r: Run, sample=None):
 
 
 @pytest.mark.parametrize("config,T", [(0, 1), (1, 4), (3, 1), (3, 4), (4, 1), (4, 4), (4, 8),
-                                      (4, 16), (5, 1), (5, 4)])
+                                      (4, 16), (5, 1), (5, 4), (6, 1), (6, 4)])
 def test_decode_layer_parity(config, T):
-    """Configs 0, 1, 3 and 4 at their decode token counts, and config 5
-    ("C3b": the all-4-bit-codebook reading of config 3 at E = 512), each
-    checked on every token with the parity bars."""
+    """Configs 0, 1, 3 and 4 at their decode token counts, config 5
+    ("C3b": the all-4-bit-codebook reading of config 3 at E = 512) and config
+    6 (MXFP4 routed experts), each checked on every token with the parity
+    bars."""
     r = Run(config, T).run()
     err = check_layer(r)
     print(f"C{config} T={T}: max rel L2 {err.max():.2e}")
@@ -195,6 +196,44 @@ def test_decode_ragged_token_counts(T):
     """Token counts on both sides of the 8-column MMA tile, up to the decode
     maximum (two column tiles)."""
     check_layer(Run(1, T).run())
+
+
+@pytest.mark.parametrize("T", [7, 9, 16])
+def test_mxfp4_decode_ragged_token_counts(T):
+    """MXFP4 experts at token counts on both sides of the 8-column tile."""
+    check_layer(Run(6, T).run())
+
+
+def test_mxfp4_decode_top_of_exact_scale_range():
+    """MXFP4 down-projection scales raised by 2^19 to E8M0 bytes 137..140,
+    the top of the range where the kernels' fp16 weight e2m1 * 2^(e-127) is
+    exact (6 * 2^13 = 49152 < 65504); y is fp32 on the decode path, so
+    parity holds as for ordinary scales."""
+    r = Run(6, 4)
+    planes, _ = mi.plane_layout(r.c.fmt, r.H, r.I)
+    _, off, n, _, _, _ = [pl for pl in planes if pl[0] == "down" and pl[5] == "scales"][0]
+    r.inp.experts[:, off:off + n] += 19
+    assert int(r.inp.experts[:, off:off + n].max()) == 140
+    r.run()
+    check_layer(r)
+
+
+def test_mxfp4_decode_needs_h_multiple_of_512():
+    """MXFP4 at H = 2304 (a multiple of 256, not of 512): the decode path
+    reports STRATA_EUNSUPPORTED before launching anything."""
+    H, I, E, T, k = 2304, 640, 4, 2, 2
+    nb = sm.strata_expert_bytes(sm.FMT_MXFP4_32, H, I)
+    blobs = torch.zeros(E, nb, dtype=torch.uint8, device=DEV)
+    qw = sm.qweights(sm.FMT_MXFP4_32, E, H, I, blobs, blobs.stride(0))
+    hid = torch.zeros(T, H, dtype=torch.bfloat16, device=DEV)
+    offs = torch.tensor([0, 2, 4, 4, 4], dtype=torch.int32, device=DEV)
+    perm = torch.arange(T * k, dtype=torch.int32, device=DEV)
+    act = torch.tensor([2, 0, 1, 0, 0], dtype=torch.int32, device=DEV)
+    y = torch.empty(T * k, H, dtype=torch.float32, device=DEV)
+    ew = ws(sm.moe_experts_workspace_size(qw, T, k))
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    rc = sm.moe_experts(hid, qw, offs, perm, act, T, k, y, ew, ew.numel(), st, check=False)
+    assert rc == EUNSUPPORTED
 
 
 def test_decode_small_expert_count_and_k1():
@@ -345,6 +384,12 @@ def test_prefill_ragged(T, E):
     print(f"prefill T={T} E={E}: max rel L2 {err.max():.2e}")
 
 
+@pytest.mark.parametrize("T,E", [(17, 16), (300, 16)])
+def test_mxfp4_prefill_ragged(T, E):
+    """MXFP4 experts on the tensor-core path, every token checked."""
+    check_layer(Run(6, T, E=E).run())
+
+
 def test_prefill_one_expert_takes_everything():
     """All tokens routed to one expert (k = 1, E = 8, a bias of +50 on expert 1):
     a single expert with T tokens = many full tiles plus a tail."""
@@ -357,10 +402,10 @@ def test_prefill_one_expert_takes_everything():
     check_layer(r, sample=np.arange(0, T, 37))
 
 
-@pytest.mark.parametrize("config", [2, 3, 4])
+@pytest.mark.parametrize("config", [2, 3, 4, 6])
 def test_prefill_full_size(config):
     """The T = 8192 prefill chunks (2-bit routed; + 4-bit shared expert; 4-bit
-    large experts) at full size: RMSNorm, router logits, top-k ids and weights
+    large experts; MXFP4 routed) at full size: RMSNorm, router logits, top-k ids and weights
     and the bucket on all 8192 tokens; combine, expert outputs and layer
     output on a stratified sample of 256 tokens (the least-loaded expert's
     tokens, the most-loaded expert's full tiles and last partial tile, the
