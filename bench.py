@@ -57,7 +57,12 @@ FALLBACK_BF16_TFLOPS = 1590.0
 FALLBACK_BF16_SUSTAINED = 1400.0
 METRIC = "MoE-layer tokens/s; decode HBM GB/s and prefill TFLOPS as % of B200 peak"
 NCU_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-DEFAULT_LINES = "2:8192,2:32768,1:4"   # config:T, in this order; the last is the headline
+# config:T[:layers], in this order; the last is the headline.  Every decode
+# line streams more weight bytes per step than the 126 MB L2 holds.
+DEFAULT_LINES = "2:8192,4:8192,6:8192,2:32768,0:1:48,4:1:4,4:4,6:4:8,1:4"
+FMT_NAMES = {1: ("Q2_32", "2.5 bits/weight"), 2: ("Q4CB_32", "4.5 bits/weight"),
+             3: ("MXFP4_32", "4.25 bits/weight")}
+L2_BYTES = 126e6
 OUT_REL_L2 = 5e-3
 
 
@@ -107,10 +112,11 @@ def job_tokens_per_s(tokens_per_step_per_rank, steps, world, ms):
 
 
 def parse_lines(spec):
+    """'config:T' or 'config:T:layers' items -> [(config, T, layers or None)]."""
     out = []
     for item in spec.split(","):
-        c, t = item.split(":")
-        out.append((int(c), int(t)))
+        f = item.split(":")
+        out.append((int(f[0]), int(f[1]), int(f[2]) if len(f) > 2 else None))
     return out
 
 
@@ -527,7 +533,8 @@ def run_line(args, config, T, L, ws_, rank, dev):
         parity["pass"] = parity["pass"] and same
     result = None
     if rank == 0:
-        fmt_name = "Q2_32" if cfg.fmt == 1 else "Q4CB_32"
+        fmt_name, fmt_bits = FMT_NAMES[cfg.fmt]
+        step_bytes = sum(bytes_[:L])
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": ws_,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 4),
@@ -540,9 +547,11 @@ def run_line(args, config, T, L, ws_, rank, dev):
                        "layers": L, "T": T, "tokens_per_step_per_gpu": T,
                        "parallelism": f"replicas x{ws_}",
                        "accumulate": "f32",
-                       "weights": "2.5 bits/weight" if cfg.fmt == 1 else "4.5 bits/weight",
-                       "l2": ("no flush: per-step weight stream (~%.1f GB) >> 126 MB L2"
-                              % (sum(bytes_[:L]) / 1e9)) if not prefill else
+                       "weights": fmt_bits,
+                       "l2": (("no flush: per-step weight stream (~%.2f GB) > 126 MB L2"
+                               % (step_bytes / 1e9)) if step_bytes > L2_BYTES else
+                              ("WARNING: per-step weight stream %.0f MB fits in the 126 MB L2"
+                               % (step_bytes / 1e6))) if not prefill else
                              "no flush: per-step working set (weights + activations) > 1 GB",
                        "graphs": G},
             "e2e": {"value": round(e2e, 2), "unit": "tokens/s",
@@ -597,9 +606,9 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     lines = line_specs(args)
     results = []
-    for i, (config, T) in enumerate(lines):
+    for i, (config, T, L_line) in enumerate(lines):
         cfg = mi.CONFIGS[config]
-        L = args.layers or cfg.layers
+        L = args.layers or L_line or cfg.layers
         r = run_line(args, config, T, L, ws_, rank, dev)
         if r is not None:
             if i == len(lines) - 1 and len(results) > 0:
@@ -616,7 +625,7 @@ def run_ours(args):
 def line_specs(args):
     if args.config is not None:
         cfg = mi.CONFIGS[args.config]
-        return [(args.config, args.tokens or cfg.Ts[0])]
+        return [(args.config, args.tokens or cfg.Ts[0], None)]
     return parse_lines(args.lines)
 
 
@@ -631,9 +640,9 @@ def run_reference(args):
     ws_, rank, _ = dist_env()
     if rank != 0:
         return None
-    config, T = line_specs(args)[-1]
+    config, T, L_line = line_specs(args)[-1]
     cfg = mi.CONFIGS[config]
-    L = args.layers or cfg.layers
+    L = args.layers or L_line or cfg.layers
     decode = T <= 16
     Tu = T if decode else 16
     cached = []
