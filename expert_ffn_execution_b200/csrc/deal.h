@@ -24,8 +24,12 @@ constexpr int kTcDownOverhead = 4;  // per-down-tile cost beyond its K, 64-colum
 // positive, below r possibly negative, and where it is negative (the CTAs
 // below already carry more than their share) a CTA gets no down tile, so
 // bstart is non-decreasing and ends at ntB.
+// With fewer gate/up tiles than CTAs (q = 0) no down tile can start before
+// the gate/up tiles end (every expert's gate/up tiles are in the one round),
+// so a CTA without a gate/up tile is charged one all the same (qc, rc: the
+// charged counts): the down tiles are then split evenly over the grid.
 struct TcDeal {
-  int G, ntA, ntB, q, r;
+  int G, ntA, ntB, q, r, qc, rc;
   long long costA, costB, tot;
 };
 
@@ -36,14 +40,16 @@ STRATA_HD inline TcDeal tc_deal(int G, int U, int H, int I) {
   d.ntB = U * (H / 128);
   d.q = d.ntA / G;
   d.r = d.ntA - d.q * G;
+  d.qc = d.q == 0 ? 1 : d.q;
+  d.rc = d.q == 0 ? 0 : d.r;
   d.costA = H / 64;
   d.costB = I / 64 + kTcDownOverhead;
-  d.tot = (long long)d.ntA * d.costA + (long long)d.ntB * d.costB;
+  d.tot = ((long long)d.qc * G + d.rc) * d.costA + (long long)d.ntB * d.costB;
   return d;
 }
 
 STRATA_HD inline int tc_deal_bstart(const TcDeal& d, int c) {
-  const long long a = (long long)c * d.q + (c < d.r ? c : d.r);
+  const long long a = (long long)c * d.qc + (c < d.rc ? c : d.rc);
   const long long F = (long long)c * d.tot - (long long)d.G * d.costA * a;
   if (F <= 0) return 0;
   const long long s = F / ((long long)d.G * d.costB);

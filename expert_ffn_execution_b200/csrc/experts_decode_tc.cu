@@ -600,7 +600,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     const uint32_t swz = ((uint32_t)(r * CBR) >> 7) & (uint32_t)(NPC - 1);
     const uint32_t tl = tmem_base + ((uint32_t)(32 * qd) << 16) + kTcACol0;
     const Q4Table T4 = q4_table();
-    int gc = 0;
+    // The CTA's chunks in sequence go to the groups in turn, so this group
+    // takes every kTcGroups-th: its shared-memory stage advances by
+    // kTcGroups (S is a multiple of it) and its TMEM stage is always g.
+    // Stage, parities and the first chunk of each tile are kept as running
+    // values rather than divided out of a chunk counter per chunk.
+    static_assert(kTcTS == kTcGroups, "one TMEM stage per decoder group");
+    int cmod = 0;              // chunks of the CTA before this tile, mod kTcGroups
+    int s_cur = g, fpar = 0;   // next shared-memory stage and its full-barrier parity
+    uint32_t tpar = 1;         // parity awaited on the TMEM stage (its first use passes)
     for (int i = 0; i < tcount; ++i) {
       const bool isA = kGU && (MODE == 0 || i < nA);
       const int ib = i - nA;
@@ -611,10 +619,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         mbar_wait_guarded(&sfull[ib & 1], (ib >> 1) & 1, p.status, abort_flag);
         srow = smem + L.sbuf + (ib & 1) * L.s_bytes + r * (int)scales_row_bytes(FMT, I);
       }
-      for (int c = 0; c < nch; ++c, ++gc) {
-        if (gc % kTcGroups != g) continue;
-        const int s = gc % S;
-        mbar_wait_guarded(&full[s], (gc / S) & 1, p.status, abort_flag);
+      for (int c = (g - cmod + kTcGroups) % kTcGroups; c < nch; c += kTcGroups) {
+        const int s = s_cur;
+        const int par = fpar;
+        s_cur += kTcGroups;
+        if (s_cur >= S) {
+          s_cur -= S;
+          fpar ^= 1;
+        }
+        mbar_wait_guarded(&full[s], par, p.status, abort_flag);
         const uint8_t* st = smem + s * L.stage_bytes;
         const int kv = min(kTcKC, K - c * kTcKC);  // 256, or 128 for a ragged last chunk
         const int np = kv / PIECE_K;
@@ -657,8 +670,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         // write into the stage, which the barrier alone does not.
         fence_proxy_async_smem();
         mbar_arrive(&empty[s]);
-        const int t = gc % kTcTS;
-        mbar_wait_guarded(&tempty[t], ((gc / kTcTS) & 1) ^ 1, p.status, abort_flag);
+        const int t = g;
+        mbar_wait_guarded(&tempty[t], tpar, p.status, abort_flag);
+        tpar ^= 1u;
         tc_fence_after();
         const uint32_t ta = tl + (uint32_t)t * 128u;
         if constexpr (FMT == STRATA_FMT_Q2_32) {
@@ -709,6 +723,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         tc_fence_before();
         mbar_arrive(&tfull[t]);
       }
+      cmod = (cmod + nch) % kTcGroups;
       if (!isA) {
         fence_proxy_async_smem();  // same for the scale block and its next bulk copy
         mbar_arrive(&sempty[ib & 1]);

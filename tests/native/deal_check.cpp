@@ -42,9 +42,9 @@ static int check(int G, int U, int Umax, int H, int I) {
   // weighted work is within one down tile of Tot / G; where F(c+1) < 0 (the
   // CTAs up to c already carry more than their share) it has no down tile
   for (int c = 0; c < G; ++c) {
-    const int nA = d.q + (c < d.r ? 1 : 0);
+    const int nA = d.qc + (c < d.rc ? 1 : 0);  // charged gate/up tiles
     const auto F = [&](int x) {
-      const long long a = (long long)x * d.q + (x < d.r ? x : d.r);
+      const long long a = (long long)x * d.qc + (x < d.rc ? x : d.rc);
       return (long long)x * d.tot - (long long)d.G * d.costA * a;
     };
     const long long work = (long long)nA * d.costA + (long long)bc[c] * d.costB;  // x G below
