@@ -27,28 +27,9 @@ STRATA_DEVFN uint16_t f16_bits_checked(float v, int32_t* status) {
 
 // ---------------------------------------------------------------- loads
 // Weights are streamed once: keep them out of L1.
-STRATA_DEVFN uint4 ld_stream_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
-STRATA_DEVFN uint2 ld_stream_v2(const void* p) {
-  uint2 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(v.x), "=r"(v.y)
-               : "l"(p));
-  return v;
-}
 STRATA_DEVFN uint32_t ld_stream_u32(const void* p) {
   uint32_t v;
   asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(v) : "l"(p));
-  return v;
-}
-STRATA_DEVFN uint32_t ld_stream_u16(const void* p) {
-  uint16_t v;
-  asm volatile("ld.global.nc.L1::no_allocate.u16 %0, [%1];" : "=h"(v) : "l"(p));
   return v;
 }
 

@@ -57,9 +57,50 @@ struct PCfg {  // MODE 0: gate/up, 1: down
   static constexpr int SB = (NA + 1) * kTileBytes;
 };
 
+constexpr int kPXBytes = 4 * 16 * 32 * 2;  // epilogue transpose buffers: 4 warps x [16][32] fp16
+
 template <int MODE>
 __host__ __device__ inline size_t prefill_smem_bytes() {
-  return 1024 + (size_t)PCfg<MODE>::S * PCfg<MODE>::SB + 256;
+  return 1024 + (size_t)PCfg<MODE>::S * PCfg<MODE>::SB + 256 + kPXBytes;
+}
+
+// Epilogue store of 16 output columns (tokens c0..c0+15) of one warp's 32
+// rows: v[j] is this lane's row value for token c0 + j.  The values are
+// rounded to fp16 in pairs (an infinity from a finite value sets
+// STRATA_DEV_OVERFLOW, as in f16_bits_checked), written token-major into the
+// warp's [16][32] fp16 buffer, and read back as 16-byte pieces, so each lane
+// stores two 16-byte pieces of token rows instead of sixteen 2-byte values.
+// out + (size_t)(s0 + c0 + j) * ld + row0 is token c0 + j's row 0 of the
+// warp; only tokens with c0 + j < n are stored.
+STRATA_DEVFN void store_cols_f16(const float (&v)[16], uint16_t* xw, int lane, uint16_t* out,
+                                 size_t ld, int s0, int c0, int n, int row0, int32_t* status) {
+  uint32_t pk[8], inf = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    pk[i] = h2_as_u32(__floats2half2_rn(v[2 * i], v[2 * i + 1]));
+    inf |= __vcmpeq2(pk[i] & 0x7fff7fffu, 0x7c007c00u);
+  }
+  if (inf) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (c0 + j < n && isfinite(v[j]) && __hisinf(__float2half_rn(v[j])))
+        dev_flag(status, STRATA_DEV_OVERFLOW);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    xw[(2 * i) * 32 + lane] = (uint16_t)(pk[i] & 0xffffu);
+    xw[(2 * i + 1) * 32 + lane] = (uint16_t)(pk[i] >> 16);
+  }
+  __syncwarp();
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const int u = lane + 32 * q, j = u >> 2, part = u & 3;
+    if (c0 + j < n) {
+      const uint4 val = *reinterpret_cast<const uint4*>(xw + j * 32 + part * 8);
+      *reinterpret_cast<uint4*>(out + (size_t)(s0 + c0 + j) * ld + row0 + part * 8) = val;
+    }
+  }
+  __syncwarp();
 }
 
 // ---------------------------------------------------------------- dequant (natural order)
@@ -81,6 +122,30 @@ STRATA_DEVFN void dq_q2_natural(uint32_t w, __half2 d2, uint32_t (&R)[8]) {
   }
 }
 
+// The producers' code and scale loads allocate in L1 (evict-last): a row's
+// codes for consecutive chunks share 32-byte sectors (2-bit: two chunks per
+// sector; scales: eight), and the chunks alternate between the two producer
+// groups of the same SM, so the second touch of a sector hits L1 instead of
+// going to L2 again.  With L1::no_allocate the gate/up kernel ran 1.44x
+// longer at C2.
+STRATA_DEVFN uint4 ld_keep_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::evict_last.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+STRATA_DEVFN uint32_t ld_keep_u32(const void* p) {
+  uint32_t v;
+  asm volatile("ld.global.nc.L1::evict_last.u32 %0, [%1];" : "=r"(v) : "l"(p));
+  return v;
+}
+STRATA_DEVFN uint32_t ld_keep_u16(const void* p) {
+  uint16_t v;
+  asm volatile("ld.global.nc.L1::evict_last.u16 %0, [%1];" : "=h"(v) : "l"(p));
+  return v;
+}
+
 template <int FMT>
 struct PChunk {  // one row's codes and scales for one K chunk of 64
   uint4 c[FMT == STRATA_FMT_Q2_32 ? 1 : 2];
@@ -92,10 +157,10 @@ STRATA_DEVFN void load_chunk(PChunk<FMT>& r, const uint8_t* codes_row, const uin
                              int kc) {
   constexpr int CB = (FMT == STRATA_FMT_Q2_32) ? 16 : 32;
 #pragma unroll
-  for (int i = 0; i < CB / 16; ++i) r.c[i] = ld_stream_v4(codes_row + kc * CB + 16 * i);
+  for (int i = 0; i < CB / 16; ++i) r.c[i] = ld_keep_v4(codes_row + kc * CB + 16 * i);
   // two block scales: fp16 pairs, or two E8M0 bytes
-  r.s = FMT == STRATA_FMT_MXFP4_32 ? ld_stream_u16(scales_row + kc * 2)
-                                   : ld_stream_u32(scales_row + kc * 4);
+  r.s = FMT == STRATA_FMT_MXFP4_32 ? ld_keep_u16(scales_row + kc * 2)
+                                   : ld_keep_u32(scales_row + kc * 4);
 }
 
 // Decode one row's chunk and store it, swizzled, into a [128 x 64] fp16 tile.
@@ -246,6 +311,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
   if (warp < 4) {
     // ------------------------------------------------ epilogue
     const int m = threadIdx.x;  // TMEM lane = weight row within the tile
+    const int lane = m & 31;
+    uint16_t* xw = reinterpret_cast<uint16_t*>(smem + C::S * C::SB + 256) + warp * 16 * 32;
     int it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++it) {
       const NTile tl = tiles[u / MT];
@@ -258,29 +325,21 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
       for (int c0 = 0; c0 < n16; c0 += 16) {
         uint32_t g[16];
         tmem_ld16(tb + c0, g);
+        float v[16];
         if constexpr (MODE == 0) {
           uint32_t uu[16];
           tmem_ld16(tb + 128 + c0, uu);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < tl.n) {
-              const float gv = __uint_as_float(g[j]), uv = __uint_as_float(uu[j]);
-              const float h = silu_f32(gv) * uv;
-              out[(size_t)(tl.s0 + n) * I + mt * kPM + m] = f16_bits_checked(h, status);
-            }
-          }
+          for (int j = 0; j < 16; ++j)
+            v[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(uu[j]);
         } else {
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < tl.n)
-              out[(size_t)(tl.s0 + n) * H + mt * kPM + m] =
-                  f16_bits_checked(__uint_as_float(g[j]), status);
-          }
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(g[j]);
         }
+        store_cols_f16(v, xw, lane, out, (size_t)(MODE == 0 ? I : H), tl.s0, c0, tl.n,
+                       mt * kPM + warp * 32, status);
       }
       tc_fence_before();
       mbar_arrive(&tempty[a]);
