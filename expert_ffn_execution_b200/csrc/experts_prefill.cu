@@ -24,25 +24,32 @@
 // the size-sorted list), warp-specialised:
 //   warps 0-3  epilogue: tcgen05.ld of their TMEM lane quarter, math, stores
 //   warps 4-11 producers, two groups of four warps taking alternate K chunks
-//              (stages); one weight row per thread; codes and scales are
-//              prefetched four chunks ahead in registers, decoded to fp16
+//              (stages); one weight row per thread; the row's codes come
+//              from a code stage in shared memory, its scales are
+//              prefetched a few chunks ahead in registers; decoded to fp16
 //              and stored into the 128-byte-swizzled K-major stage layout;
 //              thread 0 of a group also issues the TMA load of the B tile
-//   warp 12    tensor memory allocation and the single MMA-issuing thread
+//   warp 12    tensor memory allocation and the MMA issue (one elected lane)
+//   warp 13    the TMA loads of the code stages: 64 code bytes of each of
+//              the tile's weight rows (gate and up: both planes in one box),
+//              several chunks ahead of the producers
 // Stages are guarded by mbarriers (full: producers + TMA bytes; empty:
-// tcgen05.commit), accumulators by tmem_full/tmem_empty.  Every wait is
-// bounded (clock budget) and reports STRATA_DEV_TIMEOUT instead of hanging.
+// tcgen05.commit), code stages by cfull (TMA bytes) / cempty (the 256
+// producers), accumulators by tmem_full/tmem_empty.  Every wait is bounded
+// (clock budget) and reports STRATA_DEV_TIMEOUT instead of hanging.
 #include <algorithm>
 
 #include "routing.cuh"
 #include "tc05.cuh"
+#include "tmap.h"
 
 namespace strata {
 
 constexpr int kPM = 128;       // weight rows per tile (MMA M)
 constexpr int kPN = 128;       // tokens per n-tile (MMA N <= 128)
 constexpr int kPK = 64;        // K per stage: one 128-byte swizzle row of fp16
-constexpr int kPThreads = 13 * 32;  // 4 epilogue + 8 producer + 1 MMA warps
+constexpr int kPThreads = 14 * 32;  // 4 epilogue + 8 producer + 1 MMA + 1 code-TMA warps
+constexpr int kPCodeRow = 64;       // code bytes of one weight row per code stage
 constexpr int kTileBytes = kPM * kPK * 2;  // 16 KB per operand tile
 constexpr int kAccCols = 256;              // TMEM columns per accumulator set
 
@@ -53,15 +60,20 @@ struct NTile {
 template <int MODE>
 struct PCfg {  // MODE 0: gate/up, 1: down
   static constexpr int NA = (MODE == 0) ? 2 : 1;
-  static constexpr int S = (MODE == 0) ? 4 : 6;
+  static constexpr int S = (MODE == 0) ? 3 : 6;   // A/B stages
   static constexpr int SB = (NA + 1) * kTileBytes;
+  static constexpr int CSN = 3;                      // code stages
+  static constexpr int CSB = NA * kPM * kPCodeRow;   // bytes per code stage
 };
 
 constexpr int kPXBytes = 4 * 16 * 32 * 2;  // epilogue transpose buffers: 4 warps x [16][32] fp16
 
+// Shared memory from a 1024-byte aligned base: S stages | CSN code stages |
+// barriers (256 B) | the epilogue's transpose buffers.
 template <int MODE>
 __host__ __device__ inline size_t prefill_smem_bytes() {
-  return 1024 + (size_t)PCfg<MODE>::S * PCfg<MODE>::SB + 256 + kPXBytes;
+  using C = PCfg<MODE>;
+  return 1024 + (size_t)C::S * C::SB + (size_t)C::CSN * C::CSB + 256 + kPXBytes;
 }
 
 // Epilogue store of 16 output columns (tokens c0..c0+15) of one warp's 32
@@ -122,19 +134,10 @@ STRATA_DEVFN void dq_q2_natural(uint32_t w, __half2 d2, uint32_t (&R)[8]) {
   }
 }
 
-// The producers' code and scale loads allocate in L1 (evict-last): a row's
-// codes for consecutive chunks share 32-byte sectors (2-bit: two chunks per
-// sector; scales: eight), and the chunks alternate between the two producer
-// groups of the same SM, so the second touch of a sector hits L1 instead of
-// going to L2 again.  With L1::no_allocate the gate/up kernel ran 1.44x
-// longer at C2.
-STRATA_DEVFN uint4 ld_keep_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.L1::evict_last.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+// The producers' scale loads allocate in L1 (evict-last): a row's scales for
+// eight consecutive chunks share one 32-byte sector, and the chunks alternate
+// between the two producer groups of the same SM, so later touches of a
+// sector hit L1 instead of going to L2 again.
 STRATA_DEVFN uint32_t ld_keep_u32(const void* p) {
   uint32_t v;
   asm volatile("ld.global.nc.L1::evict_last.u32 %0, [%1];" : "=r"(v) : "l"(p));
@@ -152,15 +155,36 @@ struct PChunk {  // one row's codes and scales for one K chunk of 64
   uint32_t s;
 };
 
+// Code bytes of one row per 64-K chunk, and chunks per code stage.
 template <int FMT>
-STRATA_DEVFN void load_chunk(PChunk<FMT>& r, const uint8_t* codes_row, const uint8_t* scales_row,
-                             int kc) {
-  constexpr int CB = (FMT == STRATA_FMT_Q2_32) ? 16 : 32;
-#pragma unroll
-  for (int i = 0; i < CB / 16; ++i) r.c[i] = ld_keep_v4(codes_row + kc * CB + 16 * i);
-  // two block scales: fp16 pairs, or two E8M0 bytes
+__host__ __device__ constexpr int p_chunk_code_bytes() {
+  return FMT == STRATA_FMT_Q2_32 ? 16 : 32;
+}
+template <int FMT>
+__host__ __device__ constexpr int p_chunks_per_cs() {
+  return kPCodeRow / p_chunk_code_bytes<FMT>();
+}
+
+// The chunk's two block scales (fp16 pairs, or two E8M0 bytes), from global
+// memory a few chunks ahead of use.
+template <int FMT>
+STRATA_DEVFN void load_chunk_scales(PChunk<FMT>& r, const uint8_t* scales_row, int kc) {
   r.s = FMT == STRATA_FMT_MXFP4_32 ? ld_keep_u16(scales_row + kc * 2)
                                    : ld_keep_u32(scales_row + kc * 4);
+}
+
+// The chunk's codes from its code stage: row `row` of plane `cs_row` (64
+// bytes, 64-byte swizzled by the TMA: 16-byte unit u of row r sits at
+// u ^ ((r >> 1) & 3)), slot `slot` of the stage.
+template <int FMT>
+STRATA_DEVFN void load_chunk_codes(PChunk<FMT>& r, const uint8_t* cs_row, int row, int slot) {
+  constexpr int NU = p_chunk_code_bytes<FMT>() / 16;
+  const int swz = (row >> 1) & 3;
+#pragma unroll
+  for (int i = 0; i < NU; ++i) {
+    const int unit = (slot * NU + i) ^ swz;
+    r.c[i] = *reinterpret_cast<const uint4*>(cs_row + unit * 16);
+  }
 }
 
 // Decode one row's chunk and store it, swizzled, into a [128 x 64] fp16 tile.
@@ -260,7 +284,9 @@ prefill_gather_kernel(const uint16_t* __restrict__ hidden, const int32_t* __rest
 // ---------------------------------------------------------------- grouped GEMM
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(kPThreads, 1)
-prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __restrict__ wbase,
+prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
+                    const __grid_constant__ CUtensorMap cmap,  // weight codes
+                    const uint8_t* __restrict__ wbase,
                     uint64_t stride, int H, int I, const NTile* __restrict__ tiles,
                     const int* __restrict__ ntiles_ptr, uint16_t* __restrict__ out,
                     int32_t* status) {
@@ -268,11 +294,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::S * C::SB);
+  uint8_t* cstages = smem + C::S * C::SB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(cstages + C::CSN * C::CSB);
   uint64_t* empty = full + C::S;
   uint64_t* tfull = empty + C::S;
   uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
+  uint64_t* cfull = tempty + 2;
+  uint64_t* cempty = cfull + C::CSN;
+  uint64_t* done = cempty + C::CSN;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -284,6 +313,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
   const int ntiles = *ntiles_ptr;
   const int total = ntiles * MT;
   const Planes P = plane_offsets(FMT, H, I);
+  constexpr int CPC = p_chunks_per_cs<FMT>();
+  const int CSU = (KC + CPC - 1) / CPC;  // code stages per unit
+  const int nunits = (total > (int)blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::S; ++s) {
@@ -294,6 +326,10 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 128);
     }
+    for (int c = 0; c < C::CSN; ++c) {
+      mbar_init(&cfull[c], 1);
+      mbar_init(&cempty[c], 256);
+    }
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -303,6 +339,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
     tmem_relinquish();
   }
   if (threadIdx.x == 4 * 32) prefetch_tensormap(&bmap);
+  if (threadIdx.x == 13 * 32) prefetch_tensormap(&cmap);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -312,7 +349,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
     // ------------------------------------------------ epilogue
     const int m = threadIdx.x;  // TMEM lane = weight row within the tile
     const int lane = m & 31;
-    uint16_t* xw = reinterpret_cast<uint16_t*>(smem + C::S * C::SB + 256) + warp * 16 * 32;
+    uint16_t* xw = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(full) + 256) + warp * 16 * 32;
     int it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++it) {
       const NTile tl = tiles[u / MT];
@@ -349,15 +386,14 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
     const int pg = (warp - 4) >> 2;   // group: takes chunks j = pg, pg + 2, ...
     const int r = threadIdx.x & 127;  // weight row within the tile
     const Q4Table T4 = q4_table();
-    const uint64_t crow = codes_row_bytes(FMT, K), srow = scales_row_bytes(FMT, K);
+    const uint64_t srow = scales_row_bytes(FMT, K);
     constexpr int NA = C::NA;
-    constexpr int PD = (FMT != STRATA_FMT_Q2_32 && NA == 2) ? 3 : 4;  // register budget
-    const int nunits = (total > (int)blockIdx.x) ? (total - blockIdx.x + gridDim.x - 1) / gridDim.x : 0;
+    constexpr int PD = 4;  // scale prefetch depth (chunks of this group)
     const int nchunks = nunits * KC;
     // flat chunk sequence of this CTA: j -> unit blockIdx.x + (j / KC) * grid, chunk j % KC
     PChunk<FMT> ring[PD + 1][NA];
     int jp = pg, p_ui = -1;
-    const uint8_t *pc[NA], *ps[NA];
+    const uint8_t* ps[NA];
     auto prefetch = [&](PChunk<FMT> (&slot)[NA]) {
       if (jp < nchunks) {
         const int ui = jp / KC, kc = jp - ui * KC;
@@ -370,12 +406,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
 #pragma unroll
           for (int a = 0; a < NA; ++a) {
             const int mat = (MODE == 0) ? a : 2;
-            pc[a] = blob + P.codes[mat] + (uint64_t)row * crow;
             ps[a] = blob + P.scales[mat] + (uint64_t)row * srow;
           }
         }
 #pragma unroll
-        for (int a = 0; a < NA; ++a) load_chunk<FMT>(slot[a], pc[a], ps[a], kc);
+        for (int a = 0; a < NA; ++a) load_chunk_scales<FMT>(slot[a], ps[a], kc);
         jp += 2;
       }
     };
@@ -402,13 +437,49 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap, const uint8_t* __r
             mbar_expect_tx(&full[s], kTileBytes);
             tma_load_2d(stage + C::NA * kTileBytes, &bmap, kc * kPK, s0, &full[s]);
           }
+          // the chunk's codes: code stage gcs of the CTA's sequence, slot kc % CPC
+          const int gcs = ui * CSU + kc / CPC, slot = kc - (kc / CPC) * CPC;
+          const int ci = gcs % C::CSN;
+          mbar_wait_guarded(&cfull[ci], (gcs / C::CSN) & 1, status, abort_flag);
+          const uint8_t* cst = cstages + ci * C::CSB + r * kPCodeRow;
 #pragma unroll
-          for (int a = 0; a < NA; ++a) store_chunk<FMT>(ring[q][a], stage + a * kTileBytes, r, T4);
+          for (int a = 0; a < NA; ++a) {
+            load_chunk_codes<FMT>(ring[q][a], cst + a * kPM * kPCodeRow, r, slot);
+            store_chunk<FMT>(ring[q][a], stage + a * kTileBytes, r, T4);
+          }
+          // the generic-proxy shared accesses above (A rows written, codes
+          // read) before the async-proxy accesses that follow the barriers
           fence_proxy_async_smem();
           mbar_arrive(&full[s]);
+          // this group's last chunk of the code stage (the groups take the
+          // slots of their own parity; every code stage has >= 2 chunks)
+          const int in_cs = min(CPC, KC - (kc / CPC) * CPC);
+          if (slot + 2 >= in_cs) mbar_arrive(&cempty[ci]);
         }
       }
     }
+  } else if (warp == 13) {
+    // ------------------------------------------------ code stages by TMA:
+    // 64 code bytes of each of the unit's 128 weight rows (both planes for
+    // gate/up), in the producers' order, CSN stages ahead
+    if (elect_one()) {
+      int gcs = 0;
+      for (int ui = 0; ui < nunits; ++ui) {
+        const int u = blockIdx.x + ui * gridDim.x;
+        const int e = tiles[u / MT].e, mt = u % MT;
+        for (int cs = 0; cs < CSU; ++cs, ++gcs) {
+          const int ci = gcs % C::CSN;
+          if (!mbar_wait_guarded(&cempty[ci], ((gcs / C::CSN) & 1) ^ 1, status, abort_flag)) break;
+          mbar_arrive_expect_tx(&cfull[ci], C::CSB);
+          uint8_t* dst = cstages + ci * C::CSB;
+          if constexpr (MODE == 0)
+            tma_load_4d(dst, &cmap, cs * kPCodeRow, mt * kPM, 0, e, &cfull[ci]);
+          else
+            tma_load_3d(dst, &cmap, cs * kPCodeRow, mt * kPM, e, &cfull[ci]);
+        }
+      }
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------ MMA issue: the whole
     // warp runs the loop (converged); one elected lane issues each stage's
@@ -479,50 +550,48 @@ PrefillWs prefill_ws(int T, int H, int I, int E, int k, int shared_mode) {
   return w;
 }
 
-// The driver's tensor-map encoder, looked up through the runtime so the
-// library does not link against libcuda (it still loads where no driver is
-// installed; the entry point is resolved on first use on a GPU machine).
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_tiled() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
+// The B operand: [rows, cols] fp16, boxes of 64 columns x kPN rows.
 bool make_map(CUtensorMap* map, const void* base, int cols, long long rows) {
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
   const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)kPN};
-  const cuuint32_t estr[2] = {1, 1};
-  EncodeTiledFn enc = encode_tiled();
-  if (!enc) return false;
-  const CUresult r = enc(
-      map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// The weight codes, boxes of kPCodeRow bytes x kPM rows, 64-byte swizzled.
+// Gate/up: [E][2 planes][I rows][H code bytes] (the plane step is the gate
+// -> up plane distance, so one box holds a tile's gate and up rows); down:
+// [E][H rows][I code bytes].
+bool make_code_map(CUtensorMap* map, int mode, const PrefillArgs& a, int E) {
+  const Planes PL = plane_offsets(a.fmt, a.H, a.I);
+  if (mode == 0) {
+    const cuuint64_t row = codes_row_bytes(a.fmt, a.H);
+    const cuuint64_t dims[4] = {row, (cuuint64_t)a.I, 2, (cuuint64_t)E};
+    const cuuint64_t str[3] = {row, PL.codes[1] - PL.codes[0], a.stride};
+    const cuuint32_t box[4] = {(cuuint32_t)kPCodeRow, (cuuint32_t)kPM, 2, 1};
+    return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, a.wbase + PL.codes[0], dims, str, box,
+                     CU_TENSOR_MAP_SWIZZLE_64B);
+  }
+  const cuuint64_t row = codes_row_bytes(a.fmt, a.I);
+  const cuuint64_t dims[3] = {row, (cuuint64_t)a.H, (cuuint64_t)E};
+  const cuuint64_t str[2] = {row, a.stride};
+  const cuuint32_t box[3] = {(cuuint32_t)kPCodeRow, (cuuint32_t)kPM, 1};
+  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, a.wbase + PL.codes[2], dims, str, box,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 template <int MODE, int FMT>
-cudaError_t launch_gemm(const CUtensorMap& map, const PrefillArgs& a, const NTile* tiles,
+cudaError_t launch_gemm(const CUtensorMap& map, const PrefillArgs& a, int E, const NTile* tiles,
                         const int* count, uint16_t* out, cudaStream_t st) {
+  CUtensorMap cmap;
+  if (!make_code_map(&cmap, MODE, a, E)) return cudaErrorInvalidValue;
   auto kern = prefill_gemm_kernel<MODE, FMT>;
   const size_t smem = prefill_smem_bytes<MODE>();
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<a.num_sms, kPThreads, smem, st>>>(map, a.wbase, a.stride, a.H, a.I, tiles, count, out,
-                                          a.status);
+  kern<<<a.num_sms, kPThreads, smem, st>>>(map, cmap, a.wbase, a.stride, a.H, a.I, tiles, count,
+                                          out, a.status);
   return cudaGetLastError();
 }
 
@@ -534,6 +603,10 @@ uint64_t prefill_workspace_bytes(int T, int H, int I, int E, int k, int shared_m
 
 cudaError_t launch_experts_prefill(const PrefillArgs& a, cudaStream_t st) {
   if (a.H % kPM || a.I % kPM || a.H % kPK || a.I % kPK) return cudaErrorNotSupported;
+  // every code row holds at least one code stage (64 bytes)
+  if (codes_row_bytes(a.fmt, a.I) < (uint64_t)kPCodeRow ||
+      codes_row_bytes(a.fmt, a.H) < (uint64_t)kPCodeRow)
+    return cudaErrorNotSupported;
   const PrefillWs L = prefill_ws(a.T, a.H, a.I, a.E, a.k, a.shared_mode);
   if (a.ws_bytes < L.total) return cudaErrorInvalidValue;
   uint8_t* base = reinterpret_cast<uint8_t*>(a.ws);
@@ -554,16 +627,16 @@ cudaError_t launch_experts_prefill(const PrefillArgs& a, cudaStream_t st) {
   CUtensorMap mx, mh;
   if (!make_map(&mx, X, a.H, P) || !make_map(&mh, h, a.I, P)) return cudaErrorInvalidValue;
   if (a.fmt == STRATA_FMT_Q2_32) {
-    if ((e = launch_gemm<0, STRATA_FMT_Q2_32>(mx, a, tiles, count, h, st)) != cudaSuccess) return e;
-    return launch_gemm<1, STRATA_FMT_Q2_32>(mh, a, tiles, count, a.y, st);
+    if ((e = launch_gemm<0, STRATA_FMT_Q2_32>(mx, a, E, tiles, count, h, st)) != cudaSuccess) return e;
+    return launch_gemm<1, STRATA_FMT_Q2_32>(mh, a, E, tiles, count, a.y, st);
   }
   if (a.fmt == STRATA_FMT_MXFP4_32) {
-    if ((e = launch_gemm<0, STRATA_FMT_MXFP4_32>(mx, a, tiles, count, h, st)) != cudaSuccess)
+    if ((e = launch_gemm<0, STRATA_FMT_MXFP4_32>(mx, a, E, tiles, count, h, st)) != cudaSuccess)
       return e;
-    return launch_gemm<1, STRATA_FMT_MXFP4_32>(mh, a, tiles, count, a.y, st);
+    return launch_gemm<1, STRATA_FMT_MXFP4_32>(mh, a, E, tiles, count, a.y, st);
   }
-  if ((e = launch_gemm<0, STRATA_FMT_Q4CB_32>(mx, a, tiles, count, h, st)) != cudaSuccess) return e;
-  return launch_gemm<1, STRATA_FMT_Q4CB_32>(mh, a, tiles, count, a.y, st);
+  if ((e = launch_gemm<0, STRATA_FMT_Q4CB_32>(mx, a, E, tiles, count, h, st)) != cudaSuccess) return e;
+  return launch_gemm<1, STRATA_FMT_Q4CB_32>(mh, a, E, tiles, count, a.y, st);
 }
 
 }  // namespace strata
