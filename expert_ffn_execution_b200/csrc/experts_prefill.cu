@@ -4,9 +4,10 @@
 // dequantised to fp16 tiles in shared memory and multiplied on the 5th-gen
 // tensor cores (tcgen05.mma, fp16 x fp16 -> fp32 in tensor memory).  The
 // GEMMs are "swap-AB": the MMA's 128-row A operand is a tile of one expert's
-// weight rows and the N columns are that expert's tokens (<= 128 per tile,
+// weight rows and the N columns are that expert's tokens (<= 256 per tile,
 // padded to a multiple of 16), so skewed per-expert token counts waste at
-// most 15 columns per tile instead of up to 127 rows.
+// most 15 columns per tile instead of up to 127 rows, and an expert with up
+// to 256 tokens has its weights dequantised once per layer.
 //
 // Per call:
 //   1. plan:   per-expert token counts (from offsets) -> a list of n-tiles
@@ -14,9 +15,11 @@
 //              partial ones by decreasing size.
 //   2. gather: X[s] = fp16(hidden[token of sorted pair s]) (exact: bf16 has 8
 //              significant bits), so the B operand is a plain 2-D TMA tile.
-//   3. gate/up GEMM: units (n-tile, 128 rows of I); A = gate rows and the
-//              same up rows, two accumulators in TMEM; the epilogue applies
-//              SwiGLU and writes h fp16 [P, I] in sorted order.
+//   3. gate/up GEMM: units (n-tile, 64 rows of I); A = those 64 gate rows
+//              (TMEM lanes 0-63) and the same 64 up rows (lanes 64-127), one
+//              accumulator; the epilogue pairs the lanes through shared
+//              memory, applies SwiGLU and writes h fp16 [P, I] in sorted
+//              order.
 //   4. down GEMM: units (n-tile, 128 rows of H); B = h tiles by TMA; the
 //              epilogue writes y fp16 [P, H] in sorted order.
 //
@@ -31,7 +34,7 @@
 //              thread 0 of a group also issues the TMA load of the B tile
 //   warp 12    tensor memory allocation and the MMA issue (one elected lane)
 //   warp 13    the TMA loads of the code stages: 64 code bytes of each of
-//              the tile's weight rows (gate and up: both planes in one box),
+//              the tile's 128 A rows (gate and up: both planes in one box),
 //              several chunks ahead of the producers
 // Stages are guarded by mbarriers (full: producers + TMA bytes; empty:
 // tcgen05.commit), code stages by cfull (TMA bytes) / cempty (the 256
@@ -46,34 +49,45 @@
 namespace strata {
 
 constexpr int kPM = 128;       // weight rows per tile (MMA M)
-constexpr int kPN = 128;       // tokens per n-tile (MMA N <= 128)
+constexpr int kPN = 256;       // tokens per n-tile (MMA N <= 256)
 constexpr int kPK = 64;        // K per stage: one 128-byte swizzle row of fp16
 constexpr int kPThreads = 14 * 32;  // 4 epilogue + 8 producer + 1 MMA + 1 code-TMA warps
 constexpr int kPCodeRow = 64;       // code bytes of one weight row per code stage
-constexpr int kTileBytes = kPM * kPK * 2;  // 16 KB per operand tile
+constexpr int kTileBytes = kPM * kPK * 2;   // A tile: 16 KB
+constexpr int kBTileBytes = kPN * kPK * 2;  // B tile: 32 KB
 constexpr int kAccCols = 256;              // TMEM columns per accumulator set
 
 struct NTile {
   int e, s0, n, pad;
 };
 
+// The B operand's tensor maps, boxes of 64 columns x {64, 128, 256} rows.
+struct BMaps {
+  CUtensorMap m[3];
+};
+
+// One unit = one n-tile x one 128-row A tile.  Gate/up: rows 0-63 of the A
+// tile are 64 gate rows and rows 64-127 the same 64 up rows, so one
+// accumulator holds both and the epilogue pairs them; down: 128 rows of H.
 template <int MODE>
 struct PCfg {  // MODE 0: gate/up, 1: down
-  static constexpr int NA = (MODE == 0) ? 2 : 1;
-  static constexpr int S = (MODE == 0) ? 3 : 6;   // A/B stages
-  static constexpr int SB = (NA + 1) * kTileBytes;
-  static constexpr int CSN = 3;                      // code stages
-  static constexpr int CSB = NA * kPM * kPCodeRow;   // bytes per code stage
+  static constexpr int RPU = (MODE == 0) ? kPM / 2 : kPM;  // rows of each matrix per unit
+  static constexpr int S = 4;                           // A/B stages
+  static constexpr int SB = kTileBytes + kBTileBytes;
+  static constexpr int CSN = 3;                         // code stages
+  static constexpr int CSB = kPM * kPCodeRow;           // bytes per code stage
 };
 
 constexpr int kPXBytes = 4 * 16 * 32 * 2;  // epilogue transpose buffers: 4 warps x [16][32] fp16
+constexpr int kPUBytes = 64 * 17 * 4;      // gate/up epilogue: 64 up rows x 16 columns (+1 pad)
 
 // Shared memory from a 1024-byte aligned base: S stages | CSN code stages |
-// barriers (256 B) | the epilogue's transpose buffers.
+// barriers (256 B) | the epilogue's transpose buffers | its up-value
+// exchange (gate/up).
 template <int MODE>
 __host__ __device__ inline size_t prefill_smem_bytes() {
   using C = PCfg<MODE>;
-  return 1024 + (size_t)C::S * C::SB + (size_t)C::CSN * C::CSB + 256 + kPXBytes;
+  return 1024 + (size_t)C::S * C::SB + (size_t)C::CSN * C::CSB + 256 + kPXBytes + kPUBytes;
 }
 
 // Epilogue store of 16 output columns (tokens c0..c0+15) of one warp's 32
@@ -284,7 +298,7 @@ prefill_gather_kernel(const uint16_t* __restrict__ hidden, const int32_t* __rest
 // ---------------------------------------------------------------- grouped GEMM
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(kPThreads, 1)
-prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
+prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64, 128, 256 rows
                     const __grid_constant__ CUtensorMap cmap,  // weight codes
                     const uint8_t* __restrict__ wbase,
                     uint64_t stride, int H, int I, const NTile* __restrict__ tiles,
@@ -308,7 +322,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
   const int warp = threadIdx.x >> 5;
   const int K = (MODE == 0) ? H : I;
   const int Mtot = (MODE == 0) ? I : H;
-  const int MT = Mtot / kPM;
+  const int MT = Mtot / C::RPU;
   const int KC = K / kPK;
   const int ntiles = *ntiles_ptr;
   const int total = ntiles * MT;
@@ -338,7 +352,11 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
     tmem_alloc(tmem_slot, 2 * kAccCols);
     tmem_relinquish();
   }
-  if (threadIdx.x == 4 * 32) prefetch_tensormap(&bmap);
+  if (threadIdx.x == 4 * 32) {
+    prefetch_tensormap(&bmaps.m[0]);
+    prefetch_tensormap(&bmaps.m[1]);
+    prefetch_tensormap(&bmaps.m[2]);
+  }
   if (threadIdx.x == 13 * 32) prefetch_tensormap(&cmap);
   tc_fence_before();
   __syncthreads();
@@ -350,6 +368,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
     const int m = threadIdx.x;  // TMEM lane = weight row within the tile
     const int lane = m & 31;
     uint16_t* xw = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(full) + 256) + warp * 16 * 32;
+    float* xu = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256 + kPXBytes);
     int it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x, ++it) {
       const NTile tl = tiles[u / MT];
@@ -362,21 +381,30 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
       for (int c0 = 0; c0 < n16; c0 += 16) {
         uint32_t g[16];
         tmem_ld16(tb + c0, g);
-        float v[16];
+        tmem_wait_ld();
         if constexpr (MODE == 0) {
-          uint32_t uu[16];
-          tmem_ld16(tb + 128 + c0, uu);
-          tmem_wait_ld();
+          // lanes 64-127 hold the up rows: they hand their values to the
+          // gate lanes 0-63 of the same rows through shared memory
+          if (warp >= 2) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[j] = silu_f32(__uint_as_float(g[j])) * __uint_as_float(uu[j]);
+            for (int j = 0; j < 16; ++j) xu[(m - 64) * 17 + j] = __uint_as_float(g[j]);
+          }
+          named_bar_sync(1, 128);
+          if (warp < 2) {
+            float v[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = silu_f32(__uint_as_float(g[j])) * xu[m * 17 + j];
+            store_cols_f16(v, xw, lane, out, (size_t)I, tl.s0, c0, tl.n,
+                           mt * C::RPU + warp * 32, status);
+          }
+          named_bar_sync(1, 128);  // the exchange buffer is reused
         } else {
-          tmem_wait_ld();
+          float v[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(g[j]);
+          store_cols_f16(v, xw, lane, out, (size_t)H, tl.s0, c0, tl.n, mt * kPM + warp * 32,
+                         status);
         }
-        store_cols_f16(v, xw, lane, out, (size_t)(MODE == 0 ? I : H), tl.s0, c0, tl.n,
-                       mt * kPM + warp * 32, status);
       }
       tc_fence_before();
       mbar_arrive(&tempty[a]);
@@ -387,8 +415,12 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
     const int r = threadIdx.x & 127;  // weight row within the tile
     const Q4Table T4 = q4_table();
     const uint64_t srow = scales_row_bytes(FMT, K);
-    constexpr int NA = C::NA;
+    constexpr int NA = 1;  // one weight row per thread
     constexpr int PD = 4;  // scale prefetch depth (chunks of this group)
+    // this thread's matrix and row offset within the unit: gate/up rows
+    // 0-63 gate, 64-127 up; down: rows of H
+    const int mat = (MODE == 0) ? (r >> 6) : 2;
+    const int roff = (MODE == 0) ? (r & 63) : r;
     const int nchunks = nunits * KC;
     // flat chunk sequence of this CTA: j -> unit blockIdx.x + (j / KC) * grid, chunk j % KC
     PChunk<FMT> ring[PD + 1][NA];
@@ -401,13 +433,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
           p_ui = ui;
           const int u = blockIdx.x + ui * gridDim.x;
           const NTile tl = tiles[u / MT];
-          const int row = (u % MT) * kPM + r;
+          const int row = (u % MT) * C::RPU + roff;
           const uint8_t* blob = wbase + (uint64_t)tl.e * stride;
-#pragma unroll
-          for (int a = 0; a < NA; ++a) {
-            const int mat = (MODE == 0) ? a : 2;
-            ps[a] = blob + P.scales[mat] + (uint64_t)row * srow;
-          }
+          ps[0] = blob + P.scales[mat] + (uint64_t)row * srow;
         }
 #pragma unroll
         for (int a = 0; a < NA; ++a) load_chunk_scales<FMT>(slot[a], ps[a], kc);
@@ -416,7 +444,7 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
     };
 #pragma unroll
     for (int s = 0; s < PD; ++s) prefetch(ring[s]);
-    int c_ui = -1, s0 = 0;
+    int c_ui = -1, s0 = 0, nb = 0;
     for (int j0 = pg; j0 < nchunks; j0 += 2 * (PD + 1)) {
 #pragma unroll
       for (int q = 0; q <= PD; ++q) {
@@ -426,27 +454,30 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
           const int ui = j / KC, kc = j - ui * KC;
           if (ui != c_ui) {
             c_ui = ui;
-            s0 = tiles[(blockIdx.x + ui * gridDim.x) / MT].s0;
+            const NTile tl = tiles[(blockIdx.x + ui * gridDim.x) / MT];
+            s0 = tl.s0;
+            nb = tl.n <= 64 ? 0 : tl.n <= 128 ? 1 : 2;
           }
           const int s = j % C::S;
           mbar_wait_guarded(&empty[s], ((j / C::S) & 1) ^ 1, status, abort_flag);
           uint8_t* stage = smem + s * C::SB;
           if (r == 0) {
-            // B tile: expected bytes first, then the copy; the arrival comes
-            // with the other producers' after this thread's A row is stored
-            mbar_expect_tx(&full[s], kTileBytes);
-            tma_load_2d(stage + C::NA * kTileBytes, &bmap, kc * kPK, s0, &full[s]);
+            // B tile: one box of 64, 128 or 256 rows, the smallest that
+            // covers the n-tile; expected bytes first, then the copy; the
+            // arrival comes with the other producers' after this thread's A
+            // row is stored
+            mbar_expect_tx(&full[s], (uint32_t)(64 << nb) * kPK * 2);
+            tma_load_2d(stage + kTileBytes, &bmaps.m[nb], kc * kPK, s0, &full[s]);
           }
           // the chunk's codes: code stage gcs of the CTA's sequence, slot kc % CPC
           const int gcs = ui * CSU + kc / CPC, slot = kc - (kc / CPC) * CPC;
           const int ci = gcs % C::CSN;
           mbar_wait_guarded(&cfull[ci], (gcs / C::CSN) & 1, status, abort_flag);
           const uint8_t* cst = cstages + ci * C::CSB + r * kPCodeRow;
-#pragma unroll
-          for (int a = 0; a < NA; ++a) {
-            load_chunk_codes<FMT>(ring[q][a], cst + a * kPM * kPCodeRow, r, slot);
-            store_chunk<FMT>(ring[q][a], stage + a * kTileBytes, r, T4);
-          }
+          // code stage rows: gate/up [2 planes][64 rows], down [128 rows]:
+          // row r of the A tile either way
+          load_chunk_codes<FMT>(ring[q][0], cst, r, slot);
+          store_chunk<FMT>(ring[q][0], stage, r, T4);
           // the generic-proxy shared accesses above (A rows written, codes
           // read) before the async-proxy accesses that follow the barriers
           fence_proxy_async_smem();
@@ -460,8 +491,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
     }
   } else if (warp == 13) {
     // ------------------------------------------------ code stages by TMA:
-    // 64 code bytes of each of the unit's 128 weight rows (both planes for
-    // gate/up), in the producers' order, CSN stages ahead
+    // 64 code bytes of each of the unit's 128 A rows (gate/up: 64 rows of
+    // both planes in one box), in the producers' order, CSN stages ahead
     if (elect_one()) {
       int gcs = 0;
       for (int ui = 0; ui < nunits; ++ui) {
@@ -473,9 +504,9 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
           mbar_arrive_expect_tx(&cfull[ci], C::CSB);
           uint8_t* dst = cstages + ci * C::CSB;
           if constexpr (MODE == 0)
-            tma_load_4d(dst, &cmap, cs * kPCodeRow, mt * kPM, 0, e, &cfull[ci]);
+            tma_load_4d(dst, &cmap, cs * kPCodeRow, mt * C::RPU, 0, e, &cfull[ci]);
           else
-            tma_load_3d(dst, &cmap, cs * kPCodeRow, mt * kPM, e, &cfull[ci]);
+            tma_load_3d(dst, &cmap, cs * kPCodeRow, mt * C::RPU, e, &cfull[ci]);
         }
       }
     }
@@ -484,7 +515,6 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
     // ------------------------------------------------ MMA issue: the whole
     // warp runs the loop (converged); one elected lane issues each stage's
     // MMAs in one asm statement, with warp-uniform operands
-    static_assert(kTileBytes / 16 == 1024, "second A tile 1024 descriptor units on");
     static_assert(kPK == 64, "four K16 steps per stage");
     const uint32_t tbase = __shfl_sync(0xffffffffu, tmem_base, 0);
     const uint32_t dhi = smem_desc_k128_hi(1024);
@@ -504,9 +534,8 @@ prefill_gemm_kernel(const __grid_constant__ CUtensorMap bmap,
         __syncwarp();
         tc_fence_after();
         const uint32_t st = smem0 + (uint32_t)(s * C::SB);
-        mma_stage_ss_warp<MODE == 0>(d0, smem_desc_k128_lo(st),
-                                     smem_desc_k128_lo(st + C::NA * kTileBytes), dhi, idesc,
-                                     (uint32_t)(kc > 0));
+        mma_stage_ss_warp(d0, smem_desc_k128_lo(st), smem_desc_k128_lo(st + kTileBytes), dhi,
+                          idesc, (uint32_t)(kc > 0));
         mma_commit_warp(&empty[s]);
       }
       mma_commit_warp(&tfull[a]);
@@ -550,26 +579,32 @@ PrefillWs prefill_ws(int T, int H, int I, int E, int k, int shared_mode) {
   return w;
 }
 
-// The B operand: [rows, cols] fp16, boxes of 64 columns x kPN rows.
-bool make_map(CUtensorMap* map, const void* base, int cols, long long rows) {
+// The B operand: [rows, cols] fp16, boxes of 64 columns x 64, 128 and 256
+// rows (an n-tile loads the smallest box that covers it).
+bool make_bmaps(BMaps* maps, const void* base, int cols, long long rows) {
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)kPN};
-  return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_128B);
+  for (int i = 0; i < 3; ++i) {
+    const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)(64 << i)};
+    if (!make_tmap(&maps->m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+      return false;
+  }
+  return true;
 }
 
-// The weight codes, boxes of kPCodeRow bytes x kPM rows, 64-byte swizzled.
-// Gate/up: [E][2 planes][I rows][H code bytes] (the plane step is the gate
-// -> up plane distance, so one box holds a tile's gate and up rows); down:
-// [E][H rows][I code bytes].
+// The weight codes, boxes of kPCodeRow bytes x 128 rows, 64-byte swizzled.
+// Gate/up: [E][2 planes][I rows][H code bytes], boxes of 64 rows x both
+// planes (the plane step is the gate -> up plane distance, so one box holds
+// a unit's 64 gate rows and the same 64 up rows); down: [E][H rows][I code
+// bytes].
 bool make_code_map(CUtensorMap* map, int mode, const PrefillArgs& a, int E) {
   const Planes PL = plane_offsets(a.fmt, a.H, a.I);
   if (mode == 0) {
     const cuuint64_t row = codes_row_bytes(a.fmt, a.H);
     const cuuint64_t dims[4] = {row, (cuuint64_t)a.I, 2, (cuuint64_t)E};
     const cuuint64_t str[3] = {row, PL.codes[1] - PL.codes[0], a.stride};
-    const cuuint32_t box[4] = {(cuuint32_t)kPCodeRow, (cuuint32_t)kPM, 2, 1};
+    const cuuint32_t box[4] = {(cuuint32_t)kPCodeRow, (cuuint32_t)(kPM / 2), 2, 1};
     return make_tmap(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, a.wbase + PL.codes[0], dims, str, box,
                      CU_TENSOR_MAP_SWIZZLE_64B);
   }
@@ -582,7 +617,7 @@ bool make_code_map(CUtensorMap* map, int mode, const PrefillArgs& a, int E) {
 }
 
 template <int MODE, int FMT>
-cudaError_t launch_gemm(const CUtensorMap& map, const PrefillArgs& a, int E, const NTile* tiles,
+cudaError_t launch_gemm(const BMaps& map, const PrefillArgs& a, int E, const NTile* tiles,
                         const int* count, uint16_t* out, cudaStream_t st) {
   CUtensorMap cmap;
   if (!make_code_map(&cmap, MODE, a, E)) return cudaErrorInvalidValue;
@@ -624,8 +659,8 @@ cudaError_t launch_experts_prefill(const PrefillArgs& a, cudaStream_t st) {
                                                  a.k, (int)P, a.T, a.H, X, a.status);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  CUtensorMap mx, mh;
-  if (!make_map(&mx, X, a.H, P) || !make_map(&mh, h, a.I, P)) return cudaErrorInvalidValue;
+  BMaps mx, mh;
+  if (!make_bmaps(&mx, X, a.H, P) || !make_bmaps(&mh, h, a.I, P)) return cudaErrorInvalidValue;
   if (a.fmt == STRATA_FMT_Q2_32) {
     if ((e = launch_gemm<0, STRATA_FMT_Q2_32>(mx, a, E, tiles, count, h, st)) != cudaSuccess) return e;
     return launch_gemm<1, STRATA_FMT_Q2_32>(mh, a, E, tiles, count, a.y, st);

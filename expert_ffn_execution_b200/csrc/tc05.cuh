@@ -381,41 +381,25 @@ STRATA_DEVFN void mma_half_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_
 // One 64-K shared-memory stage of a prefill tile, issued by a whole converged
 // warp with a single elect.sync: four K16 MMAs (kind::f16, A and B K-major
 // 128-byte-swizzled in shared memory, descriptors sharing the high word
-// d_hi) into the accumulator at d_tmem; with TWO, four more for the second A
-// tile (16 KB after the first) into d_tmem + 128.  Step kk reads A and B at
+// d_hi) into the accumulator at d_tmem.  Step kk reads A and B at
 // a_lo / b_lo + 2 kk (32 bytes further along K); the first step accumulates
 // iff `accumulate` is nonzero, the others always.
-template <bool TWO>
 STRATA_DEVFN void mma_stage_ss_warp(uint32_t d_tmem, uint32_t a_lo, uint32_t b_lo, uint32_t d_hi,
                                     uint32_t idesc, uint32_t accumulate) {
-#define STRATA_MMA_SS(DOFF, AOFF, BOFF, ACC)                                      \
-  "add.u32 d, %0, " #DOFF ";\n\t"                                               \
+#define STRATA_MMA_SS(AOFF, BOFF, ACC)                                            \
   "add.u32 a, %1, " #AOFF ";\n\t"                                               \
   "add.u32 b, %2, " #BOFF ";\n\t"                                               \
   "mov.b64 ad, {a, %3};\n\t"                                                    \
   "mov.b64 bd, {b, %3};\n\t"                                                    \
-  "@e tcgen05.mma.cta_group::1.kind::f16 [d], ad, bd, %4, " ACC ";\n\t"
-  if constexpr (TWO) {
-    asm volatile(
-        "{\n\t.reg .pred e, p;\n\t.reg .b32 d, a, b;\n\t.reg .b64 ad, bd;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        STRATA_MMA_SS(0, 0, 0, "p") STRATA_MMA_SS(128, 1024, 0, "p")
-        STRATA_MMA_SS(0, 2, 2, "1") STRATA_MMA_SS(128, 1026, 2, "1")
-        STRATA_MMA_SS(0, 4, 4, "1") STRATA_MMA_SS(128, 1028, 4, "1")
-        STRATA_MMA_SS(0, 6, 6, "1") STRATA_MMA_SS(128, 1030, 6, "1")
-        "}" ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred e, p;\n\t.reg .b32 d, a, b;\n\t.reg .b64 ad, bd;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        STRATA_MMA_SS(0, 0, 0, "p") STRATA_MMA_SS(0, 2, 2, "1")
-        STRATA_MMA_SS(0, 4, 4, "1") STRATA_MMA_SS(0, 6, 6, "1")
-        "}" ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-  }
+  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %4, " ACC ";\n\t"
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t.reg .b32 a, b;\n\t.reg .b64 ad, bd;\n\t"
+      "setp.ne.b32 p, %5, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      STRATA_MMA_SS(0, 0, "p") STRATA_MMA_SS(2, 2, "1")
+      STRATA_MMA_SS(4, 4, "1") STRATA_MMA_SS(6, 6, "1")
+      "}" ::"r"(d_tmem), "r"(a_lo), "r"(b_lo), "r"(d_hi), "r"(idesc), "r"(accumulate)
+      : "memory");
 #undef STRATA_MMA_SS
 }
 
