@@ -73,7 +73,15 @@ constexpr int kTcACol0 = 64;      // A stage t at columns 64 + 128 t (accumulato
 constexpr int kTcTmemCols = 512;
 constexpr int kTcMaxStages = 16;
 constexpr int kTcSmemBudget = 227 * 1024;
-constexpr int kTcFusedMinStages = 9;  // fewer: run the two-kernel form
+// The fused form runs with at least kTcFusedMinStages shared-memory stages,
+// or with kTcGroups when each CTA has at most kTcFusedFewTiles tiles (its
+// work is then too short for the deeper pipeline of the two-kernel form to
+// repay that form's second launch); else the two kernels run.  Measured on
+// B200: 4-bit experts at H = 2560, T = 4 (6 stages) 60.2 -> 45.9 us fused;
+// H = 4096, T = 1 (3 stages, 7 tiles) 62.5 -> 52.2 us; H = 4096, T = 4
+// (3 stages, 14 tiles) 128.0 -> 134.2 us, so that one stays two kernels.
+constexpr int kTcFusedMinStages = 6;
+constexpr int kTcFusedFewTiles = 8;
 constexpr int kTcMaxGrid = 1024;      // grids the fused tile dealing is checked for
 // Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
 // only after the MMAs of its previous one retired, so with at least as many
@@ -885,8 +893,9 @@ cudaError_t launch_sync_reset(int32_t* sync, int n, cudaStream_t st) {
 bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
   const int maxT = tc_max_tiles(2, Umax, H, I, grid);
   // the dealing counts (two ints per table slot) live in the exchange buffer
+  const int S = tc_stages(2, fmt, NB, H, I, maxT);
   return grid <= kTcMaxGrid && 8 * maxT <= 2 * 64 * 17 * 4 &&
-         tc_stages(2, fmt, NB, H, I, maxT) >= kTcFusedMinStages;
+         (S >= kTcFusedMinStages || (S >= kTcGroups && maxT <= kTcFusedFewTiles));
 }
 
 }  // namespace
