@@ -61,9 +61,9 @@ struct NTile {
   int e, s0, n, pad;
 };
 
-// The B operand's tensor maps, boxes of 64 columns x {64, 128, 256} rows.
+// The B operand's tensor maps, boxes of 64 columns x {64, 128, 192, 256} rows.
 struct BMaps {
-  CUtensorMap m[3];
+  CUtensorMap m[4];
 };
 
 // One unit = one n-tile x one 128-row A tile.  Gate/up: rows 0-63 of the A
@@ -79,7 +79,7 @@ struct PCfg {  // MODE 0: gate/up, 1: down
 };
 
 constexpr int kPXBytes = 4 * 16 * 32 * 2;  // epilogue transpose buffers: 4 warps x [16][32] fp16
-constexpr int kPUBytes = 64 * 17 * 4;      // gate/up epilogue: 64 up rows x 16 columns (+1 pad)
+constexpr int kPUBytes = 2 * 64 * 9 * 4;   // gate/up epilogue exchange: 2 x 64 rows x 8 columns (+1 pad)
 
 // Shared memory from a 1024-byte aligned base: S stages | CSN code stages |
 // barriers (256 B) | the epilogue's transpose buffers | its up-value
@@ -90,36 +90,38 @@ __host__ __device__ inline size_t prefill_smem_bytes() {
   return 1024 + (size_t)C::S * C::SB + (size_t)C::CSN * C::CSB + 256 + kPXBytes + kPUBytes;
 }
 
-// Epilogue store of 16 output columns (tokens c0..c0+15) of one warp's 32
-// rows: v[j] is this lane's row value for token c0 + j.  The values are
-// rounded to fp16 in pairs (an infinity from a finite value sets
+// Epilogue store of NC output columns (tokens c0..c0+NC-1, NC = 8 or 16) of
+// one warp's 32 rows: v[j] is this lane's row value for token c0 + j.  The
+// values are rounded to fp16 in pairs (an infinity from a finite value sets
 // STRATA_DEV_OVERFLOW, as in f16_bits_checked), written token-major into the
-// warp's [16][32] fp16 buffer, and read back as 16-byte pieces, so each lane
-// stores two 16-byte pieces of token rows instead of sixteen 2-byte values.
+// warp's [NC][32] fp16 buffer, and read back as 16-byte pieces, so each lane
+// stores NC / 8 16-byte pieces of token rows instead of NC 2-byte values.
 // out + (size_t)(s0 + c0 + j) * ld + row0 is token c0 + j's row 0 of the
 // warp; only tokens with c0 + j < n are stored.
-STRATA_DEVFN void store_cols_f16(const float (&v)[16], uint16_t* xw, int lane, uint16_t* out,
+template <int NC>
+STRATA_DEVFN void store_cols_f16(const float (&v)[NC], uint16_t* xw, int lane, uint16_t* out,
                                  size_t ld, int s0, int c0, int n, int row0, int32_t* status) {
-  uint32_t pk[8], inf = 0;
+  static_assert(NC == 8 || NC == 16, "8 or 16 columns");
+  uint32_t pk[NC / 2], inf = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < NC / 2; ++i) {
     pk[i] = h2_as_u32(__floats2half2_rn(v[2 * i], v[2 * i + 1]));
     inf |= __vcmpeq2(pk[i] & 0x7fff7fffu, 0x7c007c00u);
   }
   if (inf) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
+    for (int j = 0; j < NC; ++j)
       if (c0 + j < n && isfinite(v[j]) && __hisinf(__float2half_rn(v[j])))
         dev_flag(status, STRATA_DEV_OVERFLOW);
   }
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int i = 0; i < NC / 2; ++i) {
     xw[(2 * i) * 32 + lane] = (uint16_t)(pk[i] & 0xffffu);
     xw[(2 * i + 1) * 32 + lane] = (uint16_t)(pk[i] >> 16);
   }
   __syncwarp();
 #pragma unroll
-  for (int q = 0; q < 2; ++q) {
+  for (int q = 0; q < NC / 8; ++q) {
     const int u = lane + 32 * q, j = u >> 2, part = u & 3;
     if (c0 + j < n) {
       const uint4 val = *reinterpret_cast<const uint4*>(xw + j * 32 + part * 8);
@@ -298,7 +300,7 @@ prefill_gather_kernel(const uint16_t* __restrict__ hidden, const int32_t* __rest
 // ---------------------------------------------------------------- grouped GEMM
 template <int MODE, int FMT>
 __global__ void __launch_bounds__(kPThreads, 1)
-prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64, 128, 256 rows
+prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256 rows
                     const __grid_constant__ CUtensorMap cmap,  // weight codes
                     const uint8_t* __restrict__ wbase,
                     uint64_t stride, int H, int I, const NTile* __restrict__ tiles,
@@ -353,9 +355,7 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64, 128
     tmem_relinquish();
   }
   if (threadIdx.x == 4 * 32) {
-    prefetch_tensormap(&bmaps.m[0]);
-    prefetch_tensormap(&bmaps.m[1]);
-    prefetch_tensormap(&bmaps.m[2]);
+    for (int i = 0; i < 4; ++i) prefetch_tensormap(&bmaps.m[i]);
   }
   if (threadIdx.x == 13 * 32) prefetch_tensormap(&cmap);
   tc_fence_before();
@@ -383,27 +383,34 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64, 128
         tmem_ld16(tb + c0, g);
         tmem_wait_ld();
         if constexpr (MODE == 0) {
-          // lanes 64-127 hold the up rows: they hand their values to the
-          // gate lanes 0-63 of the same rows through shared memory
-          if (warp >= 2) {
+          // Lanes 0-63 hold gate rows, lanes 64-127 the same up rows.  The
+          // gate lanes finish columns 0-7 and the up lanes columns 8-15 of
+          // each pair: each half hands the other 8 of its values to the
+          // partner lane through shared memory (up -> region 0, gate ->
+          // region 1).
+          const int row = m & 63;
+          const bool upl = warp >= 2;
+          float* xo = xu + (upl ? 0 : 64 * 9);
+          const float* xi = xu + (upl ? 64 * 9 : 0);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) xu[(m - 64) * 17 + j] = __uint_as_float(g[j]);
-          }
+          for (int j = 0; j < 8; ++j) xo[row * 9 + j] = __uint_as_float(upl ? g[j] : g[8 + j]);
           named_bar_sync(1, 128);
-          if (warp < 2) {
-            float v[16];
+          float v[8];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = silu_f32(__uint_as_float(g[j])) * xu[m * 17 + j];
-            store_cols_f16(v, xw, lane, out, (size_t)I, tl.s0, c0, tl.n,
-                           mt * C::RPU + warp * 32, status);
+          for (int j = 0; j < 8; ++j) {
+            const float gv = upl ? xi[row * 9 + j] : __uint_as_float(g[j]);
+            const float uv = upl ? __uint_as_float(g[8 + j]) : xi[row * 9 + j];
+            v[j] = silu_f32(gv) * uv;
           }
-          named_bar_sync(1, 128);  // the exchange buffer is reused
+          store_cols_f16<8>(v, xw, lane, out, (size_t)I, tl.s0, c0 + (upl ? 8 : 0), tl.n,
+                            mt * C::RPU + (warp & 1) * 32, status);
+          named_bar_sync(1, 128);  // the exchange buffers are reused
         } else {
           float v[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(g[j]);
-          store_cols_f16(v, xw, lane, out, (size_t)H, tl.s0, c0, tl.n, mt * kPM + warp * 32,
-                         status);
+          store_cols_f16<16>(v, xw, lane, out, (size_t)H, tl.s0, c0, tl.n, mt * kPM + warp * 32,
+                             status);
         }
       }
       tc_fence_before();
@@ -456,17 +463,17 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64, 128
             c_ui = ui;
             const NTile tl = tiles[(blockIdx.x + ui * gridDim.x) / MT];
             s0 = tl.s0;
-            nb = tl.n <= 64 ? 0 : tl.n <= 128 ? 1 : 2;
+            nb = (tl.n + 63) / 64 - 1;  // box of 64 (nb + 1) rows
           }
           const int s = j % C::S;
           mbar_wait_guarded(&empty[s], ((j / C::S) & 1) ^ 1, status, abort_flag);
           uint8_t* stage = smem + s * C::SB;
           if (r == 0) {
-            // B tile: one box of 64, 128 or 256 rows, the smallest that
-            // covers the n-tile; expected bytes first, then the copy; the
-            // arrival comes with the other producers' after this thread's A
-            // row is stored
-            mbar_expect_tx(&full[s], (uint32_t)(64 << nb) * kPK * 2);
+            // B tile: one box of 64, 128, 192 or 256 rows, the smallest
+            // that covers the n-tile; expected bytes first, then the copy;
+            // the arrival comes with the other producers' after this
+            // thread's A row is stored
+            mbar_expect_tx(&full[s], (uint32_t)(64 * (nb + 1)) * kPK * 2);
             tma_load_2d(stage + kTileBytes, &bmaps.m[nb], kc * kPK, s0, &full[s]);
           }
           // the chunk's codes: code stage gcs of the CTA's sequence, slot kc % CPC
@@ -579,13 +586,13 @@ PrefillWs prefill_ws(int T, int H, int I, int E, int k, int shared_mode) {
   return w;
 }
 
-// The B operand: [rows, cols] fp16, boxes of 64 columns x 64, 128 and 256
-// rows (an n-tile loads the smallest box that covers it).
+// The B operand: [rows, cols] fp16, boxes of 64 columns x 64, 128, 192 and
+// 256 rows (an n-tile loads the smallest box that covers it).
 bool make_bmaps(BMaps* maps, const void* base, int cols, long long rows) {
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  for (int i = 0; i < 3; ++i) {
-    const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)(64 << i)};
+  for (int i = 0; i < 4; ++i) {
+    const cuuint32_t box[2] = {(cuuint32_t)kPK, (cuuint32_t)(64 * (i + 1))};
     if (!make_tmap(&maps->m[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, base, dims, strides, box,
                    CU_TENSOR_MAP_SWIZZLE_128B))
       return false;
