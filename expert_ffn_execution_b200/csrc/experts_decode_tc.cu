@@ -83,6 +83,7 @@ constexpr int kTcSmemBudget = 227 * 1024;
 constexpr int kTcFusedMinStages = 6;
 constexpr int kTcFusedFewTiles = 8;
 constexpr int kTcMaxGrid = 1024;      // grids the fused tile dealing is checked for
+constexpr long long kDrainCycles = 40000000;  // about 20 ms: copies in flight at the end
 // Chunk c decodes into TMEM stage c % kTcTS; a group reaches its next chunk
 // only after the MMAs of its previous one retired, so with at least as many
 // stages as groups no waiter runs two phases ahead of a stage's barrier.
@@ -280,6 +281,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   uint64_t* done = tbl_ready + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* issued = const_cast<int*>(abort_flag) + 1;  // producer: chunks, h loads, scale blocks
   TcTile* tbl = reinterpret_cast<TcTile*>(smem + L.tbl);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -310,6 +312,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     mbar_init(tbl_ready, 128);
     mbar_init(done, 1);
     *abort_flag = 0;
+    issued[0] = issued[1] = issued[2] = 0;
     fence_barrier_init();
   }
   if (warp == kTcMmaWarp) {
@@ -389,20 +392,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   if (warp == kTcProdWarp) {
     // ------------------------------------------------ TMA producer
     if (elect_one()) {
-      int gc = 0, bseq = -1, prev_e = -1;
+      int gc = 0, bseq = -1, prev_e = -1, nsc = 0;
+      bool ok = true;  // false once a wait has given up: issue nothing more
+      // the next stage, once free (-1 after a wait gave up)
       auto next_stage = [&](uint32_t tx) {
         const int s = gc % S;
-        mbar_wait_guarded(&empty[s], ((gc / S) & 1) ^ 1, p.status, abort_flag);
+        if (!ok || !mbar_wait_guarded(&empty[s], ((gc / S) & 1) ^ 1, p.status, abort_flag)) {
+          ok = false;
+          return -1;
+        }
         mbar_arrive_expect_tx(&full[s], tx);
         ++gc;
         return s;
       };
       // the expert's h rows [s0, s0 + NB) into the next B buffer
       auto load_h = [&](int e) {
+        if (!ok || !mbar_wait_guarded(&bempty[(bseq + 1) & 1], (((bseq + 1) >> 1) & 1) ^ 1,
+                                      p.status, abort_flag)) {
+          ok = false;
+          return;
+        }
         ++bseq;
         const int b = bseq & 1;
         const int s0 = p.shared_mode ? 0 : p.offsets[e];
-        mbar_wait_guarded(&bempty[b], ((bseq >> 1) & 1) ^ 1, p.status, abort_flag);
         const uint32_t ab = (uint32_t)p.NB * 128u;
         mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
         for (int a = 0; a < I / 64; ++a)
@@ -415,6 +427,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
           const int e = expert_of(u);
           for (int c = 0; c < nchA; ++c) {
             const int s = next_stage(L.codes_bytes + 128u * 16u);
+            if (s < 0) break;
             uint8_t* st = smem + s * L.stage_bytes;
             // gate rows rb*64.. then the same up rows: one box over both
             // planes for the codes, one for the scales
@@ -440,7 +453,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
           const int e = expert_of(u);
           // the tile's scales: rows rb*128.. of the down plane, all of K
           const int sb = ib & 1;
-          mbar_wait_guarded(&sempty[sb], ((ib >> 1) & 1) ^ 1, p.status, abort_flag);
+          if (!ok || !mbar_wait_guarded(&sempty[sb], ((ib >> 1) & 1) ^ 1, p.status, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++nsc;
           const uint32_t sblk = 128u * (uint32_t)scales_row_bytes(FMT, I);
           mbar_arrive_expect_tx(&sfull[sb], sblk);
           bulk_g2s(smem + L.sbuf + sb * L.s_bytes,
@@ -448,7 +465,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
                    &sfull[sb]);
           auto issue_b = [&](int c) {
             const int s = next_stage(L.codes_bytes);
-            tma_load_3d(smem + s * L.stage_bytes, &md, c * CBR, rb * 128, e, &full[s]);
+            if (s >= 0) tma_load_3d(smem + s * L.stage_bytes, &md, c * CBR, rb * 128, e, &full[s]);
           };
           const bool new_h = ib == 0 || e != prev_e;
           if constexpr (MODE == 1) {
@@ -465,14 +482,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
             if (new_h) {
               // the expert's h is complete once each of its gate/up tiles
               // has counted itself; then read it through the async proxy
-              gmem_wait_geq(p.sync + u, tpeA, p.status, abort_flag);
+              if (!gmem_wait_geq(p.sync + u, tpeA, p.status, abort_flag)) ok = false;
               fence_proxy_async_global();
               load_h(e);
             }
           }
           prev_e = e;
         }
+        if (!ok) break;
       }
+      issued[0] = gc;
+      issued[1] = bseq + 1;
+      issued[2] = nsc;
     }
     __syncwarp();
   } else {
@@ -800,6 +821,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
   }
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag && threadIdx.x == kTcProdWarp * 32) {
+    // A wait gave up somewhere, so stages, h blocks or scale blocks may never
+    // have been consumed: before the CTA exits, every copy the producer
+    // started must have landed.  Wait, bounded, for the last phase armed on
+    // each barrier a copy completes.  (Without an abort every such phase
+    // has been waited for by its consumer already.)
+    const int gc = issued[0], nh = issued[1], nsc = issued[2];
+    for (int s = 0; s < S && s < gc; ++s)
+      mbar_wait_bounded(&full[s], ((gc - 1 - s) / S) & 1, p.status, kDrainCycles);
+    for (int b = 0; b < 2 && b < nh; ++b) {
+      const int q = (nh - 1) - (((nh - 1) - b) & 1);  // last h load into buffer b
+      mbar_wait_bounded(&bfull[b], (q >> 1) & 1, p.status, kDrainCycles);
+    }
+    for (int b = 0; b < 2 && b < nsc; ++b) {
+      const int q = (nsc - 1) - (((nsc - 1) - b) & 1);  // last scale block into buffer b
+      mbar_wait_bounded(&sfull[b], (q >> 1) & 1, p.status, kDrainCycles);
+    }
+  }
   if (warp == kTcMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem_base, kTcTmemCols);
@@ -894,7 +933,13 @@ bool tc_fused_fits(int NB, int H, int I, int Umax, int fmt, int grid) {
   const int maxT = tc_max_tiles(2, Umax, H, I, grid);
   // the dealing counts (two ints per table slot) live in the exchange buffer
   const int S = tc_stages(2, fmt, NB, H, I, maxT);
-  return grid <= kTcMaxGrid && 8 * maxT <= 2 * 64 * 17 * 4 &&
+  // The producer issues all of a down tile's chunks before it waits for
+  // that expert's h, and until h is there each decoder group holds at most
+  // one chunk in registers and one in its TMEM stage: the stages and groups
+  // must take every chunk of a down tile, or the producer would wait for a
+  // stage that only the h it has not loaded yet can free.
+  const int nchB = (I + kTcKC - 1) / kTcKC;
+  return grid <= kTcMaxGrid && 8 * maxT <= 2 * 64 * 17 * 4 && S + 2 * kTcGroups >= nchB &&
          (S >= kTcFusedMinStages || (S >= kTcGroups && maxT <= kTcFusedFewTiles));
 }
 
