@@ -53,6 +53,7 @@ constexpr int kPN = 256;       // tokens per n-tile (MMA N <= 256)
 constexpr int kPK = 64;        // K per stage: one 128-byte swizzle row of fp16
 constexpr int kPThreads = 14 * 32;  // 4 epilogue + 8 producer + 1 MMA + 1 code-TMA warps
 constexpr int kPCodeRow = 64;       // code bytes of one weight row per code stage
+constexpr long long kPDrainCycles = 40000000;  // about 20 ms: copies in flight at the end
 constexpr int kTileBytes = kPM * kPK * 2;   // A tile: 16 KB
 constexpr int kBTileBytes = kPN * kPK * 2;  // B tile: 32 KB
 constexpr int kAccCols = 256;              // TMEM columns per accumulator set
@@ -317,9 +318,12 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
   uint64_t* tempty = tfull + 2;
   uint64_t* cfull = tempty + 2;
   uint64_t* cempty = cfull + C::CSN;
-  uint64_t* done = cempty + C::CSN;
+  uint64_t* bfull = cempty + C::CSN;  // B tile copies (count 1: the copy's bytes)
+  uint64_t* done = bfull + C::S;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* cs_issued = const_cast<int*>(abort_flag) + 1;  // code stages the TMA warp started
+  int* b_issued = cs_issued + 1;                      // B copies each producer group started
 
   const int warp = threadIdx.x >> 5;
   const int K = (MODE == 0) ? H : I;
@@ -337,6 +341,7 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
     for (int s = 0; s < C::S; ++s) {
       mbar_init(&full[s], 128);
       mbar_init(&empty[s], 1);
+      mbar_init(&bfull[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
@@ -348,6 +353,8 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
     }
     mbar_init(done, 1);
     *abort_flag = 0;
+    *cs_issued = 0;
+    b_issued[0] = b_issued[1] = 0;
     fence_barrier_init();
   }
   if (warp == 12) {
@@ -451,8 +458,9 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
     };
 #pragma unroll
     for (int s = 0; s < PD; ++s) prefetch(ring[s]);
-    int c_ui = -1, s0 = 0, nb = 0;
-    for (int j0 = pg; j0 < nchunks; j0 += 2 * (PD + 1)) {
+    int c_ui = -1, s0 = 0, nb = 0, nbi = 0;
+    bool ok = true;
+    for (int j0 = pg; j0 < nchunks && ok; j0 += 2 * (PD + 1)) {
 #pragma unroll
       for (int q = 0; q <= PD; ++q) {
         const int j = j0 + 2 * q;
@@ -466,15 +474,17 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
             nb = (tl.n + 63) / 64 - 1;  // box of 64 (nb + 1) rows
           }
           const int s = j % C::S;
-          mbar_wait_guarded(&empty[s], ((j / C::S) & 1) ^ 1, status, abort_flag);
+          if (!mbar_wait_guarded(&empty[s], ((j / C::S) & 1) ^ 1, status, abort_flag)) {
+            ok = false;  // a wait gave up: start no more copies
+            break;
+          }
           uint8_t* stage = smem + s * C::SB;
           if (r == 0) {
             // B tile: one box of 64, 128, 192 or 256 rows, the smallest
-            // that covers the n-tile; expected bytes first, then the copy;
-            // the arrival comes with the other producers' after this
-            // thread's A row is stored
-            mbar_expect_tx(&full[s], (uint32_t)(64 * (nb + 1)) * kPK * 2);
-            tma_load_2d(stage + kTileBytes, &bmaps.m[nb], kc * kPK, s0, &full[s]);
+            // that covers the n-tile, on its own barrier
+            mbar_arrive_expect_tx(&bfull[s], (uint32_t)(64 * (nb + 1)) * kPK * 2);
+            tma_load_2d(stage + kTileBytes, &bmaps.m[nb], kc * kPK, s0, &bfull[s]);
+            ++nbi;
           }
           // the chunk's codes: code stage gcs of the CTA's sequence, slot kc % CPC
           const int gcs = ui * CSU + kc / CPC, slot = kc - (kc / CPC) * CPC;
@@ -496,6 +506,7 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
         }
       }
     }
+    if (r == 0) b_issued[pg] = nbi;
   } else if (warp == 13) {
     // ------------------------------------------------ code stages by TMA:
     // 64 code bytes of each of the unit's 128 A rows (gate/up: 64 rows of
@@ -516,6 +527,7 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
             tma_load_3d(dst, &cmap, cs * kPCodeRow, mt * C::RPU, e, &cfull[ci]);
         }
       }
+      *cs_issued = gcs;
     }
     __syncwarp();
   } else {
@@ -537,7 +549,8 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
       const uint32_t d0 = tbase + a * kAccCols;
       for (int kc = 0; kc < KC && ok; ++kc, ++it_k) {
         const int s = it_k % C::S;
-        ok = mbar_wait_guarded(&full[s], (it_k / C::S) & 1, status, abort_flag);
+        ok = mbar_wait_guarded(&full[s], (it_k / C::S) & 1, status, abort_flag) &&
+             mbar_wait_guarded(&bfull[s], (it_k / C::S) & 1, status, abort_flag);
         __syncwarp();
         tc_fence_after();
         const uint32_t st = smem0 + (uint32_t)(s * C::SB);
@@ -555,6 +568,23 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
   }
   tc_fence_before();
   __syncthreads();
+  if (*abort_flag && threadIdx.x == 13 * 32) {
+    // A wait gave up, so stages and code stages may never have been
+    // consumed: before the CTA exits, every copy must have landed.  B copies
+    // and code copies complete on barriers of their own (count 1), so the
+    // last phase armed on each completes exactly when its copy lands: wait
+    // for those, bounded.  Group g's B copies were chunks g, g + 2, ...
+    for (int g = 0; g < 2; ++g) {
+      const int n = b_issued[g];
+      for (int i = n - 1; i >= 0 && i >= n - C::S / 2; --i) {
+        const int j = g + 2 * i;  // the group's i-th chunk: stage j % S, phase j / S
+        mbar_wait_bounded(&bfull[j % C::S], (j / C::S) & 1, status, kPDrainCycles);
+      }
+    }
+    const int ncs = *cs_issued;
+    for (int c = 0; c < C::CSN && c < ncs; ++c)
+      mbar_wait_bounded(&cfull[c], ((ncs - 1 - c) / C::CSN) & 1, status, kPDrainCycles);
+  }
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * kAccCols);
