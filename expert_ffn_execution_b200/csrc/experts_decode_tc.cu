@@ -407,6 +407,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
       };
       // the expert's h rows [s0, s0 + NB) into the next B buffer
       auto load_h = [&](int e) {
+        // the expert's first sorted row: loaded before the wait, which hides
+        // its latency
+        const int s0 = p.shared_mode ? 0 : p.offsets[e];
         if (!ok || !mbar_wait_guarded(&bempty[(bseq + 1) & 1], (((bseq + 1) >> 1) & 1) ^ 1,
                                       p.status, abort_flag)) {
           ok = false;
@@ -414,7 +417,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
         }
         ++bseq;
         const int b = bseq & 1;
-        const int s0 = p.shared_mode ? 0 : p.offsets[e];
         const uint32_t ab = (uint32_t)p.NB * 128u;
         mbar_arrive_expect_tx(&bfull[b], ab * (uint32_t)(I / 64));
         for (int a = 0; a < I / 64; ++a)

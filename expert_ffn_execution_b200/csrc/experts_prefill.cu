@@ -430,7 +430,7 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
     const Q4Table T4 = q4_table();
     const uint64_t srow = scales_row_bytes(FMT, K);
     constexpr int NA = 1;  // one weight row per thread
-    constexpr int PD = 4;  // scale prefetch depth (chunks of this group)
+    constexpr int PD = 1;  // scale prefetch depth (chunks of this group; 1 measured faster than 2, 4 or 8)
     // this thread's matrix and row offset within the unit: gate/up rows
     // 0-63 gate, 64-127 up; down: rows of H
     const int mat = (MODE == 0) ? (r >> 6) : 2;
