@@ -25,7 +25,8 @@ def _u16(t):
 def _layer(seed, fmt=mi.FMT_Q2, shared=False, E_=E):
     wr = _u16(mi.gen_router(H, E_, seed))
     bias = mi.gen_zipf_bias(E_, 1.1, seed + 1).numpy()
-    d = (0.005, 0.02) if fmt == mi.FMT_Q2 else (0.0005, 0.002)
+    d = {mi.FMT_Q2: (0.005, 0.02), mi.FMT_Q4CB: (0.0005, 0.002),
+         mi.FMT_MXFP4: (2.0**-9, 2.0**-6)}[fmt]
     blobs = mi.gen_experts(fmt, E_, H, I, d, seed + 2).numpy()
     sb = mi.gen_experts(mi.FMT_Q4CB, 1, H, I, (0.0005, 0.002), seed + 3).numpy()[0] if shared else None
     return wr, bias, blobs, sb
@@ -59,7 +60,8 @@ def test_ranges_counts_and_local_ids():
 
 
 @pytest.mark.parametrize("G,T,fmt,shared", [(2, 5, mi.FMT_Q2, False), (3, 4, mi.FMT_Q2, True),
-                                            (4, 1, mi.FMT_Q4CB, False), (1, 3, mi.FMT_Q2, True)])
+                                            (4, 1, mi.FMT_Q4CB, False), (1, 3, mi.FMT_Q2, True),
+                                            (2, 4, mi.FMT_MXFP4, True)])
 def test_in_process_split_equals_single_rank(G, T, fmt, shared):
     wr, bias, blobs, sb = _layer(100 + G, fmt, shared)
     xs = [mi.gen_x(T, H, 200 + r) for r in range(G)]
