@@ -36,7 +36,8 @@
 //      launched just before, so the workspace needs no initial contents.
 //   0, 1  gate/up alone, then down alone (chained by programmatic dependent
 //      launch): used when the fused form's shared memory leaves too few
-//      stages.
+//      stages, or too few to hold a down tile's chunks in flight, and when
+//      the cooperative launch of the fused grid is refused.
 // Every CTA of a fused grid is resident at once (one per SM, grid <= SMs),
 // and a CTA's gate/up tiles depend on nothing outside it, so the waits on the
 // counters always end; they are bounded all the same.

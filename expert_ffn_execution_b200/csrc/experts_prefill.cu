@@ -29,7 +29,7 @@
 //   warps 4-11 producers, two groups of four warps taking alternate K chunks
 //              (stages); one weight row per thread; the row's codes come
 //              from a code stage in shared memory, its scales are
-//              prefetched a few chunks ahead in registers; decoded to fp16
+//              prefetched a chunk ahead in registers; decoded to fp16
 //              and stored into the 128-byte-swizzled K-major stage layout;
 //              thread 0 of a group also issues the TMA load of the B tile
 //   warp 12    tensor memory allocation and the MMA issue (one elected lane)
@@ -183,7 +183,7 @@ __host__ __device__ constexpr int p_chunks_per_cs() {
 }
 
 // The chunk's two block scales (fp16 pairs, or two E8M0 bytes), from global
-// memory a few chunks ahead of use.
+// memory ahead of use (PD chunks of the group).
 template <int FMT>
 STRATA_DEVFN void load_chunk_scales(PChunk<FMT>& r, const uint8_t* scales_row, int kc) {
   r.s = FMT == STRATA_FMT_MXFP4_32 ? ld_keep_u16(scales_row + kc * 2)

@@ -249,7 +249,9 @@ STRATA_API int32_t moe_route(const float* x, int32_t T, int32_t H, float eps,
  *      path, tcgen05 grouped GEMM over dequantised fp16 tiles).
  *   offsets/perm/active: as written by moe_bucket for the same (T, k, E).
  * Limits: H, I multiples of 128; w->num_experts = E as given to moe_bucket;
- * decode: H a multiple of 256, else STRATA_EUNSUPPORTED.
+ * decode: H a multiple of 256 (512 for MXFP4_32), else STRATA_EUNSUPPORTED;
+ * prefill: every code row at least 64 bytes (H and I >= 256 for Q2_32,
+ * >= 128 for the 4-bit formats), else STRATA_EUNSUPPORTED.
  * Concurrency (decode path): the fused kernel runs one CTA per SM and its
  * down tiles wait for gate/up tiles of other CTAs, so all its CTAs must be
  * resident together.  Do not run decode moe_experts calls concurrently with
