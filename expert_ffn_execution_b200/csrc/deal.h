@@ -94,4 +94,16 @@ STRATA_HD inline int tc_deal_down_tile_counted(const TcDeal& d, const int* gt_al
   return d.ntB - 1 - jp;
 }
 
+// Barrier phase bookkeeping of the drains that follow an abort.  Items
+// 0..n-1 (chunks, copies) use the slots of a ring of `ring` barriers in
+// turn: item i arms slot i % ring in its phase i / ring.  The parity of the
+// last phase armed on slot s (s < min(n, ring)):
+STRATA_HD inline int last_armed_parity(int n, int ring, int s) {
+  return ((n - 1 - s) / ring) & 1;
+}
+
+// The last of items 0..n-1 that used buffer b of a double buffer (item i
+// uses buffer i & 1), for b < min(n, 2).
+STRATA_HD inline int last_item_of_buffer(int n, int b) { return (n - 1) - (((n - 1) - b) & 1); }
+
 }  // namespace strata

@@ -832,15 +832,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     // has been waited for by its consumer already.)
     const int gc = issued[0], nh = issued[1], nsc = issued[2];
     for (int s = 0; s < S && s < gc; ++s)
-      mbar_wait_bounded(&full[s], ((gc - 1 - s) / S) & 1, p.status, kDrainCycles);
-    for (int b = 0; b < 2 && b < nh; ++b) {
-      const int q = (nh - 1) - (((nh - 1) - b) & 1);  // last h load into buffer b
-      mbar_wait_bounded(&bfull[b], (q >> 1) & 1, p.status, kDrainCycles);
-    }
-    for (int b = 0; b < 2 && b < nsc; ++b) {
-      const int q = (nsc - 1) - (((nsc - 1) - b) & 1);  // last scale block into buffer b
-      mbar_wait_bounded(&sfull[b], (q >> 1) & 1, p.status, kDrainCycles);
-    }
+      mbar_wait_bounded(&full[s], last_armed_parity(gc, S, s), p.status, kDrainCycles);
+    for (int b = 0; b < 2 && b < nh; ++b)  // h loads: double buffer, phase = load / 2
+      mbar_wait_bounded(&bfull[b], (last_item_of_buffer(nh, b) >> 1) & 1, p.status, kDrainCycles);
+    for (int b = 0; b < 2 && b < nsc; ++b)  // scale blocks: the same
+      mbar_wait_bounded(&sfull[b], (last_item_of_buffer(nsc, b) >> 1) & 1, p.status,
+                        kDrainCycles);
   }
   if (warp == kTcMmaWarp) {
     tc_fence_after();

@@ -42,6 +42,7 @@
 // (clock budget) and reports STRATA_DEV_TIMEOUT instead of hanging.
 #include <algorithm>
 
+#include "deal.h"
 #include "routing.cuh"
 #include "tc05.cuh"
 #include "tmap.h"
@@ -583,7 +584,7 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
     }
     const int ncs = *cs_issued;
     for (int c = 0; c < C::CSN && c < ncs; ++c)
-      mbar_wait_bounded(&cfull[c], ((ncs - 1 - c) / C::CSN) & 1, status, kPDrainCycles);
+      mbar_wait_bounded(&cfull[c], last_armed_parity(ncs, C::CSN, c), status, kPDrainCycles);
   }
   if (warp == 12) {
     tc_fence_after();

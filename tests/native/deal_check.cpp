@@ -5,7 +5,8 @@
 // weighted work within one down tile (inside it, none gets a down tile), and
 // no CTA gets more tiles than the
 // table capacity computed for any larger expert count, and the per-round-count
-// form of the down-tile index agrees with the direct one.  Prints "ok <cases>" or the first
+// form of the down-tile index agrees with the direct one; and the abort drains'
+// barrier phase bookkeeping.  Prints "ok <cases>" or the first
 // failure, and exits non-zero on a failure.
 #include <cstdio>
 #include <vector>
@@ -81,7 +82,34 @@ static int check(int G, int U, int Umax, int H, int I) {
   return 0;
 }
 
+// The drains' phase bookkeeping against a direct replay of the arming order.
+static int check_drain_phases() {
+  for (int ring = 1; ring <= 16; ++ring)
+    for (int n = 1; n <= 80; ++n)
+      for (int s = 0; s < ring && s < n; ++s) {
+        int last = -1;
+        for (int i = 0; i < n; ++i)
+          if (i % ring == s) last = i;
+        if (last_armed_parity(n, ring, s) != ((last / ring) & 1)) {
+          std::printf("FAIL last_armed_parity n=%d ring=%d s=%d\n", n, ring, s);
+          return 1;
+        }
+      }
+  for (int n = 1; n <= 80; ++n)
+    for (int b = 0; b < 2 && b < n; ++b) {
+      int last = -1;
+      for (int i = 0; i < n; ++i)
+        if ((i & 1) == b) last = i;
+      if (last_item_of_buffer(n, b) != last) {
+        std::printf("FAIL last_item_of_buffer n=%d b=%d\n", n, b);
+        return 1;
+      }
+    }
+  return 0;
+}
+
 int main() {
+  if (check_drain_phases()) return 1;
   const int shapes[][2] = {{2560, 640}, {256, 128}, {512, 256}, {512, 384}, {4096, 1024},
                            {4096, 2048}, {2048, 1408}, {7168, 2048}};
   const int grids[] = {1, 2, 3, 7, 64, 132, 148, 160, 1024};
