@@ -50,16 +50,6 @@ STRATA_DEVFN uint16_t float_to_bf16_bits(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
-// ---------------------------------------------------------------- mma.sync
-// D[16x8] += A[16x16] * B[16x8], fp16 inputs, fp32 accumulate.
-STRATA_DEVFN void mma_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
-      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
 STRATA_DEVFN float silu_f32(float g) { return g / (1.0f + expf(-g)); }
 
 STRATA_DEVFN float warp_sum(float v) {
@@ -90,7 +80,6 @@ STRATA_DEVFN void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-
 
 STRATA_DEVFN void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
@@ -133,7 +122,6 @@ STRATA_DEVFN bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-
 
 // ldmatrix x4, transposed (four 8x8 b16 tiles).
 STRATA_DEVFN void ldsm_x4_trans(uint32_t (&r)[4], const void* p) {

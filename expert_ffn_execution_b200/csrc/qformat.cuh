@@ -7,12 +7,13 @@
 // gate codes|scales, up codes|scales, down codes|scales, each plane on a
 // 256-byte boundary.
 //
-// Register-level decode for the mma.sync decode path.  A "group" is 16
-// consecutive K elements of one row.  Decoding a group yields eight fp16x2
-// registers R[0..7]; R[i] holds the elements (pi(2i), pi(2i+1)) of the group,
-// where pi is a fixed permutation chosen per format to minimise instructions:
-//   Q2_32  : pi(2i) = i, pi(2i+1) = i + 8  (pairs (0,8), (1,9), ...)
-//   Q4CB_32: identity                      (pairs (0,1), (2,3), ...)
+// Register-level decode of the decode path (and the format helpers both
+// expert kernels use).  A "group" is 16 consecutive K elements of one row.
+// Decoding a group yields eight fp16x2 registers R[0..7]; R[i] holds the
+// elements (pi(2i), pi(2i+1)) of the group, where pi is a fixed permutation
+// chosen per format to minimise instructions:
+//   Q2_32            : pi(2i) = i, pi(2i+1) = i + 8  (pairs (0,8), (1,9), ...)
+//   Q4CB_32, MXFP4_32: identity                      (pairs (0,1), (2,3), ...)
 // The activation operand is stored with the same permutation, so the dot
 // product over a group is unchanged.
 #pragma once
@@ -56,30 +57,6 @@ template <int FMT>
 __host__ __device__ inline int group_slot(int e) {
   if (FMT == STRATA_FMT_Q2_32) return e < 8 ? 2 * e : 2 * (e - 8) + 1;
   return e;
-}
-
-// ---------------------------------------------------------------- Q2_32
-// Element j of the 32-bit word sits at bits 2j.  Putting a code at mantissa
-// bit p of an fp16 whose exponent gives that bit unit weight yields
-// M_p + c exactly (M_p = 2^(10-p)); subtracting M_p + 1.5 gives c - 1.5
-// exactly; one multiply by the block scale rounds once to the nearest fp16.
-STRATA_DEVFN void dq_q2_group(uint32_t w, __half2 d2, uint32_t (&R)[8]) {
-  const uint32_t m2 = 0x000C000Cu, m4 = 0x00300030u, m6 = 0x00C000C0u, m8 = 0x03000300u;
-  const uint32_t M2 = 0x5C005C00u, M4 = 0x54005400u, M6 = 0x4C004C00u, M8 = 0x44004400u;
-  const __half2 S2 = u32_as_h2(0x5C065C06u);  // 257.5
-  const __half2 S4 = u32_as_h2(0x54185418u);  // 65.5
-  const __half2 S6 = u32_as_h2(0x4C604C60u);  // 17.5
-  const __half2 S8 = u32_as_h2(0x45804580u);  // 5.5
-  const uint32_t wl = w << 2;   // element 0 -> bit 2, element 8 -> bit 18
-  const uint32_t wr = w >> 8;   // elements 5,6,7 -> bits 2,4,6; 13,14,15 -> 18,20,22
-  R[0] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wl & m2) | M2), S2), d2));
-  R[1] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m2) | M2), S2), d2));
-  R[2] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m4) | M4), S4), d2));
-  R[3] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m6) | M6), S6), d2));
-  R[4] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((w & m8) | M8), S8), d2));
-  R[5] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wr & m2) | M2), S2), d2));
-  R[6] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wr & m4) | M4), S4), d2));
-  R[7] = h2_as_u32(__hmul2(__hsub2(u32_as_h2((wr & m6) | M6), S6), d2));
 }
 
 // ---------------------------------------------------------------- Q4CB_32

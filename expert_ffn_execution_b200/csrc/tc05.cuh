@@ -80,13 +80,6 @@ STRATA_DEVFN void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
-// Add expected transaction bytes to the current phase without arriving.
-STRATA_DEVFN void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)),
-               "r"(bytes)
-               : "memory");
-}
-
 STRATA_DEVFN void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
@@ -129,65 +122,6 @@ STRATA_DEVFN void tma_load_4d(void* dst, const CUtensorMap* map, int c0, int c1,
       : "memory");
 }
 
-// Warp-converged forms of the copy issue: every lane of a converged warp
-// executes the statement and elect.sync picks the one lane that issues, so
-// the warp-uniform operands stay in uniform registers (a lone thread in a
-// divergent branch pays a register move per operand per instruction).  The
-// stage forms arrive on the barrier with the expected bytes and issue the
-// copy in the same statement.
-// One 4-D box at (x, y, w, z).
-STRATA_DEVFN void tma_stage1_4d_warp(uint64_t* bar, uint32_t tx, void* d, const CUtensorMap* m,
-                                     int x, int y, int w, int z) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t"
-      "@e cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%2], [%3, {%4, %5, %6, %7}], [%0];\n\t}" ::"r"(smem_addr(bar)),
-      "r"(tx), "r"(smem_addr(d)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(w),
-      "r"(z)
-      : "memory");
-}
-// One 3-D box at (x, y, z).
-STRATA_DEVFN void tma_stage1_3d_warp(uint64_t* bar, uint32_t tx, void* d, const CUtensorMap* m,
-                                     int x, int y, int z) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t"
-      "@e cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%2], [%3, {%4, %5, %6}], [%0];\n\t}" ::"r"(smem_addr(bar)),
-      "r"(tx), "r"(smem_addr(d)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y), "r"(z)
-      : "memory");
-}
-STRATA_DEVFN void tma_load_2d_warp(void* dst, const CUtensorMap* map, int c0, int c1,
-                                   uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
-      "[%0], [%1, {%2, %3}], [%4];\n\t}" ::"r"(smem_addr(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_addr(bar))
-      : "memory");
-}
-STRATA_DEVFN void mbar_arrive_expect_tx_warp(uint64_t* bar, uint32_t bytes) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_addr(bar)),
-      "r"(bytes)
-      : "memory");
-}
-STRATA_DEVFN void bulk_g2s_warp(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, "
-      "[%3];\n\t}" ::"r"(smem_addr(dst)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar))
-      : "memory");
-}
-
 STRATA_DEVFN void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -225,20 +159,6 @@ STRATA_DEVFN void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 }
 STRATA_DEVFN void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-
-
-STRATA_DEVFN void tmem_ld16_wait(uint32_t a0, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
-      "tcgen05.wait::ld.sync.aligned;"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(a0)
-      : "memory");
-}
-
 STRATA_DEVFN void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -263,24 +183,13 @@ STRATA_DEVFN void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
 STRATA_DEVFN void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------- MMA
-// Shared-memory matrix descriptor, K-major operand in the 128-byte swizzled
-// layout: rows of 128 bytes, 8-row groups 1024 bytes apart (stride byte
-// offset), swizzle mode 128B, descriptor version 1.
-STRATA_DEVFN uint64_t smem_desc_k128(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFF);         // start address
-  d |= (uint64_t)1 << 16;                         // leading byte offset (unused for SW128 K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: 8 rows x 128 B
-  d |= (uint64_t)1 << 46;                         // version
-  d |= (uint64_t)2 << 61;                         // SWIZZLE_128B
-  return d;
-}
-
-// The same descriptor as its two 32-bit words: the low word carries the
-// start address (and the unused leading offset), the high word the stride
-// between 8-row groups, the descriptor version and the swizzle mode.  Start
-// addresses are advanced on the low word alone (shared addresses stay below
-// 256 KiB, so the 14-bit field never carries).
+// Shared-memory matrix descriptor of a K-major operand in the 128-byte
+// swizzled layout (rows of 128 bytes, 8-row groups `sbo` bytes apart,
+// swizzle mode 128B, descriptor version 1), as its two 32-bit words: the low
+// word carries the start address (and the unused leading offset), the high
+// word the stride between 8-row groups, the version and the swizzle mode.
+// Start addresses are advanced on the low word alone (shared addresses stay
+// below 256 KiB, so the 14-bit field never carries).
 STRATA_DEVFN uint32_t smem_desc_k128_lo(uint32_t saddr) {
   return ((saddr >> 4) & 0x3FFFu) | (1u << 16);
 }
@@ -296,18 +205,6 @@ __host__ __device__ inline uint32_t idesc_f16_f32(int n) {
          | ((uint32_t)(n >> 3) << 17)    // N
          | ((uint32_t)(128 >> 4) << 24); // M
 }
-
-STRATA_DEVFN void mma_f16_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                             uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-
 
 // Arrive on `bar` once all previously issued tcgen05 operations of this
 // thread have completed.
@@ -334,48 +231,6 @@ STRATA_DEVFN void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, ui
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], bd, %4, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-// One 128-K half of a decode tile, issued by a whole converged warp with a
-// single elect.sync: eight K16 MMAs (kind::f16, A from tensor memory) into
-// the 16 columns at d_tmem, where step kk reads A at a_tmem + 8 kk and B at
-// b_lo + (kk / 4) ATOM + (kk % 4) * 2 (16-byte units; ATOM = one 64-K atom
-// of B).  The first step accumulates iff `accumulate` is nonzero, the other
-// seven always.  One asm statement keeps the per-MMA work to three adds in
-// the issuing lane.
-template <int ATOM>
-STRATA_DEVFN void mma_half_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi,
-                                   uint32_t idesc, uint32_t accumulate) {
-  static_assert(ATOM == 64 || ATOM == 128, "B atom of 8 or 16 rows");
-#define STRATA_MMA_STEP(AOFF, BOFF, ACC)                                          \
-  "add.u32 a, %1, " #AOFF ";\n\t"                                               \
-  "add.u32 b, %2, " #BOFF ";\n\t"                                               \
-  "mov.b64 bd, {b, %3};\n\t"                                                    \
-  "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a], bd, %4, " ACC ";\n\t"
-  if constexpr (ATOM == 128) {
-    asm volatile(
-        "{\n\t.reg .pred e, p;\n\t.reg .b32 a, b;\n\t.reg .b64 bd;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        STRATA_MMA_STEP(0, 0, "p") STRATA_MMA_STEP(8, 2, "1")
-        STRATA_MMA_STEP(16, 4, "1") STRATA_MMA_STEP(24, 6, "1")
-        STRATA_MMA_STEP(32, 128, "1") STRATA_MMA_STEP(40, 130, "1")
-        STRATA_MMA_STEP(48, 132, "1") STRATA_MMA_STEP(56, 134, "1")
-        "}" ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-  } else {
-    asm volatile(
-        "{\n\t.reg .pred e, p;\n\t.reg .b32 a, b;\n\t.reg .b64 bd;\n\t"
-        "setp.ne.b32 p, %5, 0;\n\t"
-        "elect.sync _|e, 0xffffffff;\n\t"
-        STRATA_MMA_STEP(0, 0, "p") STRATA_MMA_STEP(8, 2, "1")
-        STRATA_MMA_STEP(16, 4, "1") STRATA_MMA_STEP(24, 6, "1")
-        STRATA_MMA_STEP(32, 64, "1") STRATA_MMA_STEP(40, 66, "1")
-        STRATA_MMA_STEP(48, 68, "1") STRATA_MMA_STEP(56, 70, "1")
-        "}" ::"r"(d_tmem), "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(accumulate)
-        : "memory");
-  }
-#undef STRATA_MMA_STEP
 }
 
 // One 64-K shared-memory stage of a prefill tile, issued by a whole converged
