@@ -141,3 +141,24 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch):
     class A:
         config, tokens, layers, warmup, steps = 1, 0, 0, 3, 1
     assert bench.run_reference(A()) is None
+
+
+def test_bench_lines_name_config_tokens_and_layers():
+    """The bench's line list: config:T or config:T:layers; the default ends
+    with the headline (config 1, T = 4) and every decode line streams more
+    weight bytes per step than the 126 MB L2."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import moe_inputs as mi
+    assert bench.parse_lines("2:8192,0:1:48,1:4") == [(2, 8192, None), (0, 1, 48), (1, 4, None)]
+    lines = bench.parse_lines(bench.DEFAULT_LINES)
+    assert lines[-1] == (1, 4, None)
+    for config, T, L in lines:
+        cfg = mi.CONFIGS[config]
+        if T > 16:
+            continue
+        layers = L or cfg.layers
+        # at least one expert per token per layer: k experts of the format's blob size
+        per_step = layers * min(cfg.E, cfg.k * T) * mi.expert_bytes(cfg.fmt, cfg.H, cfg.I)
+        assert per_step > bench.L2_BYTES, (config, T, layers, per_step)
