@@ -162,3 +162,27 @@ def test_bench_lines_name_config_tokens_and_layers():
         # at least one expert per token per layer: k experts of the format's blob size
         per_step = layers * min(cfg.E, cfg.k * T) * mi.expert_bytes(cfg.fmt, cfg.H, cfg.I)
         assert per_step > bench.L2_BYTES, (config, T, layers, per_step)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` (the oracle, on the host cores) prints one
+    JSON line with the arm's keys; a one-layer C0 line keeps it to seconds."""
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "1", "--warmup", "3", "--lines", "0:1:1"],
+                         cwd=ROOT, env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    assert r["impl"] == "reference" and r["unit"] == "tokens/s" and r["higher_is_better"]
+    assert r["value"] > 0 and r["steps"] == 1 and r["warmup"] == 3 and r["n_gpus"] == 1
+    assert r["config"]["T"] == 1 and r["config"]["layers"] == 1
+    cb = r["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == r["value"] and cb["cores"] >= 1
+    assert cb["sample"]
+    assert r["e2e"] == {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert r["ms_per_step"] == pytest.approx(1e3 / r["value"], rel=1e-2)
