@@ -6,11 +6,12 @@ compiled for the host with g++ and checked exhaustively over grid sizes,
 active-expert counts and shapes: every down tile goes to exactly one CTA
 slot, the cut points are monotone, and the tile-table capacity holds.
 
-The synchronisation check runs a model of the fused kernel's barrier
-protocol (tests/native/pipeline_check.cpp) over the same dealing under
-random interleavings: it completes exactly when the in-flight capacity
-condition holds, deadlocks otherwise, and flags a parity hazard for four
-decoder groups on three tensor-memory stages."""
+The synchronisation check runs models of the expert kernels' barrier
+protocols (tests/native/pipeline_check.cpp) under random interleavings: the
+fused decode kernel over the same dealing completes exactly when the
+in-flight capacity condition holds, deadlocks otherwise, and shows a parity
+hazard for four decoder groups on three tensor-memory stages; the prefill
+grouped GEMM completes for both code widths over K sizes and unit counts."""
 import os
 import re
 import shutil
@@ -38,19 +39,34 @@ def _kernel_source():
         return f.read()
 
 
+def _prefill_source():
+    with open(os.path.join(ROOT, "expert_ffn_execution_b200", "csrc",
+                           "experts_prefill.cu")) as f:
+        return f.read()
+
+
 def test_pipeline_model_uses_the_kernels_counts():
-    """The model runs three decoder groups, one tensor-memory stage per
-    group, 256-K chunks and stage counts that are multiples of three up to
-    15; the kernel's constants and its fused-form condition must match."""
+    """The decode model runs three decoder groups, one tensor-memory stage
+    per group, 256-K chunks and stage counts that are multiples of three up
+    to 15; the prefill model four A/B stages, three code stages of 64 code
+    bytes per row (4 chunks of 2-bit codes, 2 of 4-bit), two producer groups
+    each releasing a code stage after its last chunk in it.  The kernels'
+    constants and conditions must match."""
     src = _kernel_source()
     const = dict(re.findall(r"constexpr int (kTc\w+) = (\d+);", src))
     assert const["kTcGroups"] == "3" and const["kTcTS"] == "3"
     assert const["kTcKC"] == "256" and const["kTcMaxStages"] == "16"
     assert "S + 2 * kTcGroups >= nchB" in src
+    pre = _prefill_source()
+    assert "static constexpr int S = 4;" in pre and "static constexpr int CSN = 3;" in pre
+    assert "constexpr int kPCodeRow = 64;" in pre and "constexpr int kPK = 64;" in pre
+    assert "return FMT == STRATA_FMT_Q2_32 ? 16 : 32;" in pre
+    assert "mbar_init(&cempty[c], 256);" in pre and "mbar_init(&full[s], 128);" in pre
+    assert "if (slot + 2 >= in_cs) mbar_arrive(&cempty[ci]);" in pre
 
 
 @pytest.mark.skipif(shutil.which("g++") is None, reason="needs g++")
-def test_fused_pipeline_model_completes_exactly_within_capacity(tmp_path):
+def test_pipeline_models_complete_exactly_within_capacity(tmp_path):
     exe = tmp_path / "pipeline_check"
     src = os.path.join(ROOT, "tests", "native", "pipeline_check.cpp")
     inc = os.path.join(ROOT, "expert_ffn_execution_b200", "csrc")
