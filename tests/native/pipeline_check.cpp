@@ -1,6 +1,7 @@
-// Executable models of the expert kernels' synchronisation: the fused decode
-// kernel (decode_tc_kernel in its MODE 2 form: gate/up tiles, then down
-// tiles, in one grid) and the prefill grouped GEMM (prefill_gemm_kernel).
+// Executable models of the expert kernels' synchronisation: the decode
+// kernel (decode_tc_kernel: its fused form, gate/up tiles then down tiles in
+// one grid, and its two-kernel form) and the prefill grouped GEMM
+// (prefill_gemm_kernel).
 //
 // Every role of every CTA is an actor running the sequence of barrier
 // operations that the kernel's code for that role unfolds to.  Copies land,
@@ -49,12 +50,18 @@
 //              commit the accumulator
 //   epilogue   per unit: wait for the accumulator, release it
 //
+// The decode kernel's two-kernel form runs the same roles over gate/up tiles
+// alone (round robin, no counters), then down tiles alone (a contiguous
+// range; h comes from the grid before, and the first tile's chunks up to the
+// stage count go out before its h copy).
+//
 // main() checks the decode model, for many shapes, grids and active-expert
-// counts, with the kernel's group and stage counts: every run completes
+// counts, with the kernel's group and stage counts: every fused run completes
 // exactly when stages + 2 x groups >= chunks per down tile (the fused form's
-// in-flight capacity condition) and deadlocks otherwise; four decoder groups
-// sharing three tensor-memory stages is flagged as a hazard.  It checks the
-// prefill model complete for both code widths over K sizes and unit counts.
+// in-flight capacity condition) and deadlocks otherwise; every run of both
+// grids of the two-kernel form completes; four decoder groups sharing three
+// tensor-memory stages is flagged as a hazard.  It checks the prefill model
+// complete for both code widths over K sizes and unit counts.
 // Prints "ok <runs>" or the first failure and exits non-zero on a failure.
 #include <algorithm>
 #include <cstdio>
@@ -278,13 +285,14 @@ struct Sim {
 // ---------------------------------------------------------------- fused decode
 struct DecodeParams {
   int G, U, H, I, S, groups, TS, KC;
+  int mode;  // 2 fused; 0 gate/up alone, 1 down alone (h from the grid before)
 };
 
 void build_decode(Sim& m, const DecodeParams& p) {
   const int nchA = p.H / p.KC, nchB = (p.I + p.KC - 1) / p.KC;
   const int tpeA = p.I / 64, tpeB = p.H / 128;
   m.counter.assign(p.U, 0);
-  m.counter_final.assign(p.U, tpeA);
+  m.counter_final.assign(p.U, p.mode == 2 ? tpeA : 0);
   const TcDeal d = tc_deal(p.G, p.U, p.H, p.I);
   std::vector<int> bcnt(p.G);
   for (int c = 0; c < p.G; ++c) bcnt[c] = tc_deal_bstart(d, c + 1) - tc_deal_bstart(d, c);
@@ -302,12 +310,23 @@ void build_decode(Sim& m, const DecodeParams& p) {
     const auto sfull = ring("sfull", 2, 1), sempty = ring("sempty", 2, p.groups);
     const auto bfull = ring("bfull", 2, 1), bempty = ring("bempty", 2, 1);
 
-    // the CTA's tiles: (gate/up?, active expert)
+      // the CTA's tiles: (gate/up?, active expert).  Fused: the dealing;
+    // gate/up alone: round robin; down alone: a contiguous range.
     std::vector<std::pair<bool, int>> tiles;
-    const int nA = d.q + (cta < d.r ? 1 : 0);
-    for (int i = 0; i < nA; ++i) tiles.push_back({true, (cta + i * p.G) / tpeA});
-    for (int kk = 0; kk < bcnt[cta]; ++kk)
-      tiles.push_back({false, tc_deal_down_tile(d, bcnt.data(), cta, kk) / tpeB});
+    int nA = 0;
+    if (p.mode == 2) {
+      nA = d.q + (cta < d.r ? 1 : 0);
+      for (int i = 0; i < nA; ++i) tiles.push_back({true, (cta + i * p.G) / tpeA});
+      for (int kk = 0; kk < bcnt[cta]; ++kk)
+        tiles.push_back({false, tc_deal_down_tile(d, bcnt.data(), cta, kk) / tpeB});
+    } else if (p.mode == 0) {
+      for (int j = cta; j < d.ntA; j += p.G) tiles.push_back({true, j / tpeA});
+      nA = (int)tiles.size();
+    } else {
+      const int b0 = (int)((long long)d.ntB * cta / p.G);
+      const int b1 = (int)((long long)d.ntB * (cta + 1) / p.G);
+      for (int j = b0; j < b1; ++j) tiles.push_back({false, j / tpeB});
+    }
     const int T = (int)tiles.size();
 
     {
@@ -326,12 +345,24 @@ void build_decode(Sim& m, const DecodeParams& p) {
         const int u = tiles[i].second;
         prog.push_back({WAIT, sempty[ib & 1], (ib >> 1) - 1});
         prog.push_back({COPY, sfull[ib & 1], ib >> 1});
-        for (int c = 0; c < nchB; ++c) chunk();
-        if (ib == 0 || u != prev) {
-          prog.push_back({CWAIT, u, tpeA});
+        auto load_h = [&]() {
           prog.push_back({WAIT, bempty[(bseq + 1) & 1], ((bseq + 1) >> 1) - 1});
           ++bseq;
           prog.push_back({COPY, bfull[bseq & 1], bseq >> 1});
+        };
+        const bool new_h = ib == 0 || u != prev;
+        if (p.mode == 1) {
+          // the first tile's chunks up to the stage count go out before h
+          const int pre = ib == 0 ? std::min(nchB, p.S) : 0;
+          for (int c = 0; c < pre; ++c) chunk();
+          if (new_h) load_h();
+          for (int c = pre; c < nchB; ++c) chunk();
+        } else {
+          for (int c = 0; c < nchB; ++c) chunk();
+          if (new_h) {
+            prog.push_back({CWAIT, u, tpeA});
+            load_h();
+          }
         }
         prev = u;
         ++ib;
@@ -388,7 +419,7 @@ void build_decode(Sim& m, const DecodeParams& p) {
       for (int i = 0; i < T; ++i) {
         prog.push_back({WAIT, afull[i & 1], i >> 1});
         prog.push_back({ARRIVE, aempty[i & 1], i >> 1});
-        if (tiles[i].first) prog.push_back({CADD, tiles[i].second, 1});
+        if (p.mode == 2 && tiles[i].first) prog.push_back({CADD, tiles[i].second, 1});
       }
     }
   }
@@ -488,7 +519,7 @@ int main() {
     for (int G : grids)
       for (int U : actives)
         for (int S = groups; S <= 15; S += groups) {
-          const DecodeParams p{G, U, s[0], s[1], S, groups, TS, KC};
+          const DecodeParams p{G, U, s[0], s[1], S, groups, TS, KC, 2};
           const int nchB = (s[1] + KC - 1) / KC;
           // U >= 1 active experts: some CTA has a down tile
           const bool fits = S + 2 * groups >= nchB;
@@ -509,7 +540,7 @@ int main() {
   {
     bool seen = false;
     for (int k = 0; k < 200 && !seen; ++k) {
-      const DecodeParams p{2, 3, 2560, 640, 12, 4, 3, KC};
+      const DecodeParams p{2, 3, 2560, 640, 12, 4, 3, KC, 2};
       seen = run_decode(p, 77 + k, &why) == HAZARD;
       ++runs;
     }
@@ -519,6 +550,22 @@ int main() {
     }
     std::printf("flagged as expected: %s\n", why.c_str());
   }
+  // The two-kernel form (where the fused one does not fit): both grids
+  // complete for every stage count.
+  for (const auto& s : shapes)
+    for (int G : {1, 3, 8})
+      for (int U : {1, 3, 7})
+        for (int S = groups; S <= 15; S += groups)
+          for (int mode = 0; mode < 2; ++mode) {
+            const DecodeParams p{G, U, s[0], s[1], S, groups, TS, KC, mode};
+            const Outcome o = run_decode(p, 3000017ull * (unsigned long long)runs + 3, &why);
+            ++runs;
+            if (o != COMPLETE) {
+              std::printf("FAIL decode mode %d G=%d U=%d H=%d I=%d S=%d: %s (%s)\n", mode, G, U,
+                          s[0], s[1], S, outcome_name(o), why.c_str());
+              return 1;
+            }
+          }
   // Prefill with the kernel's counts: four A/B stages, three code stages,
   // two producer groups; 4 chunks per code stage for 2-bit codes, 2 for
   // 4-bit; K a multiple of 128 (H and I are).

@@ -10,7 +10,8 @@ The synchronisation check runs models of the expert kernels' barrier
 protocols (tests/native/pipeline_check.cpp) under random interleavings: the
 fused decode kernel over the same dealing completes exactly when the
 in-flight capacity condition holds, deadlocks otherwise, and shows a parity
-hazard for four decoder groups on three tensor-memory stages; the prefill
+hazard for four decoder groups on three tensor-memory stages; both grids of
+the two-kernel decode form complete for every stage count; the prefill
 grouped GEMM completes for both code widths over K sizes and unit counts."""
 import os
 import re
