@@ -12,7 +12,11 @@ fused decode kernel over the same dealing completes exactly when the
 in-flight capacity condition holds, deadlocks otherwise, and shows a parity
 hazard for four decoder groups on three tensor-memory stages; both grids of
 the two-kernel decode form complete for every stage count; the prefill
-grouped GEMM completes for both code widths over K sizes and unit counts."""
+grouped GEMM completes for both code widths over K sizes and unit counts.
+Abort runs (an abort raised at a random step, then the kernels' drains)
+stay clean when a role releases no buffer after any of its waits gave up;
+with the releases as the kernels make them, some abort run starts a copy
+into a buffer whose previous copy is still landing."""
 import os
 import re
 import shutil
@@ -76,3 +80,4 @@ def test_pipeline_models_complete_exactly_within_capacity(tmp_path):
     assert r.returncode == 0, r.stdout + r.stderr
     assert r.stdout.splitlines()[-1].startswith("ok "), r.stdout
     assert "flagged as expected" in r.stdout
+    assert "unguarded releases after an abort" in r.stdout
