@@ -829,7 +829,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap mg,   // gate codes
     // have been consumed: before the CTA exits, every copy the producer
     // started must have landed.  Wait, bounded, for the last phase armed on
     // each barrier a copy completes.  (Without an abort every such phase
-    // has been waited for by its consumer already.)
+    // has been waited for by its consumer already.)  Known gap: the decoders
+    // and the MMA thread carry on past a failed wait and still release their
+    // buffers, so the producer can start a second copy into a buffer whose
+    // copy is still landing, which this accounting does not cover.  Releasing
+    // nothing once a thread's wait has given up closes it.
     const int gc = issued[0], nh = issued[1], nsc = issued[2];
     for (int s = 0; s < S && s < gc; ++s)
       mbar_wait_bounded(&full[s], last_armed_parity(gc, S, s), p.status, kDrainCycles);

@@ -575,6 +575,10 @@ prefill_gemm_kernel(const __grid_constant__ BMaps bmaps,  // B: boxes of 64..256
     // and code copies complete on barriers of their own (count 1), so the
     // last phase armed on each completes exactly when its copy lands: wait
     // for those, bounded.  Group g's B copies were chunks g, g + 2, ...
+    // Known gap: producers release a code stage after a code-stage wait that
+    // gave up, and the MMA warp releases the stage of the chunk in hand after
+    // a stage wait that gave up, so a second copy can start into a buffer
+    // still filling, which this accounting does not cover.
     for (int g = 0; g < 2; ++g) {
       const int n = b_issued[g];
       for (int i = n - 1; i >= 0 && i >= n - C::S / 2; --i) {
